@@ -1,0 +1,153 @@
+/*
+ * Agent Attention forward pass -- plain fp64 CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file; only the tests, the package's smoke check and the CPU
+ * baseline leg of the benchmark use it.  It shares no code, header, table or
+ * helper with the CUDA library.
+ *
+ * What it computes (per batch*head slice "bh"), written as the plain
+ * definition, with no blocking, fusion or reordering:
+ *
+ *   agents   A = adaptive average pool of Q over its grid_h x grid_w token
+ *              grid down to pool_h x pool_w agents.
+ *              [Agent Attention: On the Integration of Softmax and Linear
+ *               Attention (arXiv:2312.08874v3 summary), §4 "Efficiency":
+ *               agents from pooling is the default; §6 Conclusion: A = f(Q).]
+ *              Bin i along an axis of length G cut into P bins covers
+ *              [floor(i*G/P), ceil((i+1)*G/P)); the divisor is the number of
+ *              tokens in the bin (the usual adaptive-pool convention, the
+ *              plainest reading of "pooling").
+ *   aggregate V_A = softmax(A K^T * scale) V        (k x d)
+ *   broadcast O   = softmax(Q A^T * scale) V_A      (N x d)
+ *              [Agent Attention：Transformer计算量太大？试试这个'代理令牌'的
+ *               轻量化方案 (jsqmd.com), §1, two-stage pseudocode: stage one
+ *               aggregates K/V into the agents, stage two lets the queries
+ *               read the agents, both softmaxes scaled by 1/sqrt(d);
+ *               arXiv:2312.08874v3 summary §4 "Agent Attention": agent
+ *               aggregation followed by agent broadcast.]
+ *
+ * Softmax is evaluated as exp(x - max) / sum exp(x - max), two passes per
+ * row, in double precision.  Tokens are row-major on the grid
+ * (n = y*grid_w + x); agent j = py*pool_w + px.
+ *
+ * All arrays are contiguous, row-major, double precision:
+ *   q, k, v, o   [BH][N][d]
+ *   a, va        [BH][n_agents][d]
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* start/end of adaptive bin i when an axis of length g is cut into p bins */
+static int64_t bin_start(int64_t i, int64_t g, int64_t p) { return (i * g) / p; }
+static int64_t bin_end(int64_t i, int64_t g, int64_t p) { return ((i + 1) * g + p - 1) / p; }
+
+void oracle_agent_pool(const double* q, int64_t BH, int64_t N, int64_t d,
+                       int64_t grid_h, int64_t grid_w, int64_t pool_h, int64_t pool_w,
+                       double* a) {
+  (void)N;
+  int64_t n_agents = pool_h * pool_w;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    for (int64_t j = 0; j < n_agents; ++j) {
+      int64_t py = j / pool_w, px = j % pool_w;
+      int64_t y0 = bin_start(py, grid_h, pool_h), y1 = bin_end(py, grid_h, pool_h);
+      int64_t x0 = bin_start(px, grid_w, pool_w), x1 = bin_end(px, grid_w, pool_w);
+      double* out = a + (bh * n_agents + j) * d;
+      for (int64_t c = 0; c < d; ++c) out[c] = 0.0;
+      for (int64_t y = y0; y < y1; ++y)
+        for (int64_t x = x0; x < x1; ++x) {
+          const double* row = q + (bh * N + y * grid_w + x) * d;
+          for (int64_t c = 0; c < d; ++c) out[c] += row[c];
+        }
+      double count = (double)((y1 - y0) * (x1 - x0));
+      for (int64_t c = 0; c < d; ++c) out[c] /= count;
+    }
+  }
+}
+
+/* out[row] = softmax(scale * <x_row, keys_n>)_n  @ vals, for one row x_row.
+ * keys: [n_keys][d], vals: [n_keys][d].  work: n_keys doubles. */
+static void softmax_attend_row(const double* x_row, const double* keys, const double* vals,
+                               int64_t n_keys, int64_t d, double scale, double* work,
+                               double* out) {
+  double mx = -INFINITY;
+  for (int64_t n = 0; n < n_keys; ++n) {
+    double s = 0.0;
+    for (int64_t c = 0; c < d; ++c) s += x_row[c] * keys[n * d + c];
+    s *= scale;
+    work[n] = s;
+    if (s > mx) mx = s;
+  }
+  double total = 0.0;
+  for (int64_t n = 0; n < n_keys; ++n) {
+    work[n] = exp(work[n] - mx);
+    total += work[n];
+  }
+  for (int64_t c = 0; c < d; ++c) out[c] = 0.0;
+  for (int64_t n = 0; n < n_keys; ++n) {
+    double p = work[n] / total;
+    for (int64_t c = 0; c < d; ++c) out[c] += p * vals[n * d + c];
+  }
+}
+
+/* Agent aggregation: va[bh][j] = softmax_n(scale * A_j . K_n) @ V. */
+void oracle_agent_aggregate(const double* a, const double* k, const double* v, int64_t BH,
+                            int64_t N, int64_t d, int64_t n_agents, double scale, double* va) {
+#pragma omp parallel
+  {
+    double* work = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+#pragma omp for collapse(2) schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh)
+      for (int64_t j = 0; j < n_agents; ++j)
+        softmax_attend_row(a + (bh * n_agents + j) * d, k + bh * N * d, v + bh * N * d, N, d,
+                           scale, work, va + (bh * n_agents + j) * d);
+    free(work);
+  }
+}
+
+/* Agent broadcast: o[bh][i] = softmax_j(scale * Q_i . A_j) @ V_A. */
+void oracle_agent_broadcast(const double* q, const double* a, const double* va, int64_t BH,
+                            int64_t N, int64_t d, int64_t n_agents, double scale, double* o) {
+#pragma omp parallel
+  {
+    double* work = (double*)malloc(sizeof(double) * (size_t)(n_agents > 0 ? n_agents : 1));
+#pragma omp for collapse(2) schedule(static)
+    for (int64_t bh = 0; bh < BH; ++bh)
+      for (int64_t i = 0; i < N; ++i)
+        softmax_attend_row(q + (bh * N + i) * d, a + bh * n_agents * d, va + bh * n_agents * d,
+                           n_agents, d, scale, work, o + (bh * N + i) * d);
+    free(work);
+  }
+}
+
+/* Whole forward pass.  If agents_or_null is NULL the agents are pooled from Q
+ * (pool_h x pool_w of them); otherwise agents_or_null is [BH][n_agents][d]
+ * (learnable agents, already expanded over the batch by the caller).
+ * scratch_a and scratch_va must hold BH*n_agents*d doubles each. */
+void oracle_agent_attn(const double* q, const double* k, const double* v,
+                       const double* agents_or_null, int64_t BH, int64_t N, int64_t d,
+                       int64_t grid_h, int64_t grid_w, int64_t pool_h, int64_t pool_w,
+                       int64_t n_agents, double scale, double* scratch_a, double* scratch_va,
+                       double* o) {
+  const double* a = agents_or_null;
+  if (a == NULL) {
+    oracle_agent_pool(q, BH, N, d, grid_h, grid_w, pool_h, pool_w, scratch_a);
+    a = scratch_a;
+  }
+  oracle_agent_aggregate(a, k, v, BH, N, d, n_agents, scale, scratch_va);
+  oracle_agent_broadcast(q, a, scratch_va, BH, N, d, n_agents, scale, o);
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

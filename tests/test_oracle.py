@@ -1,0 +1,234 @@
+"""Pins for the fp64 CPU oracle (no GPU).
+
+The oracle is checked against things that do not come from itself: library
+routines (torch's adaptive average pool and scaled-dot-product attention in
+float64, scipy's softmax), the generalized-linear-attention identity of
+arXiv:2312.08874v3 (summary §4), closed forms, exact invariants, and the
+hand-derived worked examples in ``tests/golden/``.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+import torch.nn.functional as F
+
+import oracle
+from oracle import brute
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
+
+
+def rnd(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def torch_pool(q, gh, gw, ph, pw):
+    """Library adaptive average pool of q [BH, N, d] over the (gh, gw) grid."""
+    t = torch.from_numpy(q).reshape(q.shape[0], gh, gw, q.shape[-1]).permute(0, 3, 1, 2)
+    a = F.adaptive_avg_pool2d(t, (ph, pw))
+    return a.permute(0, 2, 3, 1).reshape(q.shape[0], ph * pw, q.shape[-1]).numpy()
+
+
+def sdpa(q, k, v, scale):
+    """Library scaled-dot-product attention in float64."""
+    return F.scaled_dot_product_attention(torch.from_numpy(q), torch.from_numpy(k),
+                                          torch.from_numpy(v), scale=scale).numpy()
+
+
+# ---------------------------------------------------------------- pooling
+
+@pytest.mark.parametrize("gh,gw,ph,pw", [
+    (8, 8, 2, 2), (14, 14, 7, 7), (56, 56, 7, 7), (13, 5, 5, 3),   # 13/5 and 5/3 overlap
+    (6, 10, 4, 3), (9, 9, 9, 9), (7, 4, 1, 1), (256, 16, 12, 16)])
+def test_pool_matches_library_adaptive_avg_pool(gh, gw, ph, pw):
+    q = rnd((3, gh * gw, 5), seed=gh * 100 + pw)
+    np.testing.assert_allclose(oracle.agent_pool(q, gh, gw, ph, pw),
+                               torch_pool(q, gh, gw, ph, pw), rtol=0, atol=1e-13)
+
+
+def test_pool_integer_grid_256_to_12_overlap():
+    """Q[n] = y*grid_w + x on a 256x256 grid pooled to 12x12: bins are 21 or 22
+    wide and neighbours share a row; compare with the library pool exactly."""
+    g, p = 256, 12
+    y, x = np.meshgrid(np.arange(g), np.arange(g), indexing="ij")
+    q = (y * g + x).reshape(1, g * g, 1).astype(np.float64)
+    a = oracle.agent_pool(q, g, g, p, p)
+    np.testing.assert_allclose(a, torch_pool(q, g, g, p, p), rtol=1e-15, atol=1e-9)
+    # bin of agent (0, 1) along x: [floor(256/12), ceil(512/12)) = [21, 43)
+    assert math.isclose(a[0, 1, 0], np.mean((y * g + x)[0:22, 21:43]), rel_tol=1e-15)
+
+
+# ----------------------------------------------------- whole-pass identities
+
+@pytest.mark.parametrize("seed,gh,gw,ph,pw,d,scale", [
+    (0, 6, 6, 3, 2, 5, 0.45), (1, 4, 8, 2, 2, 8, 1.0), (2, 5, 5, 5, 5, 3, 0.7),
+    (3, 8, 8, 2, 2, 32, 1 / math.sqrt(32)), (4, 3, 7, 2, 3, 4, 2.5)])
+def test_brute_force_generalized_linear_attention(seed, gh, gw, ph, pw, d, scale):
+    """O equals M V with the explicit N x N matrix M = softmax(QA^T s) softmax(AK^T s),
+    whose rows sum to one (arXiv:2312.08874v3 summary §4)."""
+    n = gh * gw
+    q, k, v = (rnd((2, n, d), seed + 10 * i) for i in range(3))
+    o = oracle.agent_attn(q, k, v, gh, gw, ph, pw, scale)
+    a_lib = torch_pool(q, gh, gw, ph, pw)
+    for bh in range(2):
+        o_b, m = brute.agent_attn_brute(q[bh], a_lib[bh], k[bh], v[bh], scale)
+        np.testing.assert_allclose(m.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+        assert (m >= 0).all()
+        np.testing.assert_allclose(o[bh], o_b, rtol=0, atol=1e-12)
+
+
+def test_pool_equal_grid_reduces_to_softmax_attention():
+    """pool = grid: every token is its own agent (A = Q), so aggregation is plain
+    softmax attention SDPA(Q, K, V) and broadcast is SDPA(Q, Q, V_A)."""
+    gh, gw, d, scale = 5, 6, 7, 0.6
+    q, k, v = (rnd((3, gh * gw, d), 40 + i) for i in range(3))
+    a = oracle.agent_pool(q, gh, gw, gh, gw)
+    np.testing.assert_allclose(a, q, rtol=0, atol=1e-15)
+    va = oracle.agent_aggregate(a, k, v, scale)
+    np.testing.assert_allclose(va, sdpa(q, k, v, scale), rtol=0, atol=1e-13)
+    o = oracle.agent_broadcast(q, a, va, scale)
+    np.testing.assert_allclose(o, sdpa(q, q, va, scale), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(oracle.agent_attn(q, k, v, gh, gw, gh, gw, scale), o,
+                               rtol=0, atol=1e-15)
+
+
+def test_single_agent_closed_form():
+    """pool 1x1: A = mean(Q); one agent takes all broadcast weight, so every output
+    row equals softmax(s mean(Q) K^T) V, a one-query SDPA."""
+    gh, gw, d, scale = 6, 5, 8, 0.8
+    q, k, v = (rnd((2, gh * gw, d), 50 + i) for i in range(3))
+    o = oracle.agent_attn(q, k, v, gh, gw, 1, 1, scale)
+    mean_q = q.mean(axis=1, keepdims=True)
+    row = sdpa(mean_q, k, v, scale)                      # [2, 1, d]
+    np.testing.assert_allclose(o, np.broadcast_to(row, o.shape), rtol=0, atol=1e-13)
+
+
+def test_equal_keys_give_mean_of_values():
+    gh, gw, d = 7, 7, 6
+    q, _, v = (rnd((2, gh * gw, d), 60 + i) for i in range(3))
+    k = np.broadcast_to(rnd((2, 1, d), 63), q.shape).copy()
+    o = oracle.agent_attn(q, k, v, gh, gw, 3, 3, 0.9)
+    np.testing.assert_allclose(o, np.broadcast_to(v.mean(axis=1, keepdims=True), o.shape),
+                               rtol=0, atol=1e-13)
+
+
+def test_constant_values_give_constant_output():
+    gh, gw, d = 6, 6, 4
+    q, k, _ = (rnd((2, gh * gw, d), 70 + i, scale=3.0) for i in range(3))
+    c = np.array([1.5, -2.0, 0.25, 7.0])
+    v = np.broadcast_to(c, q.shape).copy()
+    o = oracle.agent_attn(q, k, v, gh, gw, 2, 3, 1.0)
+    np.testing.assert_allclose(o, np.broadcast_to(c, o.shape), rtol=0, atol=1e-12)
+
+
+def test_affine_values_and_key_shift():
+    gh, gw, d, scale = 6, 8, 5, 0.7
+    q, k, v = (rnd((2, gh * gw, d), 80 + i) for i in range(3))
+    o = oracle.agent_attn(q, k, v, gh, gw, 3, 4, scale)
+    alpha, shift = -1.75, rnd((d,), 84)
+    o2 = oracle.agent_attn(q, k, alpha * v + shift, gh, gw, 3, 4, scale)
+    np.testing.assert_allclose(o2, alpha * o + shift, rtol=0, atol=1e-12)
+    u = rnd((d,), 85, scale=5.0)           # the same vector added to every key
+    o3 = oracle.agent_attn(q, k + u, v, gh, gw, 3, 4, scale)
+    np.testing.assert_allclose(o3, o, rtol=0, atol=1e-12)
+
+
+def test_convex_hull_of_values():
+    gh, gw, d = 9, 9, 6
+    q, k, v = (rnd((3, gh * gw, d), 90 + i, scale=2.0) for i in range(3))
+    o = oracle.agent_attn(q, k, v, gh, gw, 3, 3, 1.0)
+    lo, hi = v.min(axis=1, keepdims=True), v.max(axis=1, keepdims=True)
+    assert (o >= lo - 1e-12).all() and (o <= hi + 1e-12).all()
+
+
+def test_joint_permutation_of_keys_and_values():
+    gh, gw, d = 8, 6, 5
+    q, k, v = (rnd((2, gh * gw, d), 100 + i) for i in range(3))
+    perm = np.random.default_rng(103).permutation(gh * gw)
+    o = oracle.agent_attn(q, k, v, gh, gw, 2, 3, 0.8)
+    o_p = oracle.agent_attn(q, k[:, perm], v[:, perm], gh, gw, 2, 3, 0.8)
+    np.testing.assert_allclose(o_p, o, rtol=0, atol=1e-13)
+
+
+def test_learnable_agents_and_agent_permutation():
+    """Externally supplied agents [H, k, d] shared over the batch; the output does
+    not depend on agent order."""
+    B, H, gh, gw, d, n_ag = 2, 3, 5, 6, 8, 7
+    q, k, v = (rnd((B, H, gh * gw, d), 110 + i) for i in range(3))
+    agents = rnd((H, n_ag, d), 113, scale=0.7)
+    o = oracle.agent_attn(q, k, v, gh, gw, 1, 1, 0.5, agents=agents)
+    perm = np.random.default_rng(114).permutation(n_ag)
+    o_p = oracle.agent_attn(q, k, v, gh, gw, 1, 1, 0.5, agents=agents[:, perm])
+    np.testing.assert_allclose(o_p, o, rtol=0, atol=1e-13)
+    # the shared agents equal an explicit per-batch copy, and match the brute force
+    full = np.broadcast_to(agents, (B,) + agents.shape)
+    o_full = oracle.agent_attn(q, k, v, gh, gw, 1, 1, 0.5, agents=full)
+    np.testing.assert_allclose(o_full, o, rtol=0, atol=0)
+    o_b, _ = brute.agent_attn_brute(q[1, 2], agents[2], k[1, 2], v[1, 2], 0.5)
+    np.testing.assert_allclose(o[1, 2], o_b, rtol=0, atol=1e-12)
+
+
+def test_scale_to_zero_gives_mean_of_values():
+    gh, gw, d = 6, 6, 4
+    q, k, v = (rnd((2, gh * gw, d), 120 + i) for i in range(3))
+    o = oracle.agent_attn(q, k, v, gh, gw, 3, 3, 1e-12)
+    np.testing.assert_allclose(o, np.broadcast_to(v.mean(axis=1, keepdims=True), o.shape),
+                               rtol=0, atol=1e-9)
+
+
+@pytest.mark.parametrize("mult", [4.0, 100.0])
+def test_sharp_logits_match_library_softmax(mult):
+    """Scale 1 and inputs x4 or x100 (logits in the thousands): stage outputs match
+    scipy's softmax and stay finite."""
+    gh, gw, d = 6, 6, 8
+    q, k, v = (rnd((2, gh * gw, d), 130 + i, scale=mult) for i in range(3))
+    a = oracle.agent_pool(q, gh, gw, 2, 2)
+    va = oracle.agent_aggregate(a, k, v, 1.0)
+    ref_va = scipy.special.softmax(np.einsum("bjc,bnc->bjn", a, k), axis=-1) @ v
+    np.testing.assert_allclose(va, ref_va, rtol=1e-12, atol=1e-12 * mult)
+    o = oracle.agent_broadcast(q, a, va, 1.0)
+    ref_o = scipy.special.softmax(np.einsum("bnc,bjc->bnj", q, a), axis=-1) @ va
+    np.testing.assert_allclose(o, ref_o, rtol=1e-12, atol=1e-12 * mult)
+    assert np.isfinite(o).all()
+
+
+# ------------------------------------------------------ worked examples
+
+def _eval(x):
+    if isinstance(x, str):
+        return float(eval(x, {"__builtins__": {}}, {"e": math.e, "log": math.log}))
+    return float(x)
+
+
+def _mat(rows):
+    return np.array([[_eval(x) for x in r] for r in rows], dtype=np.float64)
+
+
+def _golden_cases():
+    with open(GOLDEN) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _golden_cases(), ids=lambda c: c["name"])
+def test_hand_derived_worked_examples(case):
+    gh, gw = case["grid"]
+    ph, pw = case["pool"]
+    q, k, v = (_mat(case[n])[None] for n in ("q", "k", "v"))
+    a = oracle.agent_pool(q, gh, gw, ph, pw)
+    np.testing.assert_allclose(a[0], _mat(case["expected_agents"]), rtol=0, atol=1e-14)
+    va = oracle.agent_aggregate(a, k, v, case["scale"])
+    np.testing.assert_allclose(va[0], _mat(case["expected_va"]), rtol=0, atol=1e-13)
+    o = oracle.agent_attn(q, k, v, gh, gw, ph, pw, case["scale"])
+    np.testing.assert_allclose(o[0], _mat(case["expected_o"]), rtol=0, atol=1e-13)
+
+
+def test_oracle_is_fp64_and_deterministic():
+    q, k, v = (rnd((1, 64, 32), 140 + i) for i in range(3))
+    o1 = oracle.agent_attn(q, k, v, 8, 8, 2, 2, 0.2)
+    o2 = oracle.agent_attn(q, k, v, 8, 8, 2, 2, 0.2)
+    assert o1.dtype == np.float64
+    np.testing.assert_array_equal(o1, o2)
