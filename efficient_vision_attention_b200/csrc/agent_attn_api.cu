@@ -1,0 +1,587 @@
+// Host side of the Agent Attention C ABI (include/agent_attn.h): argument
+// validation, scratch layout, kernel selection and launch sequencing.
+//
+// Launch sequence of one forward pass on `stream`:
+//   agent_pool (skipped for learnable agents)
+//   -> agent_aggregate (split over keys; partial U, running max, running sum)
+//   -> agent_merge (log-sum-exp merge of the splits into V_A)
+//   -> agent_broadcast
+// bf16 problems with d <= 64 run the tcgen05/TMA tensor-core kernels for the
+// aggregation and the broadcast; every other problem runs the SIMT kernels.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/agent_attn.h"
+#include "common.cuh"
+#include "kernels_simt.cuh"
+#include "kernels_tc.cuh"
+
+namespace aa {
+namespace {
+
+thread_local char g_cuda_err[384] = "AA_ERR_CUDA: no CUDA error recorded on this thread";
+
+int cuda_fail(cudaError_t e, const char* what) {
+  snprintf(g_cuda_err, sizeof(g_cuda_err), "AA_ERR_CUDA: %s: %s (%s)", what, cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return AA_ERR_CUDA;
+}
+#define AA_CUDA(call)                                   \
+  do {                                                  \
+    cudaError_t _e = (call);                            \
+    if (_e != cudaSuccess) return cuda_fail(_e, #call); \
+  } while (0)
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+int device_sm_count(int* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev >= 0 && dev < kMaxDevices) {
+    int c = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (c > 0) {
+      *out = c;
+      return AA_OK;
+    }
+  }
+  int c = 0;
+  e = cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+  if (dev >= 0 && dev < kMaxDevices) g_sm_count[dev].store(c, std::memory_order_relaxed);
+  *out = c;
+  return AA_OK;
+}
+
+// Library-owned stream-ordered memory pool per device.  Freed scratch stays
+// in the pool (release threshold = max) so that repeated calls do not map and
+// unmap device memory; the pool is created on first use on each device.
+std::atomic<cudaMemPool_t> g_pool[kMaxDevices];
+
+int device_pool(cudaMemPool_t* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) {
+    e = cudaDeviceGetDefaultMemPool(out, dev);
+    return e == cudaSuccess ? AA_OK : cuda_fail(e, "cudaDeviceGetDefaultMemPool");
+  }
+  cudaMemPool_t p = g_pool[dev].load(std::memory_order_acquire);
+  if (p != nullptr) {
+    *out = p;
+    return AA_OK;
+  }
+  cudaMemPoolProps props;
+  memset(&props, 0, sizeof(props));
+  props.allocType = cudaMemAllocationTypePinned;
+  props.handleTypes = cudaMemHandleTypeNone;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  cudaMemPool_t fresh = nullptr;
+  e = cudaMemPoolCreate(&fresh, &props);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
+  unsigned long long keep = ~0ull;
+  e = cudaMemPoolSetAttribute(fresh, cudaMemPoolAttrReleaseThreshold, &keep);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolSetAttribute");
+  cudaMemPool_t expected = nullptr;
+  if (!g_pool[dev].compare_exchange_strong(expected, fresh)) {
+    cudaMemPoolDestroy(fresh);
+    fresh = expected;
+  }
+  *out = fresh;
+  return AA_OK;
+}
+
+int scratch_alloc(void** ptr, size_t bytes, cudaStream_t st) {
+  cudaMemPool_t pool = nullptr;
+  int rc = device_pool(&pool);
+  if (rc != AA_OK) return rc;
+  cudaError_t e = cudaMallocFromPoolAsync(ptr, bytes, pool, st);
+  return e == cudaSuccess ? AA_OK : cuda_fail(e, "cudaMallocFromPoolAsync");
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Problem {
+  int B, H, N, d, k;
+  int grid_h, grid_w, pool_h, pool_w;  // pool_h == 0: learnable agents
+  float scale;
+  int dtype;
+  long long BH() const { return (long long)B * H; }
+  size_t elem() const { return dtype == AA_FP32 ? 4 : 2; }
+};
+
+int validate_common(int B, int H, int N, int d, int k, float scale, int dtype) {
+  if (dtype != AA_FP32 && dtype != AA_BF16) return AA_ERR_UNSUPPORTED;
+  if (B < 1 || H < 1 || N < 1) return AA_ERR_SHAPE;
+  if (d < 8 || d > 128 || (d % 8) != 0) return AA_ERR_UNSUPPORTED;
+  if (k < 1 || k > 256) return AA_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return AA_ERR_VALUE;
+  if ((long long)B * H * (long long)N > (1LL << 40)) return AA_ERR_SHAPE;
+  return AA_OK;
+}
+
+int validate_grid(int N, int grid_h, int grid_w, int pool_h, int pool_w) {
+  if (grid_h < 1 || grid_w < 1 || (long long)grid_h * grid_w != N) return AA_ERR_SHAPE;
+  if (pool_h < 1 || pool_w < 1 || pool_h > grid_h || pool_w > grid_w) return AA_ERR_SHAPE;
+  return AA_OK;
+}
+
+bool use_tensor_cores(const Problem& p) { return p.dtype == AA_BF16 && tc_supported(p.d, p.k); }
+
+// Scratch layout.  Every region starts on a 256-byte boundary.
+struct Scratch {
+  size_t a_off, va_off, pu_off, pml_off, total;
+  SplitPlan plan;
+  int simt_row_blocks;
+  int simt_cols_per_split;
+};
+
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+void plan_scratch(const Problem& p, int sm_count, Scratch* s) {
+  const long long BH = p.BH();
+  memset(s, 0, sizeof(*s));
+  if (use_tensor_cores(p)) {
+    tc_plan_aggregate(BH, p.N, p.k, sm_count, &s->plan);
+  } else {
+    const int row_blocks = (p.k + kSimtRows - 1) / kSimtRows;
+    long long want = (2LL * sm_count + BH * row_blocks - 1) / (BH * row_blocks);
+    const long long max_splits = (p.N + 127) / 128;
+    if (want > max_splits) want = max_splits;
+    if (want < 1) want = 1;
+    int cps = (int)((p.N + want - 1) / want);
+    cps = (cps + kSimtCols - 1) / kSimtCols * kSimtCols;
+    const int splits = (p.N + cps - 1) / cps;
+    s->plan.fixed = splits;
+    s->plan.slots = splits;
+    s->simt_row_blocks = row_blocks;
+    s->simt_cols_per_split = cps;
+  }
+  const size_t agents_bytes = (size_t)BH * p.k * p.d * p.elem();
+  size_t off = 0;
+  s->a_off = off;
+  off += round256(agents_bytes);
+  s->va_off = off;
+  off += round256(agents_bytes);
+  s->pu_off = off;
+  off += round256((size_t)BH * s->plan.slots * p.k * p.d * sizeof(float));
+  s->pml_off = off;
+  off += round256((size_t)BH * s->plan.slots * p.k * 2 * sizeof(float));
+  s->total = off;
+}
+
+template <typename KernelT>
+int ensure_smem(KernelT kernel, size_t bytes, std::atomic<int>* flags) {
+  int dev = 0;
+  AA_CUDA(cudaGetDevice(&dev));
+  if (dev < kMaxDevices && flags[dev].load(std::memory_order_relaxed) >= (int)bytes)
+    return AA_OK;
+  AA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  if (dev < kMaxDevices) flags[dev].store((int)bytes, std::memory_order_relaxed);
+  return AA_OK;
+}
+
+std::atomic<int> g_simt_smem_f32[kMaxDevices];
+std::atomic<int> g_simt_smem_bf16[kMaxDevices];
+
+struct AgentsRef {
+  const void* ptr;
+  long long bstride, hstride;  // elements
+};
+
+template <typename T>
+int launch_pool(const Problem& p, const void* q, float* a_f32, T* a_lowp, cudaStream_t st) {
+  dim3 grid(p.pool_h, (unsigned)p.BH());
+  if (p.BH() > 65535) {
+    // y-dimension limit: launch the slices in chunks
+    for (long long b0 = 0; b0 < p.BH(); b0 += 65535) {
+      const long long nb = (p.BH() - b0 < 65535) ? p.BH() - b0 : 65535;
+      const long long qoff = b0 * (long long)p.N * p.d;
+      const long long aoff = b0 * (long long)p.k * p.d;
+      agent_pool_kernel<T><<<dim3(p.pool_h, (unsigned)nb), 256, 0, st>>>(
+          static_cast<const T*>(q) + qoff, a_f32 ? a_f32 + aoff : nullptr,
+          a_lowp ? a_lowp + aoff : nullptr, p.N, p.d, p.grid_h, p.grid_w, p.pool_h, p.pool_w);
+      AA_CUDA(cudaGetLastError());
+    }
+    return AA_OK;
+  }
+  agent_pool_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(q), a_f32, a_lowp, p.N, p.d,
+                                             p.grid_h, p.grid_w, p.pool_h, p.pool_w);
+  AA_CUDA(cudaGetLastError());
+  return AA_OK;
+}
+
+template <typename T>
+int launch_simt_attend(const SimtAttendArgs& args, long long BH, cudaStream_t st) {
+  const size_t smem = simt_attend_smem_bytes(args.d);
+  int rc = ensure_smem(simt_attend_kernel<T>, smem,
+                       sizeof(T) == 4 ? g_simt_smem_f32 : g_simt_smem_bf16);
+  if (rc != AA_OK) return rc;
+  const long long blocks = BH * args.splits * args.row_blocks;
+  if (blocks > 0x7fffffffLL) return AA_ERR_SHAPE;
+  simt_attend_kernel<T><<<(unsigned)blocks, kSimtThreads, smem, st>>>(args);
+  AA_CUDA(cudaGetLastError());
+  return AA_OK;
+}
+
+template <typename T>
+int launch_merge(const Problem& p, const Scratch& s, char* ws, float* va_f32, T* va_lowp,
+                 cudaStream_t st) {
+  const long long rows = p.BH() * p.k;
+  const long long blocks = (rows + 7) / 8;
+  if (blocks > 0x7fffffffLL) return AA_ERR_SHAPE;
+  agent_merge_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(
+      reinterpret_cast<const float*>(ws + s.pu_off), reinterpret_cast<const float*>(ws + s.pml_off),
+      s.plan, p.BH(), p.k, p.d, va_f32, va_lowp);
+  AA_CUDA(cudaGetLastError());
+  return AA_OK;
+}
+
+// Aggregation + merge.  agents are in the run dtype (fp32 path: float).
+template <typename T>
+int run_aggregate(const Problem& p, const Scratch& s, const AgentsRef& ag, const void* k,
+                  const void* v, char* ws, float* va_f32, T* va_lowp, cudaStream_t st) {
+  const long long qstride_h = (long long)p.N * p.d, qstride_b = qstride_h * p.H;
+  if (use_tensor_cores(p)) {
+    cudaError_t e = tc_launch_aggregate(ag.ptr, ag.bstride, ag.hstride, k, v, p.B, p.H, p.N, p.d,
+                                        p.k, p.scale * kLog2e, s.plan,
+                                        reinterpret_cast<float*>(ws + s.pu_off),
+                                        reinterpret_cast<float*>(ws + s.pml_off), st);
+    if (e != cudaSuccess) return cuda_fail(e, "agent_aggregate (tensor cores) launch");
+  } else {
+    SimtAttendArgs a;
+    memset(&a, 0, sizeof(a));
+    a.rows = ag.ptr;
+    a.rows_bstride = ag.bstride;
+    a.rows_hstride = ag.hstride;
+    a.cols = k;
+    a.cols_bstride = qstride_b;
+    a.cols_hstride = qstride_h;
+    a.vals = v;
+    a.vals_bstride = qstride_b;
+    a.vals_hstride = qstride_h;
+    a.H = p.H;
+    a.n_rows = p.k;
+    a.n_cols = p.N;
+    a.d = p.d;
+    a.scale_log2 = p.scale * kLog2e;
+    a.row_blocks = s.simt_row_blocks;
+    a.splits = s.plan.fixed;
+    a.cols_per_split = s.simt_cols_per_split;
+    a.part_u = reinterpret_cast<float*>(ws + s.pu_off);
+    a.part_ml = reinterpret_cast<float*>(ws + s.pml_off);
+    a.slots = s.plan.slots;
+    int rc = launch_simt_attend<T>(a, p.BH(), st);
+    if (rc != AA_OK) return rc;
+  }
+  return launch_merge<T>(p, s, ws, va_f32, va_lowp, st);
+}
+
+template <typename T>
+int run_broadcast(const Problem& p, const void* q, const AgentsRef& ag, const void* va,
+                  void* out, cudaStream_t st) {
+  const long long qstride_h = (long long)p.N * p.d, qstride_b = qstride_h * p.H;
+  const long long vstride_h = (long long)p.k * p.d, vstride_b = vstride_h * p.H;
+  if (use_tensor_cores(p)) {
+    int sms = 0;
+    int rc = device_sm_count(&sms);
+    if (rc != AA_OK) return rc;
+    cudaError_t e = tc_launch_broadcast(q, ag.ptr, ag.bstride, va, out, p.B, p.H, p.N, p.d, p.k,
+                                        p.scale * kLog2e, sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "agent_broadcast (tensor cores) launch");
+    return AA_OK;
+  }
+  SimtAttendArgs a;
+  memset(&a, 0, sizeof(a));
+  a.rows = q;
+  a.rows_bstride = qstride_b;
+  a.rows_hstride = qstride_h;
+  a.cols = ag.ptr;
+  a.cols_bstride = ag.bstride;
+  a.cols_hstride = ag.hstride;
+  a.vals = va;
+  a.vals_bstride = vstride_b;
+  a.vals_hstride = vstride_h;
+  a.H = p.H;
+  a.n_rows = p.N;
+  a.n_cols = p.k;
+  a.d = p.d;
+  a.scale_log2 = p.scale * kLog2e;
+  a.row_blocks = (p.N + kSimtRows - 1) / kSimtRows;
+  a.splits = 1;
+  a.cols_per_split = p.k;
+  a.out = out;
+  a.out_bstride = qstride_b;
+  a.out_hstride = qstride_h;
+  return launch_simt_attend<T>(a, p.BH(), st);
+}
+
+template <typename T>
+int run_forward(const Problem& p, const Scratch& s, const void* q, const void* k, const void* v,
+                const AgentsRef* learnable, void* out, char* ws, cudaStream_t st) {
+  AgentsRef ag;
+  const long long ahs = (long long)p.k * p.d;
+  if (learnable) {
+    ag = *learnable;
+  } else {
+    T* a_ws = reinterpret_cast<T*>(ws + s.a_off);
+    int rc = (sizeof(T) == 4)
+                 ? launch_pool<T>(p, q, reinterpret_cast<float*>(a_ws), nullptr, st)
+                 : launch_pool<T>(p, q, nullptr, a_ws, st);
+    if (rc != AA_OK) return rc;
+    ag.ptr = a_ws;
+    ag.bstride = ahs * p.H;
+    ag.hstride = ahs;
+  }
+  T* va_ws = reinterpret_cast<T*>(ws + s.va_off);
+  int rc = (sizeof(T) == 4)
+               ? run_aggregate<T>(p, s, ag, k, v, ws, reinterpret_cast<float*>(va_ws), nullptr, st)
+               : run_aggregate<T>(p, s, ag, k, v, ws, nullptr, va_ws, st);
+  if (rc != AA_OK) return rc;
+  return run_broadcast<T>(p, q, ag, va_ws, out, st);
+}
+
+int forward_impl(const Problem& p, const void* q, const void* k, const void* v,
+                 const AgentsRef* learnable, void* out, void* user_ws, size_t user_ws_bytes,
+                 bool have_user_ws, cudaStream_t st) {
+  int sms = 0;
+  int rc = device_sm_count(&sms);
+  if (rc != AA_OK) return rc;
+  Scratch s;
+  plan_scratch(p, sms, &s);
+  char* ws = nullptr;
+  bool owned = false;
+  if (have_user_ws) {
+    if (user_ws == nullptr) return AA_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(user_ws) & 255u) != 0) return AA_ERR_ALIGN;
+    if (user_ws_bytes < s.total) return AA_ERR_WORKSPACE;
+    ws = static_cast<char*>(user_ws);
+  } else {
+    rc = scratch_alloc(reinterpret_cast<void**>(&ws), s.total, st);
+    if (rc != AA_OK) return rc;
+    owned = true;
+  }
+  rc = (p.dtype == AA_FP32)
+           ? run_forward<float>(p, s, q, k, v, learnable, out, ws, st)
+           : run_forward<__nv_bfloat16>(p, s, q, k, v, learnable, out, ws, st);
+  if (owned) {
+    cudaError_t e = cudaFreeAsync(ws, st);
+    if (rc == AA_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
+  }
+  return rc;
+}
+
+int check_tensor_ptrs(const void* q, const void* k, const void* v, const void* out) {
+  if (!q || !k || !v || !out) return AA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return AA_ERR_ALIGN;
+  return AA_OK;
+}
+
+int pooled_forward(const void* q, const void* k, const void* v, const void* agents_or_null,
+                   void* out, int B, int H, int N, int d, int grid_h, int grid_w, int pool_h,
+                   int pool_w, float scale, int dtype, void* ws, size_t ws_bytes, bool have_ws,
+                   void* stream) {
+  int rc = validate_grid(N, grid_h, grid_w, pool_h, pool_w);
+  if (rc != AA_OK) return rc;
+  const int kk = pool_h * pool_w;
+  rc = validate_common(B, H, N, d, kk, scale, dtype);
+  if (rc != AA_OK) return rc;
+  rc = check_tensor_ptrs(q, k, v, out);
+  if (rc != AA_OK) return rc;
+  if (agents_or_null && !aligned16(agents_or_null)) return AA_ERR_ALIGN;
+  Problem p{B, H, N, d, kk, grid_h, grid_w, pool_h, pool_w, scale, dtype};
+  AgentsRef learn{agents_or_null, 0, (long long)kk * d};
+  return forward_impl(p, q, k, v, agents_or_null ? &learn : nullptr, out, ws, ws_bytes, have_ws,
+                      static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+}  // namespace aa
+
+using namespace aa;
+
+extern "C" {
+
+int agent_attn_forward(const void* q, const void* k, const void* v, const void* agents_or_null,
+                       void* out, int B, int H, int N, int d, int grid_h, int grid_w, int pool_h,
+                       int pool_w, float scale, int dtype, void* stream) {
+  return pooled_forward(q, k, v, agents_or_null, out, B, H, N, d, grid_h, grid_w, pool_h, pool_w,
+                        scale, dtype, nullptr, 0, false, stream);
+}
+
+int agent_attn_forward_ws(const void* q, const void* k, const void* v, const void* agents_or_null,
+                          void* out, int B, int H, int N, int d, int grid_h, int grid_w,
+                          int pool_h, int pool_w, float scale, int dtype, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  return pooled_forward(q, k, v, agents_or_null, out, B, H, N, d, grid_h, grid_w, pool_h, pool_w,
+                        scale, dtype, workspace, ws_bytes, true, stream);
+}
+
+int agent_attn_forward_agents(const void* q, const void* k, const void* v, const void* agents,
+                              int n_agents, long long agents_batch_stride, void* out, int B,
+                              int H, int N, int d, float scale, int dtype, void* stream) {
+  int rc = validate_common(B, H, N, d, n_agents, scale, dtype);
+  if (rc != AA_OK) return rc;
+  rc = check_tensor_ptrs(q, k, v, out);
+  if (rc != AA_OK) return rc;
+  if (!agents) return AA_ERR_NULL;
+  if (!aligned16(agents)) return AA_ERR_ALIGN;
+  if (agents_batch_stride < 0 || (agents_batch_stride % 8) != 0) return AA_ERR_ALIGN;
+  Problem p{B, H, N, d, n_agents, 0, 0, 0, 0, scale, dtype};
+  AgentsRef learn{agents, agents_batch_stride, (long long)n_agents * d};
+  return forward_impl(p, q, k, v, &learn, out, nullptr, 0, false,
+                      static_cast<cudaStream_t>(stream));
+}
+
+size_t agent_attn_workspace_bytes(int B, int H, int N, int d, int n_agents, int dtype) {
+  if (validate_common(B, H, N, d, n_agents, 1.0f, dtype) != AA_OK) return 0;
+  int sms = 0;
+  if (device_sm_count(&sms) != AA_OK) return 0;
+  Problem p{B, H, N, d, n_agents, 0, 0, 0, 0, 1.0f, dtype};
+  Scratch s;
+  plan_scratch(p, sms, &s);
+  return s.total;
+}
+
+int agent_attn_forward_host(const void* q_host, const void* k_host, const void* v_host,
+                            const void* agents_host_or_null, void* out_host, int B, int H, int N,
+                            int d, int grid_h, int grid_w, int pool_h, int pool_w, float scale,
+                            int dtype, void* stream) {
+  int rc = validate_grid(N, grid_h, grid_w, pool_h, pool_w);
+  if (rc != AA_OK) return rc;
+  const int kk = pool_h * pool_w;
+  rc = validate_common(B, H, N, d, kk, scale, dtype);
+  if (rc != AA_OK) return rc;
+  if (!q_host || !k_host || !v_host || !out_host) return AA_ERR_NULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t eb = dtype == AA_FP32 ? 4 : 2;
+  const size_t tbytes = round256((size_t)B * H * N * d * eb);
+  const size_t abytes = agents_host_or_null ? round256((size_t)H * kk * d * eb) : 0;
+  char* dev = nullptr;
+  rc = scratch_alloc(reinterpret_cast<void**>(&dev), 4 * tbytes + abytes, st);
+  if (rc != AA_OK) return rc;
+  char *dq = dev, *dk = dev + tbytes, *dv = dev + 2 * tbytes, *dout = dev + 3 * tbytes;
+  char* da = agents_host_or_null ? dev + 4 * tbytes : nullptr;
+  const size_t raw = (size_t)B * H * N * d * eb;
+  cudaError_t e = cudaMemcpyAsync(dq, q_host, raw, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k_host, raw, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v_host, raw, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && da)
+    e = cudaMemcpyAsync(da, agents_host_or_null, (size_t)H * kk * d * eb, cudaMemcpyHostToDevice,
+                        st);
+  if (e != cudaSuccess) {
+    cudaFreeAsync(dev, st);
+    return cuda_fail(e, "cudaMemcpyAsync(host to device)");
+  }
+  rc = pooled_forward(dq, dk, dv, da, dout, B, H, N, d, grid_h, grid_w, pool_h, pool_w, scale,
+                      dtype, nullptr, 0, false, stream);
+  if (rc == AA_OK) {
+    e = cudaMemcpyAsync(out_host, dout, raw, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) rc = cuda_fail(e, "cudaMemcpyAsync(device to host)");
+  }
+  cudaError_t e2 = cudaFreeAsync(dev, st);
+  if (rc == AA_OK && e2 != cudaSuccess) rc = cuda_fail(e2, "cudaFreeAsync");
+  cudaError_t e3 = cudaStreamSynchronize(st);
+  if (rc == AA_OK && e3 != cudaSuccess) rc = cuda_fail(e3, "cudaStreamSynchronize");
+  return rc;
+}
+
+int agent_attn_stage_pool(const void* q, float* agents_f32, void* agents_lowp, int B, int H, int N,
+                          int d, int grid_h, int grid_w, int pool_h, int pool_w, int dtype,
+                          void* stream) {
+  int rc = validate_grid(N, grid_h, grid_w, pool_h, pool_w);
+  if (rc != AA_OK) return rc;
+  rc = validate_common(B, H, N, d, pool_h * pool_w, 1.0f, dtype);
+  if (rc != AA_OK) return rc;
+  if (!q) return AA_ERR_NULL;
+  if (dtype == AA_FP32) agents_lowp = nullptr;
+  if (!agents_f32 && !agents_lowp) return AA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(agents_f32) || !aligned16(agents_lowp)) return AA_ERR_ALIGN;
+  Problem p{B, H, N, d, pool_h * pool_w, grid_h, grid_w, pool_h, pool_w, 1.0f, dtype};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == AA_FP32) return launch_pool<float>(p, q, agents_f32, nullptr, st);
+  return launch_pool<__nv_bfloat16>(p, q, agents_f32, static_cast<__nv_bfloat16*>(agents_lowp),
+                                    st);
+}
+
+int agent_attn_stage_aggregate(const void* agents, long long agents_batch_stride, const void* k,
+                               const void* v, float* va_f32, void* va_lowp, int B, int H, int N,
+                               int d, int n_agents, float scale, int dtype, void* stream) {
+  int rc = validate_common(B, H, N, d, n_agents, scale, dtype);
+  if (rc != AA_OK) return rc;
+  if (!agents || !k || !v) return AA_ERR_NULL;
+  if (dtype == AA_FP32) va_lowp = nullptr;
+  if (!va_f32 && !va_lowp) return AA_ERR_NULL;
+  if (!aligned16(agents) || !aligned16(k) || !aligned16(v) || !aligned16(va_f32) ||
+      !aligned16(va_lowp))
+    return AA_ERR_ALIGN;
+  if (agents_batch_stride < 0 || (agents_batch_stride % 8) != 0) return AA_ERR_ALIGN;
+  int sms = 0;
+  rc = device_sm_count(&sms);
+  if (rc != AA_OK) return rc;
+  Problem p{B, H, N, d, n_agents, 0, 0, 0, 0, scale, dtype};
+  Scratch s;
+  plan_scratch(p, sms, &s);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = nullptr;
+  rc = scratch_alloc(reinterpret_cast<void**>(&ws), s.total, st);
+  if (rc != AA_OK) return rc;
+  AgentsRef ag{agents, agents_batch_stride, (long long)n_agents * d};
+  rc = (dtype == AA_FP32)
+           ? run_aggregate<float>(p, s, ag, k, v, ws, va_f32, nullptr, st)
+           : run_aggregate<__nv_bfloat16>(p, s, ag, k, v, ws, va_f32,
+                                          static_cast<__nv_bfloat16*>(va_lowp), st);
+  cudaError_t e = cudaFreeAsync(ws, st);
+  if (rc == AA_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
+  return rc;
+}
+
+int agent_attn_stage_broadcast(const void* q, const void* agents, long long agents_batch_stride,
+                               const void* va, void* out, int B, int H, int N, int d,
+                               int n_agents, float scale, int dtype, void* stream) {
+  int rc = validate_common(B, H, N, d, n_agents, scale, dtype);
+  if (rc != AA_OK) return rc;
+  if (!q || !agents || !va || !out) return AA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(agents) || !aligned16(va) || !aligned16(out))
+    return AA_ERR_ALIGN;
+  if (agents_batch_stride < 0 || (agents_batch_stride % 8) != 0) return AA_ERR_ALIGN;
+  Problem p{B, H, N, d, n_agents, 0, 0, 0, 0, scale, dtype};
+  AgentsRef ag{agents, agents_batch_stride, (long long)n_agents * d};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return (dtype == AA_FP32) ? run_broadcast<float>(p, q, ag, va, out, st)
+                            : run_broadcast<__nv_bfloat16>(p, q, ag, va, out, st);
+}
+
+const char* agent_attn_status_string(int status) {
+  switch (status) {
+    case AA_OK: return "AA_OK: success";
+    case AA_ERR_NULL: return "AA_ERR_NULL: a required pointer is NULL";
+    case AA_ERR_SHAPE: return "AA_ERR_SHAPE: inconsistent sizes (N vs grid, pool vs grid, B/H/N)";
+    case AA_ERR_UNSUPPORTED: return "AA_ERR_UNSUPPORTED: dtype, head dim d or agent count k not supported";
+    case AA_ERR_ALIGN: return "AA_ERR_ALIGN: pointer or stride not aligned as required";
+    case AA_ERR_WORKSPACE: return "AA_ERR_WORKSPACE: caller workspace too small";
+    case AA_ERR_CUDA: return g_cuda_err;
+    case AA_ERR_VALUE: return "AA_ERR_VALUE: scale must be finite and > 0";
+    case AA_ERR_TIMEOUT:
+      return "AA_ERR_TIMEOUT: a kernel's bounded wait expired (pipeline stalled); results invalid";
+    default: return "unknown agent_attn status";
+  }
+}
+
+const char* agent_attn_version(void) { return "0.1.0"; }
+
+int agent_attn_check_device_error(void) {
+  unsigned int word = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&word, tc::g_watchdog, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol(watchdog)");
+  if (word == 0) return AA_OK;
+  e = cudaMemcpyToSymbol(tc::g_watchdog, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol(watchdog)");
+  return AA_ERR_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,164 @@
+/*
+ * agent_attn.h -- C ABI of the B200 (sm_100a) Agent Attention forward pass.
+ *
+ * The operation (per batch b and head h, "slice"):
+ *
+ *   A   = agents: pool_h x pool_w adaptive average pool of Q over its
+ *         grid_h x grid_w token grid, or externally supplied learnable agents.
+ *         [Agent Attention: On the Integration of Softmax and Linear Attention,
+ *          arXiv:2312.08874v3 summary, §4 "Efficiency" (pooling is the default
+ *          agent source; learnable parameters are another) and §6 (A = f(Q)).]
+ *   V_A = softmax(A K^T * scale) V            agent aggregation  (k x d)
+ *   O   = softmax(Q A^T * scale) V_A          agent broadcast    (N x d)
+ *         [jsqmd.com, "Agent Attention：Transformer计算量太大？试试这个'代理令牌'
+ *          的轻量化方案", §1 two-stage pseudocode (scale 1/sqrt(d) in both
+ *          softmaxes); arXiv:2312.08874v3 summary §4 "Agent Attention".]
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Tensors are contiguous row-major [B, H, N, d] device buffers of the element
+ * type `dtype` (AA_FP32: float, AA_BF16: bfloat16).  Tokens are row-major on
+ * the grid, token n = y * grid_w + x; agent j = py * pool_w + px.  Adaptive
+ * pooling bin i of an axis of length G cut into P bins covers tokens
+ * [floor(i*G/P), ceil((i+1)*G/P)); neighbouring bins may share a row when P
+ * does not divide G.  `scale` multiplies the logits of both softmaxes (the
+ * pages use 1/sqrt(d)).
+ *
+ * Limits: B, H, N >= 1; N == grid_h * grid_w for pooled agents;
+ * 1 <= pool_h <= grid_h, 1 <= pool_w <= grid_w; 1 <= k <= 256 agents;
+ * 8 <= d <= 128 with d % 8 == 0; every pointer 16-byte aligned; scale finite
+ * and > 0; `out` must not alias an input.
+ *
+ * Ownership: the caller owns every buffer.  The library keeps no pointer to
+ * them after a call returns.  Its only global state is per device: a cache of
+ * the SM count and a library-owned stream-ordered memory pool (created on
+ * first use, release threshold = unlimited) from which the entry points
+ * without a caller workspace take their scratch; calls on different streams
+ * are independent.
+ *
+ * Errors: every call validates all arguments before it launches anything and
+ * returns an aa_status.  AA_ERR_CUDA means a CUDA call or launch failed; the
+ * CUDA error text of the last such failure on the calling thread is then
+ * available from agent_attn_status_string(AA_ERR_CUDA).  Calls are
+ * asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream)
+ * unless stated otherwise.
+ */
+#ifndef AGENT_ATTN_H_
+#define AGENT_ATTN_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define AA_API __attribute__((visibility("default")))
+#else
+#define AA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  AA_OK = 0,
+  AA_ERR_NULL = 1,         /* a required pointer is NULL                              */
+  AA_ERR_SHAPE = 2,        /* sizes inconsistent (N != grid_h*grid_w, pool > grid...) */
+  AA_ERR_UNSUPPORTED = 3,  /* dtype, d or k outside the supported set                 */
+  AA_ERR_ALIGN = 4,        /* a pointer is not 16-byte aligned                        */
+  AA_ERR_WORKSPACE = 5,    /* caller workspace too small                              */
+  AA_ERR_CUDA = 6,         /* a CUDA runtime / driver call or a launch failed         */
+  AA_ERR_VALUE = 7,        /* scale not finite or not > 0                              */
+  AA_ERR_TIMEOUT = 8       /* a kernel's bounded wait expired (see check_device_error) */
+} aa_status;
+
+typedef enum { AA_FP32 = 0, AA_BF16 = 1 } aa_dtype;
+
+/* Whole forward pass with pooled agents.
+ *   q, k, v, out : [B, H, N, d] device buffers of `dtype`.
+ *   agents_or_null: NULL -> agents are pooled from q (pool_h x pool_w of them);
+ *                   non-NULL -> [H, pool_h*pool_w, d] learnable agents of
+ *                   `dtype`, shared over the batch (grid only checked vs N).
+ * Scratch memory (agents, partial aggregation state, V_A) is taken from the
+ * library's stream-ordered pool on `stream` and returned to it (freed in
+ * stream order) before the call returns. */
+AA_API int agent_attn_forward(const void* q, const void* k, const void* v, const void* agents_or_null,
+                       void* out, int B, int H, int N, int d, int grid_h, int grid_w, int pool_h,
+                       int pool_w, float scale, int dtype, void* stream);
+
+/* Same as agent_attn_forward, with caller-provided scratch: `workspace` is a
+ * device buffer of at least agent_attn_workspace_bytes(B, H, N, d,
+ * pool_h*pool_w, dtype) bytes, 256-byte aligned; AA_ERR_WORKSPACE otherwise.
+ * Its contents on entry do not matter and are garbage on exit. */
+AA_API int agent_attn_forward_ws(const void* q, const void* k, const void* v, const void* agents_or_null,
+                          void* out, int B, int H, int N, int d, int grid_h, int grid_w,
+                          int pool_h, int pool_w, float scale, int dtype, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/* Forward pass with externally supplied (learnable) agents; pooling is skipped.
+ *   agents: n_agents x d agent rows of `dtype`; slice (b, h) reads
+ *           agents + b*agents_batch_stride + h*n_agents*d (elements), so a
+ *           stride of 0 shares one [H, n_agents, d] set over the batch and a
+ *           stride of H*n_agents*d reads a full [B, H, n_agents, d] tensor.
+ *           agents_batch_stride must be 0 or a multiple of 8 elements. */
+AA_API int agent_attn_forward_agents(const void* q, const void* k, const void* v, const void* agents,
+                              int n_agents, long long agents_batch_stride, void* out, int B,
+                              int H, int N, int d, float scale, int dtype, void* stream);
+
+/* Scratch bytes the forward pass needs for this problem on the current
+ * device (it depends on the device's SM count).  Returns 0 if the arguments
+ * are invalid or no device is visible. */
+AA_API size_t agent_attn_workspace_bytes(int B, int H, int N, int d, int n_agents, int dtype);
+
+/* Synchronous convenience call on HOST buffers: copies q, k, v (and agents,
+ * if non-NULL: [H, pool_h*pool_w, d]) to the device, runs the forward pass
+ * and copies the result back into out_host, all on `stream`, then
+ * synchronizes `stream`.  Device buffers come from the library's
+ * stream-ordered pool.  Host buffers should be page-locked for the copies to overlap
+ * nothing else but run at full link speed; pageable memory also works. */
+AA_API int agent_attn_forward_host(const void* q_host, const void* k_host, const void* v_host,
+                            const void* agents_host_or_null, void* out_host, int B, int H, int N,
+                            int d, int grid_h, int grid_w, int pool_h, int pool_w, float scale,
+                            int dtype, void* stream);
+
+/* ---- single stages (the same kernels the forward pass launches) ---- */
+
+/* Agent pooling only: agents_f32 [B, H, pool_h*pool_w, d] float (may be NULL)
+ * and agents_lowp [B, H, pool_h*pool_w, d] of `dtype` (may be NULL; ignored
+ * for AA_FP32).  At least one output must be non-NULL. */
+AA_API int agent_attn_stage_pool(const void* q, float* agents_f32, void* agents_lowp, int B, int H, int N,
+                          int d, int grid_h, int grid_w, int pool_h, int pool_w, int dtype,
+                          void* stream);
+
+/* Agent aggregation (split over keys, then the log-sum-exp merge of the
+ * splits): va_f32 [B, H, n_agents, d] float (may be NULL) and va_lowp
+ * [B, H, n_agents, d] of `dtype` (may be NULL for AA_FP32).  agents is
+ * addressed as in agent_attn_forward_agents.  Scratch from the library's
+ * stream-ordered pool. */
+AA_API int agent_attn_stage_aggregate(const void* agents, long long agents_batch_stride, const void* k,
+                               const void* v, float* va_f32, void* va_lowp, int B, int H, int N,
+                               int d, int n_agents, float scale, int dtype, void* stream);
+
+/* Agent broadcast: out [B, H, N, d] of `dtype` from q, agents (addressed as
+ * in agent_attn_forward_agents) and va [B, H, n_agents, d] of `dtype`. */
+AA_API int agent_attn_stage_broadcast(const void* q, const void* agents, long long agents_batch_stride,
+                               const void* va, void* out, int B, int H, int N, int d,
+                               int n_agents, float scale, int dtype, void* stream);
+
+/* Human-readable text for a status code (for AA_ERR_CUDA, includes the last
+ * CUDA error text seen on the calling thread).  Never NULL. */
+AA_API const char* agent_attn_status_string(int status);
+
+/* Reads and clears the device-side watchdog of the current device.  Every
+ * wait inside the tensor-core kernels is bounded (2 s); a wait that expires
+ * makes its CTA skip the rest of its work, leaves the outputs invalid and
+ * sets the watchdog.  Returns AA_ERR_TIMEOUT if it was set since the last
+ * check, AA_OK otherwise.  Synchronous with respect to the device. */
+AA_API int agent_attn_check_device_error(void);
+
+/* Library version, "major.minor.patch". */
+AA_API const char* agent_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AGENT_ATTN_H_ */
