@@ -16,6 +16,7 @@ from .binding import (  # noqa: F401
     agent_attn_forward_ws,
     agent_attn_stage_pool,
     agent_attn_stage_aggregate,
+    agent_attn_stage_aggregate_static,
     agent_attn_stage_broadcast,
     agent_attn_status_string,
     agent_attn_workspace_bytes,

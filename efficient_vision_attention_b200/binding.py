@@ -47,7 +47,12 @@ _SIGNATURES = {
     "agent_attn_status_string": (ctypes.c_char_p, [_i]),
     "agent_attn_version": (ctypes.c_char_p, []),
     "agent_attn_check_device_error": (_i, []),
+    "agent_attn_stage_aggregate_static": (_i, [_vp, _ll, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                               _f, _i, _vp]),
 }
+
+# Size of the library's fixed scratch array (AA_STATIC_SCRATCH_BYTES in the header).
+AA_STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class AgentAttnError(RuntimeError):
@@ -177,3 +182,17 @@ def agent_attn_stage_broadcast(q, agents, agents_batch_stride, va, out, B, H, N,
 
 def agent_attn_check_device_error(check=True):
     return _finish(load_library().agent_attn_check_device_error(), check)
+
+
+def agent_attn_stage_aggregate_static(agents, agents_batch_stride, k, v, va_f32, va_lowp, B, H,
+                                      N, d, n_agents, scale, dtype, stream=None, check=True):
+    """Aggregation stage that allocates nothing: the split partials live in a
+    fixed array inside the library.  For callers that may not allocate device
+    memory (a plugin in a framework that owns the device memory, a loop that
+    forbids allocation after start-up).  Make the first call on a device
+    before any stream capture; calls that overlap on the GPU share the array
+    and race, so serialise them."""
+    st = load_library().agent_attn_stage_aggregate_static(
+        _ptr(agents), agents_batch_stride, _ptr(k), _ptr(v), _ptr(va_f32), _ptr(va_lowp), B, H, N,
+        d, n_agents, scale, dtype, _stream(stream))
+    return _finish(st, check)

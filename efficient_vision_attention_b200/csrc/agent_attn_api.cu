@@ -399,6 +399,31 @@ int pooled_forward(const void* q, const void* k, const void* v, const void* agen
                       static_cast<cudaStream_t>(stream));
 }
 
+// Fixed scratch of agent_attn_stage_aggregate_static: a file-scope device
+// array, so that entry point needs no allocation at all.  Its device address
+// is looked up once per device (with that device current) and cached.
+static __device__ __align__(256) unsigned char g_static_scratch[AA_STATIC_SCRATCH_BYTES];
+std::atomic<void*> g_static_scratch_addr[kMaxDevices];
+
+int static_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev >= 0 && dev < kMaxDevices) {
+    void* p = g_static_scratch_addr[dev].load(std::memory_order_acquire);
+    if (p != nullptr) {
+      *out = p;
+      return AA_OK;
+    }
+  }
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+  if (dev >= 0 && dev < kMaxDevices) g_static_scratch_addr[dev].store(p, std::memory_order_release);
+  *out = p;
+  return AA_OK;
+}
+
 }  // namespace
 }  // namespace aa
 
@@ -538,6 +563,41 @@ int agent_attn_stage_aggregate(const void* agents, long long agents_batch_stride
   cudaError_t e = cudaFreeAsync(ws, st);
   if (rc == AA_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
   return rc;
+}
+
+int agent_attn_stage_aggregate_static(const void* agents, long long agents_batch_stride,
+                                      const void* k, const void* v, float* va_f32, void* va_lowp,
+                                      int B, int H, int N, int d, int n_agents, float scale,
+                                      int dtype, void* stream) {
+  int rc = validate_common(B, H, N, d, n_agents, scale, dtype);
+  if (rc != AA_OK) return rc;
+  if (!agents || !k || !v) return AA_ERR_NULL;
+  if (dtype == AA_FP32) va_lowp = nullptr;
+  if (!va_f32 && !va_lowp) return AA_ERR_NULL;
+  if (!aligned16(agents) || !aligned16(k) || !aligned16(v) || !aligned16(va_f32) ||
+      !aligned16(va_lowp))
+    return AA_ERR_ALIGN;
+  if (agents_batch_stride < 0 || (agents_batch_stride % 8) != 0) return AA_ERR_ALIGN;
+  int sms = 0;
+  rc = device_sm_count(&sms);
+  if (rc != AA_OK) return rc;
+  Problem p{B, H, N, d, n_agents, 0, 0, 0, 0, scale, dtype};
+  Scratch s;
+  plan_scratch(p, sms, &s);
+  // The aggregation touches only the partial-state regions [pu_off, total) of
+  // the scratch layout; they are placed at the start of the fixed array.
+  const size_t need = s.total - s.pu_off;
+  if (need > (size_t)AA_STATIC_SCRATCH_BYTES) return AA_ERR_WORKSPACE;
+  void* base = nullptr;
+  rc = static_scratch_address(&base);
+  if (rc != AA_OK) return rc;
+  char* ws = static_cast<char*>(base) - s.pu_off;   // only ws + pu_off onwards is addressed
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AgentsRef ag{agents, agents_batch_stride, (long long)n_agents * d};
+  return (dtype == AA_FP32)
+             ? run_aggregate<float>(p, s, ag, k, v, ws, va_f32, nullptr, st)
+             : run_aggregate<__nv_bfloat16>(p, s, ag, k, v, ws, va_f32,
+                                            static_cast<__nv_bfloat16*>(va_lowp), st);
 }
 
 int agent_attn_stage_broadcast(const void* q, const void* agents, long long agents_batch_stride,

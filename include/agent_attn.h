@@ -143,6 +143,34 @@ AA_API int agent_attn_stage_broadcast(const void* q, const void* agents, long lo
                                const void* va, void* out, int B, int H, int N, int d,
                                int n_agents, float scale, int dtype, void* stream);
 
+/* ---- aggregation without any allocation ----
+ *
+ * No counterpart in the paper: this entry point exists for callers that may
+ * not allocate device memory themselves, e.g. code running as a plugin inside
+ * a host framework that owns and budgets all device memory, or a real-time
+ * loop that forbids allocation after start-up.
+ *
+ * Same inputs, outputs and semantics as agent_attn_stage_aggregate, but the
+ * split-over-keys partial state lives in one fixed array inside the library
+ * (a file-scope __device__ array of AA_STATIC_SCRATCH_BYTES bytes, present on
+ * every device that loads the library until the process exits) instead of
+ * memory taken from a pool.  The call allocates and frees nothing.
+ *   - Problems whose partial state exceeds AA_STATIC_SCRATCH_BYTES are
+ *     rejected with AA_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - Every call shares the one array and it keeps the last call's contents;
+ *     nothing in it needs to start at zero (each call writes every partial it
+ *     reads back).  Calls whose work overlaps on the GPU (different streams,
+ *     or several host threads) race on the array: serialise them. */
+#define AA_STATIC_SCRATCH_BYTES (16u << 20)
+
+AA_API int agent_attn_stage_aggregate_static(const void* agents, long long agents_batch_stride,
+                                             const void* k, const void* v, float* va_f32,
+                                             void* va_lowp, int B, int H, int N, int d,
+                                             int n_agents, float scale, int dtype, void* stream);
+
 /* Human-readable text for a status code (for AA_ERR_CUDA, includes the last
  * CUDA error text seen on the calling thread).  Never NULL. */
 AA_API const char* agent_attn_status_string(int status);
