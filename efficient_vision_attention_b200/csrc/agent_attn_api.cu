@@ -202,14 +202,14 @@ int launch_pool(const Problem& p, const void* q, float* a_f32, T* a_lowp, cudaSt
       const long long nb = (p.BH() - b0 < 65535) ? p.BH() - b0 : 65535;
       const long long qoff = b0 * (long long)p.N * p.d;
       const long long aoff = b0 * (long long)p.k * p.d;
-      agent_pool_kernel<T><<<dim3(p.pool_h, (unsigned)nb), 256, 0, st>>>(
+      agent_pool_kernel<T><<<dim3(p.pool_h, (unsigned)nb), kPoolThreads, 0, st>>>(
           static_cast<const T*>(q) + qoff, a_f32 ? a_f32 + aoff : nullptr,
           a_lowp ? a_lowp + aoff : nullptr, p.N, p.d, p.grid_h, p.grid_w, p.pool_h, p.pool_w);
       AA_CUDA(cudaGetLastError());
     }
     return AA_OK;
   }
-  agent_pool_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(q), a_f32, a_lowp, p.N, p.d,
+  agent_pool_kernel<T><<<grid, kPoolThreads, 0, st>>>(static_cast<const T*>(q), a_f32, a_lowp, p.N, p.d,
                                              p.grid_h, p.grid_w, p.pool_h, p.pool_w);
   AA_CUDA(cudaGetLastError());
   return AA_OK;

@@ -37,6 +37,33 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&out)[8]) {
   }
 }
 
+// Raw 16-byte load and its widening (8 bf16 or, for fp32, the first of two
+// halves: fp32 rows are read as two 16-byte halves by the caller's unpack).
+__device__ __forceinline__ uint4 load16(const __nv_bfloat16* p) {
+  return *reinterpret_cast<const uint4*>(p);
+}
+__device__ __forceinline__ uint4 load16(const float* p) {
+  return *reinterpret_cast<const uint4*>(p);
+}
+__device__ __forceinline__ void unpack8(const uint4& raw, const __nv_bfloat16*, float (&out)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    out[2 * i] = f.x;
+    out[2 * i + 1] = f.y;
+  }
+}
+// fp32: 8 values span 32 bytes; `raw` holds the first 16, the rest is reloaded.
+__device__ __forceinline__ void unpack8(const uint4& raw, const float* p, float (&out)[8]) {
+  out[0] = __uint_as_float(raw.x);
+  out[1] = __uint_as_float(raw.y);
+  out[2] = __uint_as_float(raw.z);
+  out[3] = __uint_as_float(raw.w);
+  float4 b = *reinterpret_cast<const float4*>(p + 4);
+  out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+}
+
 // Adaptive pooling bin [start, end) of bin i when an axis of length g is cut
 // into p bins: [floor(i*g/p), ceil((i+1)*g/p)).
 __host__ __device__ __forceinline__ int bin_start(int i, int g, int p) {

@@ -16,16 +16,20 @@ namespace aa {
 
 // ----------------------------------------------------------------- pooling
 // One CTA per (slice bh, agent row py).  Work item = (px, 8-channel group);
-// when there are few items, several threads split the bin's rows and the
-// partial sums are reduced through shared memory.  Sums are fp32; the divisor
+// the bin's grid rows are spread over up to kPoolThreads / items threads, each
+// summing its rows' bin columns with 16-byte loads, eight in flight, and the
+// row partials are reduced through shared memory.  Small CTAs (4 per SM) keep
+// every CTA of the usual shapes resident at once.  Sums are fp32; the divisor
 // is the bin's own token count.  Writes fp32 and/or low-precision agents.
+constexpr int kPoolThreads = 256;
+
 template <typename T>
-__global__ void __launch_bounds__(256) agent_pool_kernel(const T* __restrict__ q,
-                                                         float* __restrict__ a_f32,
-                                                         T* __restrict__ a_lowp, int N, int d,
-                                                         int grid_h, int grid_w, int pool_h,
-                                                         int pool_w) {
-  __shared__ float red[256 * 8];
+__global__ void __launch_bounds__(kPoolThreads, 4) agent_pool_kernel(const T* __restrict__ q,
+                                                                  float* __restrict__ a_f32,
+                                                                  T* __restrict__ a_lowp, int N,
+                                                                  int d, int grid_h, int grid_w,
+                                                                  int pool_h, int pool_w) {
+  __shared__ float red[kPoolThreads * 8];
   const int py = blockIdx.x;
   const long long bh = blockIdx.y;
   const int y0 = bin_start(py, grid_h, pool_h), y1 = bin_end(py, grid_h, pool_h);
@@ -50,8 +54,22 @@ __global__ void __launch_bounds__(256) agent_pool_kernel(const T* __restrict__ q
       const int px = item / groups, g = item % groups;
       const int x0 = bin_start(px, grid_w, pool_w), x1 = bin_end(px, grid_w, pool_w);
       for (int y = y0 + ys; y < y1; y += ysplit) {
-        const T* row = qs + ((long long)y * grid_w) * d + g * 8;
-        for (int x = x0; x < x1; ++x) {
+        const T* row = qs + ((long long)y * grid_w + x0) * d + g * 8;
+        const int w = x1 - x0;
+        int x = 0;
+        for (; x + 8 <= w; x += 8) {       // eight independent 16-byte loads in flight
+          uint4 raw[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) raw[u] = load16(row + (long long)(x + u) * d);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            float v[8];
+            unpack8(raw[u], row + (long long)(x + u) * d, v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] += v[i];
+          }
+        }
+        for (; x < w; ++x) {
           float v[8];
           load8(row + (long long)x * d, v);
 #pragma unroll
@@ -64,9 +82,9 @@ __global__ void __launch_bounds__(256) agent_pool_kernel(const T* __restrict__ q
       for (int i = 0; i < 8; ++i) red[threadIdx.x * 8 + i] = acc[i];
       __syncthreads();
       if (item >= 0 && ys == 0) {
-        for (int s = 1; s < ysplit; ++s) {
+        for (int s2 = 1; s2 < ysplit; ++s2) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] += red[(threadIdx.x + s * items) * 8 + i];
+          for (int i = 0; i < 8; ++i) acc[i] += red[(threadIdx.x + s2 * items) * 8 + i];
         }
       }
       __syncthreads();
@@ -233,6 +251,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_attend_kernel(SimtAttendArg
 
 // ------------------------------------------------------------------ merge
 // One warp per (slice, agent row): V_A = sum_s 2^(m_s - M) U_s / sum_s 2^(m_s - M) l_s.
+// Lane s owns split s's weight (computed once); the weights are broadcast by
+// shuffles while the lanes sweep the d columns of every split's partial row.
 template <typename T>
 __global__ void __launch_bounds__(256) agent_merge_kernel(const float* __restrict__ part_u,
                                                           const float* __restrict__ part_ml,
@@ -252,24 +272,50 @@ __global__ void __launch_bounds__(256) agent_merge_kernel(const float* __restric
     mx = fmaxf(mx, part_ml[((slot0 + s) * n_agents + j) * 2]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float den = 0.f;
-  for (int s = lane; s < n_splits; s += 32) {
-    const float* ml = part_ml + ((slot0 + s) * n_agents + j) * 2;
-    den += exp2f(ml[0] - mx) * ml[1];
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f, den = 0.f;
+  for (int s0 = 0; s0 < n_splits; s0 += 32) {
+    float w = 0.f;
+    if (s0 + lane < n_splits) {
+      const float* ml = part_ml + ((slot0 + s0 + lane) * n_agents + j) * 2;
+      w = exp2f(ml[0] - mx);
+      den += w * ml[1];
+    }
+    const int cnt = min(32, n_splits - s0);
+    const long long stride = (long long)n_agents * d;      // between consecutive splits
+    const float* base = part_u + ((slot0 + s0) * n_agents + j) * (long long)d;
+    for (int s = 0; s < cnt; s += 4) {                      // four splits' loads in flight
+      float u[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = lane + 32 * q;
+          u[a][q] = (s + a < cnt && c < d) ? base[(s + a) * stride + c] : 0.f;
+        }
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const float ws = __shfl_sync(0xffffffffu, w, (s + a) & 31);
+        const float wa = (s + a < cnt) ? ws : 0.f;
+        acc0 = fmaf(wa, u[a][0], acc0);
+        acc1 = fmaf(wa, u[a][1], acc1);
+        acc2 = fmaf(wa, u[a][2], acc2);
+        acc3 = fmaf(wa, u[a][3], acc3);
+      }
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
   const float inv = 1.f / den;
-  for (int c = lane; c < d; c += 32) {
-    float acc = 0.f;
-    for (int s = 0; s < n_splits; ++s) {
-      const long long r = (slot0 + s) * n_agents + j;
-      acc += exp2f(part_ml[r * 2] - mx) * part_u[r * d + c];
+  const float accs[4] = {acc0, acc1, acc2, acc3};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = lane + 32 * q;
+    if (c < d) {
+      const float v = accs[q] * inv;
+      const long long o = row * d + c;
+      if (va_f32) va_f32[o] = v;
+      if (va_lowp) va_lowp[o] = from_f32<T>(v);
     }
-    const float v = acc * inv;
-    const long long o = row * d + c;
-    if (va_f32) va_f32[o] = v;
-    if (va_lowp) va_lowp[o] = from_f32<T>(v);
   }
 }
 

@@ -6,25 +6,33 @@
 // stream of columns, with the score tile and the output accumulator in TMEM:
 //
 //  agent_aggregate_tc  rows = agents (M = 128 per TMEM tile, 1 or 2 tiles),
-//                      columns = keys streamed in tiles of 128 through a 4-deep
-//                      TMA ring of K and V tiles.  S = A K^T (SS MMA), online
-//                      softmax in registers (one thread per agent row), P
-//                      written back into TMEM as bf16 over S, U += P V (TS MMA,
-//                      V as an MN-major operand).  A persistent grid cuts the
-//                      key tiles of all slices into equal contiguous ranges
-//                      (one range per CTA, one CTA per SM); each CTA writes one
-//                      partial (U, running max, running sum) per slice it
-//                      touches, merged afterwards by agent_merge_kernel.
+//                      columns = keys streamed in tiles of 64 through an
+//                      8-deep TMA ring of K and V tiles.  S = A K^T (SS MMA),
+//                      online softmax in registers (one thread per agent row),
+//                      P written back into TMEM as bf16 over S, U += P V (TS
+//                      MMA, V as an MN-major operand) and l += P 1 (TS MMA
+//                      against a tile of ones: the row sums come from the
+//                      tensor core, summed from the same bf16 P).  Score tiles
+//                      are double-buffered per softmax group, so the tensor
+//                      core computes tile i+1 while the group works on tile i.
+//                      A persistent grid cuts the key tiles of all slices into
+//                      equal contiguous ranges (one range per CTA, one CTA per
+//                      SM); each CTA writes one partial (U, running max,
+//                      running sum) per slice it touches, merged afterwards by
+//                      agent_merge_kernel.
 //  agent_broadcast_tc  rows = queries streamed in tiles of 128 (TMA ring),
 //                      columns = the k agents, resident in shared memory with
 //                      V_A for the whole slice.  S = Q A^T, row softmax over k
-//                      in registers, O = P V_A, 1/l applied in the epilogue,
-//                      O staged in shared memory and written with TMA stores.
+//                      in registers, O = P V_A and l = P 1 on the tensor core,
+//                      1/l applied in the epilogue, O staged in shared memory
+//                      and written with TMA stores.
 //
 // Warp roles (320 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and
 // issues the MMAs (one thread), warps 2-5 and 6-9 are two softmax groups of
 // 128 threads (thread = TMEM lane = row) working on alternating tiles (or, for
-// k > 128 in the aggregation, on the two 128-agent halves).
+// k > 128 in the aggregation, on the two 128-agent halves).  Every wait is
+// bounded; a wait that gives up makes its CTA skip the rest of its work and
+// raises the device watchdog.
 #pragma once
 
 #include <atomic>
@@ -37,12 +45,15 @@ namespace aa {
 namespace tc {
 
 constexpr int kThreads = 320;
-constexpr int kTileRows = 128;               // MMA M; keys (aggregate) or queries (broadcast) per tile
 constexpr int kRowBytes = 128;               // one swizzled 128-byte row per token (d <= 64 bf16)
-constexpr int kTileBytes = kTileRows * kRowBytes;
-constexpr int kAggStages = 4;
+constexpr int kKeyTile = 64;                 // keys per aggregation tile
+constexpr int kQTile = 128;                  // queries per broadcast tile (MMA M)
+constexpr int kKTileBytes = kKeyTile * kRowBytes;
+constexpr int kQTileBytes = kQTile * kRowBytes;
+constexpr int kAggStages = 8;
 constexpr int kBcStages = 4;
 constexpr int kMaxAgents = 256;
+constexpr int kOnesBytes = 16 * kRowBytes;   // 16 rows of bf16 ones (row-sum operand)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale only when the max grows by > 2^8
 
 struct AggParams {
@@ -67,11 +78,11 @@ struct BcParams {
 struct AggBars {
   uint64_t full[kAggStages], empty[kAggStages];
   uint64_t a_full, a_empty;
-  uint64_t s_full[2], p_full[2], pv_done[2];
-  uint64_t x_pub, x_done;    // group 1 -> group 0 hand-over of (m, l, U) per segment
+  uint64_t s_full[2][2], p_full[2][2], pv_done[2][2];   // [group][score buffer]
+  uint64_t x_pub, x_done;    // group 1 -> group 0 hand-over per segment (k <= 128)
   uint32_t tmem_base;
   int abort;
-  float m_x[128], l_x[128];
+  float m_x[128];
 };
 
 struct BcBars {
@@ -94,9 +105,18 @@ __device__ __forceinline__ void agent_coords(long long bh, int H, int b_sets, in
   *b = b_sets > 1 ? (int)(bh / H) : 0;
 }
 
+// Fill the row-sum operand (16 rows x 128 bytes of bf16 1.0) and make it
+// visible to the tensor core.
+__device__ __forceinline__ void fill_ones(uint8_t* ones) {
+  for (int i = threadIdx.x; i < kOnesBytes / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
+  fence_proxy_async_smem();
+}
+
 // ============================================================== aggregation
-constexpr size_t kAggSmemBytes =
-    1024 + (size_t)kMaxAgents * kRowBytes + 2 * (size_t)kAggStages * kTileBytes + sizeof(AggBars);
+constexpr size_t kAggSmemBytes = 1024 + (size_t)kMaxAgents * kRowBytes +
+                                 2 * (size_t)kAggStages * kKTileBytes + kOnesBytes +
+                                 sizeof(AggBars);
 
 __global__ void __launch_bounds__(kThreads, 1)
     agent_aggregate_tc_kernel(const __grid_constant__ CUtensorMap map_k,
@@ -107,8 +127,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sK = sA + kMaxAgents * kRowBytes;
-  uint8_t* sV = sK + kAggStages * kTileBytes;
-  AggBars* bars = reinterpret_cast<AggBars*>(sV + kAggStages * kTileBytes);
+  uint8_t* sV = sK + kAggStages * kKTileBytes;
+  uint8_t* sOnes = sV + kAggStages * kKTileBytes;
+  AggBars* bars = reinterpret_cast<AggBars*>(sOnes + kOnesBytes);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -118,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tps = p.tiles_per_slice;
   const bool two = p.k > 128;                 // two 128-row agent tiles
   const int d16 = (p.d + 15) >> 4;            // K steps of S = A K^T
-  const int dn = d16 * 16;                    // N of U += P V
+  const int dn = d16 * 16;                    // N of U += P V; l sits in column dn
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAggStages; ++s) {
@@ -127,11 +148,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->a_full, 1);
     mbar_init(&bars->a_empty, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 128);
-      mbar_init(&bars->pv_done[i], 1);
-    }
+    for (int g = 0; g < 2; ++g)
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&bars->s_full[g][b], 1);
+        mbar_init(&bars->p_full[g][b], 128);
+        mbar_init(&bars->pv_done[g][b], 1);
+      }
     mbar_init(&bars->x_pub, 128);
     mbar_init(&bars->x_done, 128);
     bars->abort = 0;
@@ -140,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&map_v);
     prefetch_tensormap(&map_a);
   }
+  fill_ones(sOnes);
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
@@ -148,7 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  // TMEM columns: S/P of group g at g*128, U of group g at 256 + g*128.
+  // TMEM columns: score buffer b of group g at g*128 + b*64 (P over its first
+  // 32 columns), U of group g at 256 + g*128 (dn columns), l at 256 + g*128 + dn.
 
   if (warp == 0) {
     if (lane == 0) {
@@ -172,10 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const int key0 = (int)(t - bh * tps) * kTileRows;
-          mbar_expect_tx(&bars->full[s], 2 * kTileBytes);
-          tma_load_3d(sK + s * kTileBytes, &map_k, &bars->full[s], 0, key0, (int)bh);
-          tma_load_3d(sV + s * kTileBytes, &map_v, &bars->full[s], 0, key0, (int)bh);
+          const int key0 = (int)(t - bh * tps) * kKeyTile;
+          mbar_expect_tx(&bars->full[s], 2 * kKTileBytes);
+          tma_load_3d(sK + s * kKTileBytes, &map_k, &bars->full[s], 0, key0, (int)bh);
+          tma_load_3d(sV + s * kKTileBytes, &map_v, &bars->full[s], 0, key0, (int)bh);
         }
         if (!ok) break;
       }
@@ -192,9 +216,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------- MMA issuer
-      const uint32_t idesc_s = idesc_bf16(128, kTileRows, 0, 0);
+      const uint32_t idesc_s = idesc_bf16(128, kKeyTile, 0, 0);
       const uint32_t idesc_pv = idesc_bf16(128, dn, 0, 1);
+      const uint32_t idesc_l = idesc_bf16(128, 16, 0, 1);
       const uint32_t sA_addr = smem_u32(sA), sK_addr = smem_u32(sK), sV_addr = smem_u32(sV);
+      const uint64_t ones_desc = sw128_desc(smem_u32(sOnes), 8192);
       long long it0 = 0;
       int seg = 0;
       int cnt_s[2] = {0, 0}, cnt_p[2] = {0, 0};
@@ -213,17 +239,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           for (int g = 0; g < 2; ++g) {
             if (!two && (i & 1) != g) continue;
-            if (cnt_s[g] > 0) {
-              if (!mbar_wait(&bars->pv_done[g], (uint32_t)(cnt_s[g] - 1) & 1, abort)) return false;
+            const int J = cnt_s[g], b = J & 1;
+            if (J >= 2) {   // the buffer's previous P has been consumed
+              if (!mbar_wait(&bars->pv_done[g][b], (uint32_t)((J >> 1) - 1) & 1, abort))
+                return false;
               tc_fence_after();
             }
             const int mt = two ? g : 0;
+            const uint32_t d_tm = tmem + g * 128 + b * 64;
             for (int kk = 0; kk < d16; ++kk) {
-              const uint64_t da = sw128_desc(sA_addr + mt * kTileBytes + kk * 32, 16);
-              const uint64_t db = sw128_desc(sK_addr + s * kTileBytes + kk * 32, 16);
-              mma_ss(tmem + g * 128, da, db, idesc_s, kk > 0);
+              const uint64_t da = sw128_desc(sA_addr + mt * 128 * kRowBytes + kk * 32, 16);
+              const uint64_t db = sw128_desc(sK_addr + s * kKTileBytes + kk * 32, 16);
+              mma_ss(d_tm, da, db, idesc_s, kk > 0);
             }
-            mma_commit(&bars->s_full[g]);
+            mma_commit(&bars->s_full[g][b]);
             ++cnt_s[g];
           }
           return true;
@@ -233,42 +262,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = (int)(itg % kAggStages);
           for (int g = 0; g < 2; ++g) {
             if (!two && (i & 1) != g) continue;
-            if (!mbar_wait(&bars->p_full[g], (uint32_t)cnt_p[g] & 1, abort)) return false;
+            const int J = cnt_p[g], b = J & 1;
+            if (!mbar_wait(&bars->p_full[g][b], (uint32_t)(J >> 1) & 1, abort)) return false;
             tc_fence_after();
-            for (int kk = 0; kk < kTileRows / 16; ++kk) {
-              const uint64_t db = sw128_desc(sV_addr + s * kTileBytes + kk * 2048, 8192);
-              mma_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, db, idesc_pv,
-                     (!first[g] || kk > 0) ? 1u : 0u);
+            const uint32_t p_tm = tmem + g * 128 + b * 64;
+            const uint32_t u_tm = tmem + 256 + g * 128;
+            for (int kk = 0; kk < kKeyTile / 16; ++kk) {
+              const uint32_t acc = (!first[g] || kk > 0) ? 1u : 0u;
+              const uint64_t dv = sw128_desc(sV_addr + s * kKTileBytes + kk * 2048, 8192);
+              mma_ts(u_tm, p_tm + kk * 8, dv, idesc_pv, acc);
+              mma_ts(u_tm + dn, p_tm + kk * 8, ones_desc, idesc_l, acc);
             }
             first[g] = false;
-            mma_commit(&bars->pv_done[g]);
+            mma_commit(&bars->pv_done[g][b]);
             ++cnt_p[g];
           }
           mma_commit(&bars->empty[s]);
           return true;
         };
-        if (!two) {
-          ok = issue_s(0);
-          for (int i = 0; i < n && ok; ++i) {
-            if (i + 1 < n) ok = issue_s(i + 1);
-            if (ok) ok = issue_pv(i);
-          }
-        } else {
-          for (int i = 0; i < n && ok; ++i) {
-            ok = issue_s(i);
-            if (ok) ok = issue_pv(i);
-          }
+        // one tile of look-ahead: S of tile i is issued before P V of tile i-1
+        for (int i = 0; i < n && ok; ++i) {
+          ok = issue_s(i);
+          if (ok && i > 0) ok = issue_pv(i - 1);
         }
+        if (ok) ok = issue_pv(n - 1);
         mma_commit(&bars->a_empty);
         it0 += n;
         t = seg_end;
       }
       // Let every MMA issued so far finish before TMEM is released.
       mma_commit(&bars->a_full);   // a_full is no longer waited on: use it as a drain marker
-      {
-        const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(&bars->a_full, (uint32_t)seg & 1) && globaltimer() - t0 < kWaitLimitNs) {
-        }
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&bars->a_full, (uint32_t)seg & 1) && globaltimer() - t0 < kWaitLimitNs) {
       }
     }
   } else {
@@ -279,94 +304,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;                // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;         // TMEM lane = row of the 128-row tile
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t s_col = tmem + lane_off + g * 128;
     const uint32_t u_col = tmem + lane_off + 256 + g * 128;
     const int agent = (two ? g * 128 : 0) + row;
     const bool warp_active = (two ? g * 128 : 0) + quad * 32 < p.k;
-    int cnt = 0, seg = 0;
+    int J = 0, seg = 0;
     bool ok = true;
     for (long long t = t_begin; t < t_end; ++seg) {
       const long long bh = t / tps;
       const long long seg_end = min(t_end, (bh + 1) * tps);
       const int n = (int)(seg_end - t);
       const int n_mine = two ? n : (g == 0 ? (n + 1) / 2 : n / 2);
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY;
       bool first = true;
       for (int i = 0; i < n; ++i) {
         if (!two && (i & 1) != g) continue;
-        const int key0 = (int)(t + i - bh * tps) * kTileRows;
-        const int valid = min(kTileRows, p.N - key0);
-        if (ok) ok = warp_wait(&bars->s_full[g], (uint32_t)cnt & 1, abort);
+        const int b = J & 1;
+        const uint32_t s_col = tmem + lane_off + g * 128 + b * 64;
+        const int valid = min(kKeyTile, p.N - (int)(t + i - bh * tps) * kKeyTile);
+        if (ok) ok = warp_wait(&bars->s_full[g][b], (uint32_t)(J >> 1) & 1, abort);
         tc_fence_after();
         if (ok && warp_active) {
-          // pass 1: row max over the valid keys of this tile
-          float mx = -INFINITY;
-#pragma unroll 1
-          for (int c = 0; c < kTileRows / 16; ++c) {
-            if (c * 16 >= valid) break;
-            float v[16];
-            tmem_ld16(s_col + c * 16, v);
+          float v[64];
+          tmem_ld64(s_col, v);
+          if (valid < kKeyTile) {               // ragged last tile: mask the missing keys
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              if (c * 16 + e < valid) mx = fmaxf(mx, v[e]);
+            for (int e = 0; e < 64; ++e)
+              if (e >= valid) v[e] = -INFINITY;
           }
-          const float mt = mx * p.c;
+          float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
+          float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
+          const float mt = max32(v1, max32(v0, -INFINITY)) * p.c;
           if (first) {
             m = mt;
             first = false;
           } else if (__any_sync(0xffffffffu, mt > m + kRescaleThreshold)) {
-            // the running max grew a lot: rescale U and l (PV of the previous
-            // tile has completed: it precedes this tile's S in the MMA order)
-            const float m_new = fmaxf(m, mt);
-            const float alpha = ex2(m - m_new);
-            l *= alpha;
-            m = m_new;
+            // the running max grew a lot: once the previous P V has landed,
+            // rescale U and l by 2^(m_old - m_new)
+            ok = warp_wait(&bars->pv_done[g][(J - 1) & 1], (uint32_t)((J - 1) >> 1) & 1, abort);
+            tc_fence_after();
+            if (ok) {
+              const float m_new = fmaxf(m, mt);
+              const float alpha = ex2(m - m_new);
+              m = m_new;
 #pragma unroll 1
-            for (int c = 0; c < dn / 16; ++c) {
-              float u[16];
-              tmem_ld16(u_col + c * 16, u);
+              for (int c = 0; c < dn / 16 + 1; ++c) {
+                float u[16];
+                tmem_ld16(u_col + c * 16, u);
 #pragma unroll
-              for (int e = 0; e < 16; ++e) u[e] *= alpha;
-              tmem_st16(u_col + c * 16, u);
-            }
-          }
-          // pass 2: P = 2^(S*c - m) as bf16 over the first 64 columns of S
-          float sum = 0.f;
-#pragma unroll 1
-          for (int c = 0; c < kTileRows / 16; ++c) {
-            uint32_t pk[8];
-            if (c * 16 >= valid) {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) pk[e] = 0u;
-            } else {
-              float v[16];
-              tmem_ld16(s_col + c * 16, v);
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const float x = ex2(fmaf(v[e], p.c, -m));
-                v[e] = (c * 16 + e < valid) ? x : 0.f;
-                sum += v[e];
+                for (int e = 0; e < 16; ++e) u[e] *= alpha;
+                tmem_st16(u_col + c * 16, u);
               }
-#pragma unroll
-              for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
             }
-            tmem_st8(s_col + c * 8, pk);
           }
-          l += sum;
-          tmem_wait_st();
+          if (ok) {
+            uint32_t pk[16];
+            exp_pack32(v0, p.c, -m, pk);
+            tmem_st16u(s_col, pk);
+            exp_pack32(v1, p.c, -m, pk);
+            tmem_st16u(s_col + 16, pk);
+            tmem_wait_st();
+          }
         }
         tc_fence_before();
-        mbar_arrive(&bars->p_full[g]);
-        ++cnt;
+        mbar_arrive(&bars->p_full[g][b]);
+        ++J;
       }
       // ---- segment epilogue: write this CTA's partial for slice bh
       const int slot = (int)(cta - ((bh * tps + 1) * p.ctas - 1) / p.total_tiles);
       const long long slot_row = (bh * p.slots + slot) * (long long)p.k;
-      if (n_mine > 0 && ok) ok = warp_wait(&bars->pv_done[g], (uint32_t)(cnt - 1) & 1, abort);
+      if (n_mine > 0 && ok)
+        ok = warp_wait(&bars->pv_done[g][(J - 1) & 1], (uint32_t)((J - 1) >> 1) & 1, abort);
       tc_fence_after();
       if (two) {
         if (ok && warp_active) {            // warp-uniform: the TMEM loads are warp-collective
           const bool mine = agent < p.k;
+          const float l = tmem_ld1(u_col + dn);
           float* dst = p.part_u + (slot_row + agent) * p.d;
 #pragma unroll 1
           for (int c = 0; c < dn / 16; ++c) {
@@ -385,11 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else if (g == 1) {
         // both groups hold the same agent rows over different key tiles:
-        // group 1 publishes (m, l) and waits until group 0 has read its U
-        if (n_mine > 0 && ok && warp_active && row < p.k) {
-          bars->m_x[row] = m;
-          bars->l_x[row] = l;
-        }
+        // group 1 publishes its running max and waits until group 0 has read
+        // its accumulators
+        if (n_mine > 0 && ok && warp_active && row < p.k) bars->m_x[row] = m;
         tc_fence_before();
         mbar_arrive(&bars->x_pub);
         if (ok) ok = warp_wait(&bars->x_done, (uint32_t)seg & 1, abort);
@@ -400,6 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && warp_active) {            // warp-uniform: the TMEM loads are warp-collective
           const bool mine = row < p.k;
           const bool has1 = (n / 2) > 0;
+          const uint32_t u1_col = tmem + lane_off + 256 + 128;
           float mm = m, a0 = 1.f, a1 = 0.f;
           if (has1 && mine) {
             const float m1 = bars->m_x[row];
@@ -407,8 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             a0 = ex2(m - mm);
             a1 = ex2(m1 - mm);
           }
+          float l = a0 * tmem_ld1(u_col + dn);
+          if (has1) l += a1 * tmem_ld1(u1_col + dn);
           float* dst = p.part_u + (slot_row + row) * p.d;
-          const uint32_t u1_col = tmem + lane_off + 256 + 128;
 #pragma unroll 1
           for (int c = 0; c < dn / 16; ++c) {
             float u[16];
@@ -427,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (mine) {
             p.part_ml[(slot_row + row) * 2] = mm;
-            p.part_ml[(slot_row + row) * 2 + 1] = a0 * l + (has1 ? a1 * bars->l_x[row] : 0.f);
+            p.part_ml[(slot_row + row) * 2 + 1] = l;
           }
         }
         tc_fence_before();
@@ -450,8 +462,97 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ================================================================ broadcast
 constexpr size_t kBcSmemBytes = 1024 + 2 * (size_t)kMaxAgents * kRowBytes +
-                                (size_t)kBcStages * kTileBytes + 2 * (size_t)kTileBytes +
-                                sizeof(BcBars);
+                                (size_t)kBcStages * kQTileBytes + 2 * (size_t)kQTileBytes +
+                                kOnesBytes + sizeof(BcBars);
+
+// Row max over the first kpad columns of a score row (columns >= k masked).
+// 64 columns per TMEM load; kpad (a multiple of 16) may end in a 32- or
+// 16-column remainder.
+__device__ __forceinline__ float bc_row_max(uint32_t s_col, int k, int kpad) {
+  float mx = -INFINITY;
+  int c = 0;
+#pragma unroll 1
+  for (; c + 64 <= kpad; c += 64) {
+    float v[64];
+    tmem_ld64(s_col + c, v);
+    if (c + 64 > k) {
+#pragma unroll
+      for (int e = 0; e < 64; ++e)
+        if (c + e >= k) v[e] = -INFINITY;
+    }
+    mx = max32(*reinterpret_cast<float(*)[32]>(&v[0]),
+               max32(*reinterpret_cast<float(*)[32]>(&v[32]), mx));
+  }
+#pragma unroll 1
+  for (; c < kpad; c += 32) {
+    float v[32];
+    if (c + 32 <= kpad) {
+      tmem_ld32(s_col + c, v);
+    } else {                      // a 16-column remainder
+      float h[16];
+      tmem_ld16(s_col + c, h);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        v[e] = h[e];
+        v[16 + e] = -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (c + e >= k) v[e] = -INFINITY;
+    mx = max32(v, mx);
+  }
+  return mx;
+}
+
+// P = 2^(S*c - m) as bf16 over the first kpad/2 columns (columns >= k give 0).
+__device__ __forceinline__ void bc_row_exp(uint32_t s_col, int k, int kpad, float c_scale,
+                                           float m) {
+  int c = 0;
+#pragma unroll 1
+  for (; c + 64 <= kpad; c += 64) {
+    float v[64];
+    tmem_ld64(s_col + c, v);
+    if (c + 64 > k) {
+#pragma unroll
+      for (int e = 0; e < 64; ++e)
+        if (c + e >= k) v[e] = -INFINITY;
+    }
+    uint32_t pk[16];
+    exp_pack32(*reinterpret_cast<float(*)[32]>(&v[0]), c_scale, -m, pk);
+    tmem_st16u(s_col + c / 2, pk);
+    exp_pack32(*reinterpret_cast<float(*)[32]>(&v[32]), c_scale, -m, pk);
+    tmem_st16u(s_col + c / 2 + 16, pk);
+  }
+#pragma unroll 1
+  for (; c < kpad; c += 32) {
+    float v[32];
+    uint32_t pk[16];
+    if (c + 32 <= kpad) {
+      tmem_ld32(s_col + c, v);
+    } else {
+      float h[16];
+      tmem_ld16(s_col + c, h);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        v[e] = h[e];
+        v[16 + e] = -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (c + e >= k) v[e] = -INFINITY;
+    exp_pack32(v, c_scale, -m, pk);
+    if (c + 32 <= kpad) {
+      tmem_st16u(s_col + c / 2, pk);
+    } else {
+      uint32_t lo[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lo[e] = pk[e];
+      tmem_st8(s_col + c / 2, lo);
+    }
+  }
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     agent_broadcast_tc_kernel(const __grid_constant__ CUtensorMap map_q,
@@ -464,8 +565,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sVA = sA + kMaxAgents * kRowBytes;
   uint8_t* sQ = sVA + kMaxAgents * kRowBytes;
-  uint8_t* sO = sQ + kBcStages * kTileBytes;
-  BcBars* bars = reinterpret_cast<BcBars*>(sO + 2 * kTileBytes);
+  uint8_t* sO = sQ + kBcStages * kQTileBytes;
+  uint8_t* sOnes = sO + 2 * kQTileBytes;
+  BcBars* bars = reinterpret_cast<BcBars*>(sOnes + kOnesBytes);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -499,6 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&map_va);
     prefetch_tensormap(&map_o);
   }
+  fill_ones(sOnes);
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
@@ -508,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   // TMEM: buffer b at column b*256: S over [0, kpad), P (bf16) over [0, kpad/2),
-  // O over [o_col, o_col + dn).
+  // O over [o_col, o_col + dn), l at o_col + dn.
 
   if (warp == 0) {
     if (lane == 0) {
@@ -533,9 +636,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = j % kBcStages;
         if (j >= kBcStages && !mbar_wait(&bars->q_empty[s], ((j / kBcStages) - 1) & 1, abort))
           break;
-        mbar_expect_tx(&bars->q_full[s], kTileBytes);
-        tma_load_3d(sQ + s * kTileBytes, &map_q, &bars->q_full[s], 0,
-                    (int)(t - bh * tps) * kTileRows, (int)bh);
+        mbar_expect_tx(&bars->q_full[s], kQTileBytes);
+        tma_load_3d(sQ + s * kQTileBytes, &map_q, &bars->q_full[s], 0,
+                    (int)(t - bh * tps) * kQTile, (int)bh);
       }
       if (*abort) {
         for (int i = (j > kBcStages ? j - kBcStages : 0); i < j; ++i) {
@@ -551,7 +654,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------- MMA issuer
       const uint32_t idesc_s = idesc_bf16(128, kpad, 0, 0);
       const uint32_t idesc_pv = idesc_bf16(128, dn, 0, 1);
+      const uint32_t idesc_l = idesc_bf16(128, 16, 0, 1);
       const uint32_t sA_addr = smem_u32(sA), sVA_addr = smem_u32(sVA), sQ_addr = smem_u32(sQ);
+      const uint64_t ones_desc = sw128_desc(smem_u32(sOnes), 8192);
       int n_slices = 0;
       long long cur = -1;
       auto slice_of = [&](int j) { return (t_begin + j) / tps; };
@@ -567,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&bars->q_full[s], (j / kBcStages) & 1, abort)) return false;
         tc_fence_after();
         for (int kk = 0; kk < d16; ++kk) {
-          const uint64_t da = sw128_desc(sQ_addr + s * kTileBytes + kk * 32, 16);
+          const uint64_t da = sw128_desc(sQ_addr + s * kQTileBytes + kk * 32, 16);
           const uint64_t db = sw128_desc(sA_addr + kk * 32, 16);
           mma_ss(tmem + b * 256, da, db, idesc_s, kk > 0);
         }
@@ -579,9 +684,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = j & 1;
         if (!mbar_wait(&bars->p_full[b], (j >> 1) & 1, abort)) return false;
         tc_fence_after();
+        const uint32_t o_tm = tmem + b * 256 + o_col;
         for (int kk = 0; kk < kpad / 16; ++kk) {
-          const uint64_t db = sw128_desc(sVA_addr + kk * 2048, 8192);
-          mma_ts(tmem + b * 256 + o_col, tmem + b * 256 + kk * 8, db, idesc_pv, kk > 0);
+          const uint32_t p_tm = tmem + b * 256 + kk * 8;
+          mma_ts(o_tm, p_tm, sw128_desc(sVA_addr + kk * 2048, 8192), idesc_pv, kk > 0);
+          mma_ts(o_tm + dn, p_tm, ones_desc, idesc_l, kk > 0);
         }
         mma_commit(&bars->o_full[b]);
         if (j + 1 == n_tiles || slice_of(j + 1) != slice_of(j)) mma_commit(&bars->ag_empty);
@@ -613,65 +720,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t s_col = tmem + lane_off + g * 256;
     const uint32_t o_tm = s_col + o_col;
-    uint8_t* stage = sO + g * kTileBytes;
+    uint8_t* stage = sO + g * kQTileBytes;
     const bool leader = (warp == 2 + 4 * g) && lane == 0;
     bool ok = true;
     for (int j = g; j < n_tiles; j += 2) {
       const int u = j >> 1;
       const long long t = t_begin + j;
       const long long bh = t / tps;
-      const int q0 = (int)(t - bh * tps) * kTileRows;
+      const int q0 = (int)(t - bh * tps) * kQTile;
       if (ok) ok = warp_wait(&bars->s_full[g], u & 1, abort);
       tc_fence_after();
-      float l = 0.f;
       if (ok) {
-        // pass 1: row max over the k agents
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < kpad / 16; ++c) {
-          float v[16];
-          tmem_ld16(s_col + c * 16, v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (c * 16 + e < p.k) mx = fmaxf(mx, v[e]);
-        }
-        const float m = mx * p.c;
-        // pass 2: P = 2^(S*c - m) (bf16) over the first kpad/2 columns, l = sum P
-#pragma unroll 1
-        for (int c = 0; c < kpad / 16; ++c) {
-          float v[16];
-          tmem_ld16(s_col + c * 16, v);
-          uint32_t pk[8];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x = ex2(fmaf(v[e], p.c, -m));
-            v[e] = (c * 16 + e < p.k) ? x : 0.f;
-            l += v[e];
-          }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-          tmem_st8(s_col + c * 8, pk);
-        }
+        const float m = bc_row_max(s_col, p.k, kpad) * p.c;
+        bc_row_exp(s_col, p.k, kpad, p.c, m);
         tmem_wait_st();
       }
       tc_fence_before();
       mbar_arrive(&bars->p_full[g]);
-      // epilogue: O = (P V_A) / l -> bf16 -> swizzled staging tile -> TMA store
+      // epilogue: O = (P V_A) / (P 1) -> bf16 -> swizzled staging tile -> TMA store
       if (ok) ok = warp_wait(&bars->o_full[g], u & 1, abort);
       tc_fence_after();
       float o[64];
+      float l = 1.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (ok && c < dn / 16) {
-          float v[16];
-          tmem_ld16(o_tm + c * 16, v);
+      for (int c = 0; c < 2; ++c) {
+        if (ok && c * 32 < dn) {
+          float v[32];
+          if (c * 32 + 32 <= dn) {
+            tmem_ld32(o_tm + c * 32, v);
+          } else {
+            float h[16];
+            tmem_ld16(o_tm + c * 32, h);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[c * 16 + e] = v[e];
+            for (int e = 0; e < 16; ++e) {
+              v[e] = h[e];
+              v[16 + e] = 0.f;
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[c * 32 + e] = v[e];
         } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[c * 16 + e] = 0.f;
+          for (int e = 0; e < 32; ++e) o[c * 32 + e] = 0.f;
         }
       }
+      if (ok) l = tmem_ld1(o_tm + dn);
       tc_fence_before();
       mbar_arrive(&bars->o_free[g]);
       const float inv = 1.f / l;
@@ -715,7 +808,7 @@ inline bool tc_supported(int d, int k) { return d >= 8 && d <= 64 && k >= 1 && k
 
 inline void tc_plan_aggregate(long long BH, int N, int k, int sm_count, SplitPlan* plan) {
   (void)k;
-  const int tps = (N + tc::kTileRows - 1) / tc::kTileRows;
+  const int tps = (N + tc::kKeyTile - 1) / tc::kKeyTile;
   const long long total = BH * tps;
   const int ctas = (int)(total < sm_count ? total : sm_count);
   const long long min_per_cta = total / ctas;
@@ -813,7 +906,7 @@ inline cudaError_t tc_launch_aggregate(const void* agents, long long a_bstride, 
   int a_sets = 1;
   const long long BH = (long long)B * H;
   const int box_a = n_agents > 128 ? 256 : 128;
-  if (!make_map_3d(&mk, k, d, N, BH, kTileRows) || !make_map_3d(&mv, v, d, N, BH, kTileRows) ||
+  if (!make_map_3d(&mk, k, d, N, BH, kKeyTile) || !make_map_3d(&mv, v, d, N, BH, kKeyTile) ||
       !make_map_agents(&ma, agents, d, n_agents, H, B, a_bstride, box_a, &a_sets))
     return cudaErrorInvalidValue;
   cudaError_t e = ensure_tc_smem(reinterpret_cast<const void*>(agent_aggregate_tc_kernel),
@@ -843,7 +936,7 @@ inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long l
   int a_sets = 1;
   const long long BH = (long long)B * H;
   const int kpad = round16(n_agents);
-  if (!make_map_3d(&mq, q, d, N, BH, kTileRows) || !make_map_3d(&mo, out, d, N, BH, kTileRows) ||
+  if (!make_map_3d(&mq, q, d, N, BH, kQTile) || !make_map_3d(&mo, out, d, N, BH, kQTile) ||
       !make_map_3d(&mva, va, d, n_agents, BH, kpad) ||
       !make_map_agents(&ma, agents, d, n_agents, H, B, a_bstride, kpad, &a_sets))
     return cudaErrorInvalidValue;
@@ -856,7 +949,7 @@ inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long l
   p.d = d;
   p.k = n_agents;
   p.c = c;
-  p.tiles_per_slice = (N + kTileRows - 1) / kTileRows;
+  p.tiles_per_slice = (N + kQTile - 1) / kQTile;
   p.total_tiles = BH * p.tiles_per_slice;
   p.ctas = (int)(p.total_tiles < sm_count ? p.total_tiles : sm_count);
   agent_broadcast_tc_kernel<<<p.ctas, kThreads, kBcSmemBytes, st>>>(mq, ma, mva, mo, a_sets, p);
