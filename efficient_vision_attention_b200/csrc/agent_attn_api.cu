@@ -13,7 +13,7 @@
 #include <cstdio>
 #include <cstring>
 
-#include "../../include/agent_attn.h"
+#include "agent_attn.h"
 #include "common.cuh"
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
@@ -195,23 +195,28 @@ struct AgentsRef {
 
 template <typename T>
 int launch_pool(const Problem& p, const void* q, float* a_f32, T* a_lowp, cudaStream_t st) {
-  dim3 grid(p.pool_h, (unsigned)p.BH());
-  if (p.BH() > 65535) {
-    // y-dimension limit: launch the slices in chunks
-    for (long long b0 = 0; b0 < p.BH(); b0 += 65535) {
-      const long long nb = (p.BH() - b0 < 65535) ? p.BH() - b0 : 65535;
-      const long long qoff = b0 * (long long)p.N * p.d;
-      const long long aoff = b0 * (long long)p.k * p.d;
-      agent_pool_kernel<T><<<dim3(p.pool_h, (unsigned)nb), kPoolThreads, 0, st>>>(
-          static_cast<const T*>(q) + qoff, a_f32 ? a_f32 + aoff : nullptr,
-          a_lowp ? a_lowp + aoff : nullptr, p.N, p.d, p.grid_h, p.grid_w, p.pool_h, p.pool_w);
-      AA_CUDA(cudaGetLastError());
-    }
-    return AA_OK;
+  const int per = pool_px_per_cta(p.grid_w, p.pool_w, p.d);
+  const int n_chunks = (p.pool_w + per - 1) / per;
+  const int groups = p.d / 8;
+  // token columns a chunk can span: per bins, each at most ceil(G/P) + 1 wide,
+  // processed in windows of pool_window_cols columns
+  int cols = per * ((p.grid_w + p.pool_w - 1) / p.pool_w + 1);
+  if (cols > pool_window_cols(p.d)) cols = pool_window_cols(p.d);
+  const size_t smem = (size_t)cols * groups * 8 * sizeof(float);
+  static std::atomic<int> flags[kMaxDevices];
+  int rc = ensure_smem(agent_pool_kernel<T>, smem, flags);
+  if (rc != AA_OK) return rc;
+  const long long grid_x = (long long)p.pool_h * n_chunks;
+  if (grid_x > 0x7fffffffLL) return AA_ERR_SHAPE;
+  for (long long b0 = 0; b0 < p.BH(); b0 += 65535) {     // grid.y limit: slices in chunks
+    const long long nb = (p.BH() - b0 < 65535) ? p.BH() - b0 : 65535;
+    const long long qoff = b0 * (long long)p.N * p.d;
+    const long long aoff = b0 * (long long)p.k * p.d;
+    agent_pool_kernel<T><<<dim3((unsigned)grid_x, (unsigned)nb), kPoolThreads, smem, st>>>(
+        static_cast<const T*>(q) + qoff, a_f32 ? a_f32 + aoff : nullptr,
+        a_lowp ? a_lowp + aoff : nullptr, p.N, p.d, p.grid_h, p.grid_w, p.pool_h, p.pool_w, per);
+    AA_CUDA(cudaGetLastError());
   }
-  agent_pool_kernel<T><<<grid, kPoolThreads, 0, st>>>(static_cast<const T*>(q), a_f32, a_lowp, p.N, p.d,
-                                             p.grid_h, p.grid_w, p.pool_h, p.pool_w);
-  AA_CUDA(cudaGetLastError());
   return AA_OK;
 }
 
@@ -231,10 +236,10 @@ int launch_simt_attend(const SimtAttendArgs& args, long long BH, cudaStream_t st
 template <typename T>
 int launch_merge(const Problem& p, const Scratch& s, char* ws, float* va_f32, T* va_lowp,
                  cudaStream_t st) {
-  const long long rows = p.BH() * p.k;
-  const long long blocks = (rows + 7) / 8;
+  const long long work = p.BH() * p.k * (p.d / 4);
+  const long long blocks = (work + kMergeThreads - 1) / kMergeThreads;
   if (blocks > 0x7fffffffLL) return AA_ERR_SHAPE;
-  agent_merge_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(
+  agent_merge_kernel<T><<<(unsigned)blocks, kMergeThreads, 0, st>>>(
       reinterpret_cast<const float*>(ws + s.pu_off), reinterpret_cast<const float*>(ws + s.pml_off),
       s.plan, p.BH(), p.k, p.d, va_f32, va_lowp);
   AA_CUDA(cudaGetLastError());

@@ -15,91 +15,110 @@
 namespace aa {
 
 // ----------------------------------------------------------------- pooling
-// One CTA per (slice bh, agent row py).  Work item = (px, 8-channel group);
-// the bin's grid rows are spread over up to kPoolThreads / items threads, each
-// summing its rows' bin columns with 16-byte loads, eight in flight, and the
-// row partials are reduced through shared memory.  Small CTAs (4 per SM) keep
-// every CTA of the usual shapes resident at once.  Sums are fp32; the divisor
-// is the bin's own token count.  Writes fp32 and/or low-precision agents.
-constexpr int kPoolThreads = 256;
+// One CTA per (slice bh, agent row py, chunk of agent columns px).  Phase 1:
+// one thread per (token column x of the chunk, 8-channel group) sums that
+// column over the bin's grid rows; consecutive threads read consecutive 16
+// bytes, and a thread's loads (one per row, eight in flight) need a single
+// trip to memory.  Phase 2: one thread per (px, channel group) adds its bin's
+// column sums from shared memory and divides by the bin's token count.  Sums
+// are fp32.  Writes fp32 and/or low-precision agents.
+constexpr int kPoolThreads = 512;
+
+// Agent columns per CTA, so that the chunk's token columns x channel groups
+// fit in one pass of the CTA's threads (at least one agent column).
+__host__ __forceinline__ int pool_px_per_cta(int grid_w, int pool_w, int d) {
+  const int groups = d / 8;
+  const int bin_w = (grid_w + pool_w - 1) / pool_w + 1;     // widest bin (with overlap)
+  int per = kPoolThreads / (bin_w * groups);
+  if (per < 1) per = 1;
+  if (per > pool_w) per = pool_w;
+  return per;
+}
+
+// Token columns per shared-memory window (64 KB of column sums).
+__host__ __device__ __forceinline__ int pool_window_cols(int d) { return 65536 / ((d / 8) * 32); }
 
 template <typename T>
-__global__ void __launch_bounds__(kPoolThreads, 4) agent_pool_kernel(const T* __restrict__ q,
+__global__ void __launch_bounds__(kPoolThreads) agent_pool_kernel(const T* __restrict__ q,
                                                                   float* __restrict__ a_f32,
                                                                   T* __restrict__ a_lowp, int N,
                                                                   int d, int grid_h, int grid_w,
-                                                                  int pool_h, int pool_w) {
-  __shared__ float red[kPoolThreads * 8];
-  const int py = blockIdx.x;
+                                                                  int pool_h, int pool_w,
+                                                                  int px_per_cta) {
+  extern __shared__ float colsum[];          // [token column of the window][group][8]
+  const int n_chunks = (pool_w + px_per_cta - 1) / px_per_cta;
+  const int py = blockIdx.x / n_chunks;
+  const int px0 = (blockIdx.x % n_chunks) * px_per_cta;
+  const int px1 = min(pool_w, px0 + px_per_cta);
   const long long bh = blockIdx.y;
   const int y0 = bin_start(py, grid_h, pool_h), y1 = bin_end(py, grid_h, pool_h);
+  const int xs = bin_start(px0, grid_w, pool_w), xe = bin_end(px1 - 1, grid_w, pool_w);
   const int groups = d >> 3;
-  const int items = pool_w * groups;
   const int rows = y1 - y0;
-  int ysplit = (int)blockDim.x / items;
-  if (ysplit < 1) ysplit = 1;
-  if (ysplit > rows) ysplit = rows;
   const T* qs = q + bh * (long long)N * d;
-  const long long n_agents = (long long)pool_h * pool_w;
+  const long long row_stride = (long long)grid_w * d;
+  const int wcols = pool_window_cols(d);
 
-  for (int base = 0; base < items * ysplit; base += blockDim.x) {
-    const int t = base + threadIdx.x;
-    float acc[8];
+  // phase-2 item of this thread: (px, group); there are at most kPoolThreads
+  const int items2 = (px1 - px0) * groups;
+  const int px = px0 + (int)threadIdx.x / groups, g2 = (int)threadIdx.x % groups;
+  const bool has2 = (int)threadIdx.x < items2;
+  const int bx0 = has2 ? bin_start(px, grid_w, pool_w) : 0;
+  const int bx1 = has2 ? bin_end(px, grid_w, pool_w) : 0;
+  float acc2[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    int item = -1, ys = 0;
-    if (t < items * ysplit) {
-      item = t % items;
-      ys = t / items;
-      const int px = item / groups, g = item % groups;
-      const int x0 = bin_start(px, grid_w, pool_w), x1 = bin_end(px, grid_w, pool_w);
-      for (int y = y0 + ys; y < y1; y += ysplit) {
-        const T* row = qs + ((long long)y * grid_w + x0) * d + g * 8;
-        const int w = x1 - x0;
-        int x = 0;
-        for (; x + 8 <= w; x += 8) {       // eight independent 16-byte loads in flight
-          uint4 raw[8];
+  for (int i = 0; i < 8; ++i) acc2[i] = 0.f;
+
+  for (int wx = xs; wx < xe; wx += wcols) {
+    const int we = min(xe, wx + wcols);
+    const int items = (we - wx) * groups;
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+      const int x = wx + it / groups, g = it % groups;
+      const T* col = qs + ((long long)y0 * grid_w + x) * d + g * 8;
+      float acc[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) raw[u] = load16(row + (long long)(x + u) * d);
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      int y = 0;
+      for (; y + 8 <= rows; y += 8) {      // eight independent 16-byte loads in flight
+        uint4 raw[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            float v[8];
-            unpack8(raw[u], row + (long long)(x + u) * d, v);
+        for (int u = 0; u < 8; ++u) raw[u] = load16(col + (y + u) * row_stride);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] += v[i];
-          }
-        }
-        for (; x < w; ++x) {
+        for (int u = 0; u < 8; ++u) {
           float v[8];
-          load8(row + (long long)x * d, v);
+          unpack8(raw[u], col + (y + u) * row_stride, v);
 #pragma unroll
           for (int i = 0; i < 8; ++i) acc[i] += v[i];
         }
       }
-    }
-    if (ysplit > 1) {
+      for (; y < rows; ++y) {
+        float v[8];
+        load8(col + y * row_stride, v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) red[threadIdx.x * 8 + i] = acc[i];
-      __syncthreads();
-      if (item >= 0 && ys == 0) {
-        for (int s2 = 1; s2 < ysplit; ++s2) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] += red[(threadIdx.x + s2 * items) * 8 + i];
-        }
+        for (int i = 0; i < 8; ++i) acc[i] += v[i];
       }
-      __syncthreads();
-    }
-    if (item >= 0 && ys == 0) {
-      const int px = item / groups, g = item % groups;
-      const int x0 = bin_start(px, grid_w, pool_w), x1 = bin_end(px, grid_w, pool_w);
-      const float inv = 1.f / (float)((y1 - y0) * (x1 - x0));
-      const long long off = (bh * n_agents + (long long)py * pool_w + px) * d + g * 8;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float m = acc[i] * inv;
-        if (a_f32) a_f32[off + i] = m;
-        if (a_lowp) a_lowp[off + i] = from_f32<T>(m);
+      for (int i = 0; i < 8; ++i) colsum[it * 8 + i] = acc[i];
+    }
+    __syncthreads();
+    if (has2) {
+      for (int x = max(bx0, wx); x < min(bx1, we); ++x) {
+        const float* cs = colsum + ((x - wx) * groups + g2) * 8;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc2[i] += cs[i];
       }
+    }
+    __syncthreads();
+  }
+  if (has2) {
+    const long long n_agents = (long long)pool_h * pool_w;
+    const float inv = 1.f / (float)((y1 - y0) * (bx1 - bx0));
+    const long long off = (bh * n_agents + (long long)py * pool_w + px) * d + g2 * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float m = acc2[i] * inv;
+      if (a_f32) a_f32[off + i] = m;
+      if (a_lowp) a_lowp[off + i] = from_f32<T>(m);
     }
   }
 }
@@ -250,72 +269,68 @@ __global__ void __launch_bounds__(kSimtThreads) simt_attend_kernel(SimtAttendArg
 }
 
 // ------------------------------------------------------------------ merge
-// One warp per (slice, agent row): V_A = sum_s 2^(m_s - M) U_s / sum_s 2^(m_s - M) l_s.
-// Lane s owns split s's weight (computed once); the weights are broadcast by
-// shuffles while the lanes sweep the d columns of every split's partial row.
+// V_A = sum_s 2^(m_s - M) U_s / sum_s 2^(m_s - M) l_s.  One thread per
+// (slice, agent row, 4-column group): it loads the row's (m_s, l_s) and its
+// four columns of every split's U at once (the loads are independent, so one
+// trip to memory), then combines them.  Up to kMergeUnroll splits per pass.
+constexpr int kMergeUnroll = 16;
+constexpr int kMergeThreads = 256;
+
 template <typename T>
-__global__ void __launch_bounds__(256) agent_merge_kernel(const float* __restrict__ part_u,
-                                                          const float* __restrict__ part_ml,
-                                                          SplitPlan plan, long long BH,
-                                                          int n_agents, int d,
-                                                          float* __restrict__ va_f32,
-                                                          T* __restrict__ va_lowp) {
-  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= BH * n_agents) return;
+__global__ void __launch_bounds__(kMergeThreads) agent_merge_kernel(
+    const float* __restrict__ part_u, const float* __restrict__ part_ml, SplitPlan plan,
+    long long BH, int n_agents, int d, float* __restrict__ va_f32, T* __restrict__ va_lowp) {
+  const int quads = d >> 2;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= BH * n_agents * quads) return;
+  const int cq = (int)(idx % quads);
+  const long long row = idx / quads;              // bh * n_agents + j
   const long long bh = row / n_agents;
   const int j = (int)(row % n_agents);
   const int n_splits = splits_of_slice(plan, bh);
   const long long slot0 = bh * plan.slots;
+  const long long split_stride = (long long)n_agents;      // rows between consecutive splits
+  const float* ml0 = part_ml + ((slot0)*n_agents + j) * 2;
+  const float* u0 = part_u + ((slot0)*n_agents + j) * (long long)d + cq * 4;
   float mx = -INFINITY;
-  for (int s = lane; s < n_splits; s += 32)
-    mx = fmaxf(mx, part_ml[((slot0 + s) * n_agents + j) * 2]);
+  for (int s0 = 0; s0 < n_splits; s0 += kMergeUnroll) {
+    float m[kMergeUnroll];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f, den = 0.f;
-  for (int s0 = 0; s0 < n_splits; s0 += 32) {
-    float w = 0.f;
-    if (s0 + lane < n_splits) {
-      const float* ml = part_ml + ((slot0 + s0 + lane) * n_agents + j) * 2;
-      w = exp2f(ml[0] - mx);
-      den += w * ml[1];
+    for (int a = 0; a < kMergeUnroll; ++a)
+      m[a] = (s0 + a < n_splits) ? ml0[(s0 + a) * split_stride * 2] : -INFINITY;
+#pragma unroll
+    for (int a = 0; a < kMergeUnroll; ++a) mx = fmaxf(mx, m[a]);
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.f;
+  for (int s0 = 0; s0 < n_splits; s0 += kMergeUnroll) {
+    float2 ml[kMergeUnroll];
+    float4 u[kMergeUnroll];
+#pragma unroll
+    for (int a = 0; a < kMergeUnroll; ++a) {
+      const bool ok = s0 + a < n_splits;
+      ml[a] = ok ? *reinterpret_cast<const float2*>(ml0 + (s0 + a) * split_stride * 2)
+                 : make_float2(-INFINITY, 0.f);
+      u[a] = ok ? *reinterpret_cast<const float4*>(u0 + (s0 + a) * split_stride * d)
+                : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const int cnt = min(32, n_splits - s0);
-    const long long stride = (long long)n_agents * d;      // between consecutive splits
-    const float* base = part_u + ((slot0 + s0) * n_agents + j) * (long long)d;
-    for (int s = 0; s < cnt; s += 4) {                      // four splits' loads in flight
-      float u[4][4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int c = lane + 32 * q;
-          u[a][q] = (s + a < cnt && c < d) ? base[(s + a) * stride + c] : 0.f;
-        }
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const float ws = __shfl_sync(0xffffffffu, w, (s + a) & 31);
-        const float wa = (s + a < cnt) ? ws : 0.f;
-        acc0 = fmaf(wa, u[a][0], acc0);
-        acc1 = fmaf(wa, u[a][1], acc1);
-        acc2 = fmaf(wa, u[a][2], acc2);
-        acc3 = fmaf(wa, u[a][3], acc3);
-      }
+    for (int a = 0; a < kMergeUnroll; ++a) {
+      const float w = (s0 + a < n_splits) ? exp2f(ml[a].x - mx) : 0.f;
+      den = fmaf(w, ml[a].y, den);
+      acc.x = fmaf(w, u[a].x, acc.x);
+      acc.y = fmaf(w, u[a].y, acc.y);
+      acc.z = fmaf(w, u[a].z, acc.z);
+      acc.w = fmaf(w, u[a].w, acc.w);
     }
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
   const float inv = 1.f / den;
-  const float accs[4] = {acc0, acc1, acc2, acc3};
+  const float v[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+  const long long o = row * d + cq * 4;
+  if (va_f32) *reinterpret_cast<float4*>(va_f32 + o) = make_float4(v[0], v[1], v[2], v[3]);
+  if (va_lowp) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int c = lane + 32 * q;
-    if (c < d) {
-      const float v = accs[q] * inv;
-      const long long o = row * d + c;
-      if (va_f32) va_f32[o] = v;
-      if (va_lowp) va_lowp[o] = from_f32<T>(v);
-    }
+    for (int i = 0; i < 4; ++i) va_lowp[o + i] = from_f32<T>(v[i]);
   }
 }
 

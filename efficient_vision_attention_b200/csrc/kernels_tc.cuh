@@ -8,31 +8,33 @@
 //  agent_aggregate_tc  rows = agents (M = 128 per TMEM tile, 1 or 2 tiles),
 //                      columns = keys streamed in tiles of 64 through an
 //                      8-deep TMA ring of K and V tiles.  S = A K^T (SS MMA),
-//                      online softmax in registers (one thread per agent row),
-//                      P written back into TMEM as bf16 over S, U += P V (TS
-//                      MMA, V as an MN-major operand) and l += P 1 (TS MMA
-//                      against a tile of ones: the row sums come from the
-//                      tensor core, summed from the same bf16 P).  Score tiles
-//                      are double-buffered per softmax group, so the tensor
-//                      core computes tile i+1 while the group works on tile i.
-//                      A persistent grid cuts the key tiles of all slices into
-//                      equal contiguous ranges (one range per CTA, one CTA per
-//                      SM); each CTA writes one partial (U, running max,
-//                      running sum) per slice it touches, merged afterwards by
-//                      agent_merge_kernel.
+//                      online softmax in registers, P written back into TMEM
+//                      as bf16 over S, U += P V (TS MMA, V as an MN-major
+//                      operand); the row sums are accumulated in registers.
+//                      Score tiles are double-buffered per softmax group, so
+//                      the tensor core computes tile i+1 while the group works
+//                      on tile i.  A persistent grid cuts the key tiles of all
+//                      slices into equal contiguous ranges (one range per CTA,
+//                      one CTA per SM); each CTA writes one partial (U,
+//                      running max, running sum) per slice it touches, merged
+//                      afterwards by agent_merge_kernel.
 //  agent_broadcast_tc  rows = queries streamed in tiles of 128 (TMA ring),
 //                      columns = the k agents, resident in shared memory with
 //                      V_A for the whole slice.  S = Q A^T, row softmax over k
-//                      in registers, O = P V_A and l = P 1 on the tensor core,
-//                      1/l applied in the epilogue, O staged in shared memory
-//                      and written with TMA stores.
+//                      in registers, O = P V_A on the tensor core, 1/l applied
+//                      in the epilogue, O staged in shared memory and written
+//                      with TMA stores.
 //
-// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and
-// issues the MMAs (one thread), warps 2-5 and 6-9 are two softmax groups of
-// 128 threads (thread = TMEM lane = row) working on alternating tiles (or, for
-// k > 128 in the aggregation, on the two 128-agent halves).  Every wait is
-// bounded; a wait that gives up makes its CTA skip the rest of its work and
-// raises the device watchdog.
+// Warp roles (608 threads): warp 0 issues TMA loads; warps 1 and 2 each issue
+// the MMAs of one softmax group (one thread each: a single issuing thread
+// spends about 57 cycles per tcgen05.mma, so two issuers double the MMA rate
+// and keep the groups independent); warps 3-10 and 11-18 are the two softmax
+// groups, working on alternating tiles (or, for k > 128 in the aggregation,
+// on the two 128-agent halves).  In a group, TMEM lane = row, and each row
+// has two threads (two warps share a lane quadrant) that split its columns
+// and exchange partial row maxima and sums through shared memory.  Every wait
+// is bounded; a wait that gives up makes its CTA skip the rest of its work
+// and raises the device watchdog.
 #pragma once
 
 #include <atomic>
@@ -44,7 +46,9 @@ namespace aa {
 
 namespace tc {
 
-constexpr int kThreads = 320;
+constexpr int kSoftmaxThreads = 256;           // per softmax group: 8 warps, two per lane quadrant
+constexpr int kFirstSoftmaxWarp = 3;
+constexpr int kThreads = kFirstSoftmaxWarp * 32 + 2 * kSoftmaxThreads;
 constexpr int kRowBytes = 128;               // one swizzled 128-byte row per token (d <= 64 bf16)
 constexpr int kKeyTile = 64;                 // keys per aggregation tile
 constexpr int kQTile = 128;                  // queries per broadcast tile (MMA M)
@@ -53,7 +57,6 @@ constexpr int kQTileBytes = kQTile * kRowBytes;
 constexpr int kAggStages = 8;
 constexpr int kBcStages = 4;
 constexpr int kMaxAgents = 256;
-constexpr int kOnesBytes = 16 * kRowBytes;   // 16 rows of bf16 ones (row-sum operand)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale only when the max grows by > 2^8
 
 struct AggParams {
@@ -80,17 +83,23 @@ struct AggBars {
   uint64_t a_full, a_empty;
   uint64_t s_full[2][2], p_full[2][2], pv_done[2][2];   // [group][score buffer]
   uint64_t x_pub, x_done;    // group 1 -> group 0 hand-over per segment (k <= 128)
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
   float m_x[128];
+  float l_x[2][2][128];      // [group][half][row]: partial row sums at a segment end
+  float xmax[2][2][2][128];  // [group][half][tile parity][row]: partial row maxima
 };
 
 struct BcBars {
   uint64_t q_full[kBcStages], q_empty[kBcStages];
   uint64_t ag_full, ag_empty;
   uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
+  float xmax[2][2][2][128];  // [group][half][tile parity][row]: partial row maxima
+  float xsum[2][2][2][128];  // [group][half][tile parity][row]: partial row sums
 };
 
 __host__ __device__ constexpr int round16(int x) { return (x + 15) & ~15; }
@@ -105,18 +114,17 @@ __device__ __forceinline__ void agent_coords(long long bh, int H, int b_sets, in
   *b = b_sets > 1 ? (int)(bh / H) : 0;
 }
 
-// Fill the row-sum operand (16 rows x 128 bytes of bf16 1.0) and make it
-// visible to the tensor core.
-__device__ __forceinline__ void fill_ones(uint8_t* ones) {
-  for (int i = threadIdx.x; i < kOnesBytes / 4; i += blockDim.x)
-    reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
-  fence_proxy_async_smem();
+// Bounded wait for an issuer's last commit before TMEM is released.
+__device__ __forceinline__ void drain_commits(uint64_t* bar) {
+  mma_commit(bar);
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, 0) && globaltimer() - t0 < kWaitLimitNs) {
+  }
 }
 
 // ============================================================== aggregation
 constexpr size_t kAggSmemBytes = 1024 + (size_t)kMaxAgents * kRowBytes +
-                                 2 * (size_t)kAggStages * kKTileBytes + kOnesBytes +
-                                 sizeof(AggBars);
+                                 2 * (size_t)kAggStages * kKTileBytes + sizeof(AggBars);
 
 __global__ void __launch_bounds__(kThreads, 1)
     agent_aggregate_tc_kernel(const __grid_constant__ CUtensorMap map_k,
@@ -128,8 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sK = sA + kMaxAgents * kRowBytes;
   uint8_t* sV = sK + kAggStages * kKTileBytes;
-  uint8_t* sOnes = sV + kAggStages * kKTileBytes;
-  AggBars* bars = reinterpret_cast<AggBars*>(sOnes + kOnesBytes);
+  AggBars* bars = reinterpret_cast<AggBars*>(sV + kAggStages * kKTileBytes);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -139,30 +146,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tps = p.tiles_per_slice;
   const bool two = p.k > 128;                 // two 128-row agent tiles
   const int d16 = (p.d + 15) >> 4;            // K steps of S = A K^T
-  const int dn = d16 * 16;                    // N of U += P V; l sits in column dn
+  const int dn = d16 * 16;                    // N of U += P V
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAggStages; ++s) {
       mbar_init(&bars->full[s], 1);
-      mbar_init(&bars->empty[s], 1);
+      mbar_init(&bars->empty[s], two ? 2 : 1);   // released by every group that used the tile
     }
     mbar_init(&bars->a_full, 1);
-    mbar_init(&bars->a_empty, 1);
-    for (int g = 0; g < 2; ++g)
+    mbar_init(&bars->a_empty, 2);                 // both issuers finish the segment
+    for (int g = 0; g < 2; ++g) {
       for (int b = 0; b < 2; ++b) {
         mbar_init(&bars->s_full[g][b], 1);
-        mbar_init(&bars->p_full[g][b], 128);
+        mbar_init(&bars->p_full[g][b], kSoftmaxThreads);
         mbar_init(&bars->pv_done[g][b], 1);
       }
-    mbar_init(&bars->x_pub, 128);
-    mbar_init(&bars->x_done, 128);
+      mbar_init(&bars->drain[g], 1);
+    }
+    mbar_init(&bars->x_pub, kSoftmaxThreads);
+    mbar_init(&bars->x_done, kSoftmaxThreads);
     bars->abort = 0;
     mbar_fence_init();
     prefetch_tensormap(&map_k);
     prefetch_tensormap(&map_v);
     prefetch_tensormap(&map_a);
   }
-  fill_ones(sOnes);
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
@@ -172,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   // TMEM columns: score buffer b of group g at g*128 + b*64 (P over its first
-  // 32 columns), U of group g at 256 + g*128 (dn columns), l at 256 + g*128 + dn.
+  // 32 columns), U of group g at 256 + g*128 (dn columns).
 
   if (warp == 0) {
     if (lane == 0) {
@@ -213,17 +221,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp < kFirstSoftmaxWarp) {
     if (lane == 0) {
-      // ------------------------------------------------------- MMA issuer
+      // ------------------------------------- MMA issuer of group g = warp - 1
+      const int g = warp - 1;
       const uint32_t idesc_s = idesc_bf16(128, kKeyTile, 0, 0);
       const uint32_t idesc_pv = idesc_bf16(128, dn, 0, 1);
-      const uint32_t idesc_l = idesc_bf16(128, 16, 0, 1);
-      const uint32_t sA_addr = smem_u32(sA), sK_addr = smem_u32(sK), sV_addr = smem_u32(sV);
-      const uint64_t ones_desc = sw128_desc(smem_u32(sOnes), 8192);
+      const uint32_t sA_addr = smem_u32(sA) + (two ? g : 0) * 128 * kRowBytes;
+      const uint32_t sK_addr = smem_u32(sK), sV_addr = smem_u32(sV);
+      const uint32_t u_tm = tmem + 256 + g * 128;
       long long it0 = 0;
       int seg = 0;
-      int cnt_s[2] = {0, 0}, cnt_p[2] = {0, 0};
+      int cnt_s = 0, cnt_p = 0;
       bool ok = true;
       for (long long t = t_begin; t < t_end && ok; ++seg) {
         const long long bh = t / tps;
@@ -231,82 +240,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = (int)(seg_end - t);
         if (!mbar_wait(&bars->a_full, seg & 1, abort)) break;
         tc_fence_after();
-        bool first[2] = {true, true};
+        bool first = true;
         auto issue_s = [&](int i) -> bool {
           const long long itg = it0 + i;
           const int s = (int)(itg % kAggStages);
           if (!mbar_wait(&bars->full[s], (uint32_t)(itg / kAggStages) & 1, abort)) return false;
+          const int J = cnt_s, b = J & 1;
+          if (J >= 2 && !mbar_wait(&bars->pv_done[g][b], (uint32_t)((J >> 1) - 1) & 1, abort))
+            return false;           // the buffer's previous P has been consumed
           tc_fence_after();
-          for (int g = 0; g < 2; ++g) {
-            if (!two && (i & 1) != g) continue;
-            const int J = cnt_s[g], b = J & 1;
-            if (J >= 2) {   // the buffer's previous P has been consumed
-              if (!mbar_wait(&bars->pv_done[g][b], (uint32_t)((J >> 1) - 1) & 1, abort))
-                return false;
-              tc_fence_after();
-            }
-            const int mt = two ? g : 0;
-            const uint32_t d_tm = tmem + g * 128 + b * 64;
-            for (int kk = 0; kk < d16; ++kk) {
-              const uint64_t da = sw128_desc(sA_addr + mt * 128 * kRowBytes + kk * 32, 16);
-              const uint64_t db = sw128_desc(sK_addr + s * kKTileBytes + kk * 32, 16);
-              mma_ss(d_tm, da, db, idesc_s, kk > 0);
-            }
-            mma_commit(&bars->s_full[g][b]);
-            ++cnt_s[g];
+          const uint32_t d_tm = tmem + g * 128 + b * 64;
+          for (int kk = 0; kk < d16; ++kk) {
+            const uint64_t da = sw128_desc(sA_addr + kk * 32, 16);
+            const uint64_t db = sw128_desc(sK_addr + s * kKTileBytes + kk * 32, 16);
+            mma_ss(d_tm, da, db, idesc_s, kk > 0);
           }
+          mma_commit(&bars->s_full[g][b]);
+          ++cnt_s;
           return true;
         };
         auto issue_pv = [&](int i) -> bool {
           const long long itg = it0 + i;
           const int s = (int)(itg % kAggStages);
-          for (int g = 0; g < 2; ++g) {
-            if (!two && (i & 1) != g) continue;
-            const int J = cnt_p[g], b = J & 1;
-            if (!mbar_wait(&bars->p_full[g][b], (uint32_t)(J >> 1) & 1, abort)) return false;
-            tc_fence_after();
-            const uint32_t p_tm = tmem + g * 128 + b * 64;
-            const uint32_t u_tm = tmem + 256 + g * 128;
-            for (int kk = 0; kk < kKeyTile / 16; ++kk) {
-              const uint32_t acc = (!first[g] || kk > 0) ? 1u : 0u;
-              const uint64_t dv = sw128_desc(sV_addr + s * kKTileBytes + kk * 2048, 8192);
-              mma_ts(u_tm, p_tm + kk * 8, dv, idesc_pv, acc);
-              mma_ts(u_tm + dn, p_tm + kk * 8, ones_desc, idesc_l, acc);
-            }
-            first[g] = false;
-            mma_commit(&bars->pv_done[g][b]);
-            ++cnt_p[g];
+          const int J = cnt_p, b = J & 1;
+          if (!mbar_wait(&bars->p_full[g][b], (uint32_t)(J >> 1) & 1, abort)) return false;
+          tc_fence_after();
+          const uint32_t p_tm = tmem + g * 128 + b * 64;
+          for (int kk = 0; kk < kKeyTile / 16; ++kk) {
+            const uint64_t dv = sw128_desc(sV_addr + s * kKTileBytes + kk * 2048, 8192);
+            mma_ts(u_tm, p_tm + kk * 8, dv, idesc_pv, (!first || kk > 0) ? 1u : 0u);
           }
+          first = false;
+          mma_commit(&bars->pv_done[g][b]);
           mma_commit(&bars->empty[s]);
+          ++cnt_p;
           return true;
         };
-        // one tile of look-ahead: S of tile i is issued before P V of tile i-1
-        for (int i = 0; i < n && ok; ++i) {
-          ok = issue_s(i);
-          if (ok && i > 0) ok = issue_pv(i - 1);
+        // this group's tiles of the segment: all of them for two agent tiles,
+        // else every other one; one tile of look-ahead (S of the next tile is
+        // issued before P V of the current one)
+        const int i0 = two ? 0 : g, step = two ? 1 : 2;
+        // In two-agent-tile mode both groups take every key tile; start group 1
+        // one softmax behind group 0 so their SFU-bound phases interleave.
+        if (two && g == 1 && seg == 0 && n > 0 &&
+            !mbar_wait(&bars->p_full[0][0], 0, abort))
+          ok = false;
+        if (ok && i0 < n) ok = issue_s(i0);
+        for (int i = i0; i < n && ok; i += step) {
+          if (i + step < n) ok = issue_s(i + step);
+          if (ok) ok = issue_pv(i);
         }
-        if (ok) ok = issue_pv(n - 1);
         mma_commit(&bars->a_empty);
         it0 += n;
         t = seg_end;
       }
-      // Let every MMA issued so far finish before TMEM is released.
-      mma_commit(&bars->a_full);   // a_full is no longer waited on: use it as a drain marker
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(&bars->a_full, (uint32_t)seg & 1) && globaltimer() - t0 < kWaitLimitNs) {
-      }
+      drain_commits(&bars->drain[g]);
     }
   } else {
     // ---------------------------------------------------- softmax groups
     // Every thread walks the same segments and tiles whatever happens; after a
     // failed (timed-out) wait it only skips work, so no barrier is left short.
-    const int g = (warp - 2) >> 2;            // group 0: warps 2-5, group 1: warps 6-9
+    const int sw = warp - kFirstSoftmaxWarp;  // 0..15
+    const int g = sw >> 3;                    // group 0: warps 3-10, group 1: warps 11-18
+    const int hf = (sw >> 2) & 1;             // column half of the row this thread owns
     const int quad = warp & 3;                // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;         // TMEM lane = row of the 128-row tile
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t u_col = tmem + lane_off + 256 + g * 128;
     const int agent = (two ? g * 128 : 0) + row;
     const bool warp_active = (two ? g * 128 : 0) + quad * 32 < p.k;
+    const int nch_u = dn / 16;
     int J = 0, seg = 0;
     bool ok = true;
     for (long long t = t_begin; t < t_end; ++seg) {
@@ -314,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long seg_end = min(t_end, (bh + 1) * tps);
       const int n = (int)(seg_end - t);
       const int n_mine = two ? n : (g == 0 ? (n + 1) / 2 : n / 2);
-      float m = -INFINITY;
+      float m = -INFINITY, l = 0.f;             // running max (log2 units) and this half's sum
       bool first = true;
       for (int i = 0; i < n; ++i) {
         if (!two && (i & 1) != g) continue;
@@ -323,31 +326,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int valid = min(kKeyTile, p.N - (int)(t + i - bh * tps) * kKeyTile);
         if (ok) ok = warp_wait(&bars->s_full[g][b], (uint32_t)(J >> 1) & 1, abort);
         tc_fence_after();
+        float v[32];
         if (ok && warp_active) {
-          float v[64];
-          tmem_ld64(s_col, v);
+          tmem_ld32(s_col + hf * 32, v);
           if (valid < kKeyTile) {               // ragged last tile: mask the missing keys
 #pragma unroll
-            for (int e = 0; e < 64; ++e)
-              if (e >= valid) v[e] = -INFINITY;
+            for (int e = 0; e < 32; ++e)
+              if (hf * 32 + e >= valid) v[e] = -INFINITY;
           }
-          float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
-          float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
-          const float mt = max32(v1, max32(v0, -INFINITY)) * p.c;
+          bars->xmax[g][hf][b][row] = max32(v, -INFINITY);
+        }
+        named_barrier(1 + g, kSoftmaxThreads);
+        if (ok && warp_active) {
+          const float mt =
+              fmaxf(bars->xmax[g][0][b][row], bars->xmax[g][1][b][row]) * p.c;
           if (first) {
             m = mt;
             first = false;
           } else if (__any_sync(0xffffffffu, mt > m + kRescaleThreshold)) {
             // the running max grew a lot: once the previous P V has landed,
-            // rescale U and l by 2^(m_old - m_new)
+            // rescale U and l by 2^(m_old - m_new) (each half takes alternate chunks)
             ok = warp_wait(&bars->pv_done[g][(J - 1) & 1], (uint32_t)((J - 1) >> 1) & 1, abort);
             tc_fence_after();
             if (ok) {
               const float m_new = fmaxf(m, mt);
               const float alpha = ex2(m - m_new);
               m = m_new;
+              l *= alpha;
 #pragma unroll 1
-              for (int c = 0; c < dn / 16 + 1; ++c) {
+              for (int c = hf; c < nch_u; c += 2) {
                 float u[16];
                 tmem_ld16(u_col + c * 16, u);
 #pragma unroll
@@ -358,10 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (ok) {
             uint32_t pk[16];
-            exp_pack32(v0, p.c, -m, pk);
-            tmem_st16u(s_col, pk);
-            exp_pack32(v1, p.c, -m, pk);
-            tmem_st16u(s_col + 16, pk);
+            l += exp_pack32(v, p.c, -m, pk);
+            tmem_st16u(s_col + hf * 16, pk);
             tmem_wait_st();
           }
         }
@@ -375,13 +380,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (n_mine > 0 && ok)
         ok = warp_wait(&bars->pv_done[g][(J - 1) & 1], (uint32_t)((J - 1) >> 1) & 1, abort);
       tc_fence_after();
+      bars->l_x[g][hf][row] = l;
+      if (hf == 0 && g == 1) bars->m_x[row] = m;
+      named_barrier(1 + g, kSoftmaxThreads);
       if (two) {
         if (ok && warp_active) {            // warp-uniform: the TMEM loads are warp-collective
           const bool mine = agent < p.k;
-          const float l = tmem_ld1(u_col + dn);
           float* dst = p.part_u + (slot_row + agent) * p.d;
 #pragma unroll 1
-          for (int c = 0; c < dn / 16; ++c) {
+          for (int c = hf; c < nch_u; c += 2) {
             float u[16];
             tmem_ld16(u_col + c * 16, u);
 #pragma unroll
@@ -390,16 +397,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<float4*>(dst + c * 16 + e) =
                     make_float4(u[e], u[e + 1], u[e + 2], u[e + 3]);
           }
-          if (mine) {
+          if (hf == 0 && mine) {
             p.part_ml[(slot_row + agent) * 2] = m;
-            p.part_ml[(slot_row + agent) * 2 + 1] = l;
+            p.part_ml[(slot_row + agent) * 2 + 1] = bars->l_x[g][0][row] + bars->l_x[g][1][row];
           }
         }
       } else if (g == 1) {
         // both groups hold the same agent rows over different key tiles:
-        // group 1 publishes its running max and waits until group 0 has read
-        // its accumulators
-        if (n_mine > 0 && ok && warp_active && row < p.k) bars->m_x[row] = m;
+        // group 1 has published (m, l) and waits until group 0 has read its
+        // accumulators
         tc_fence_before();
         mbar_arrive(&bars->x_pub);
         if (ok) ok = warp_wait(&bars->x_done, (uint32_t)seg & 1, abort);
@@ -418,11 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             a0 = ex2(m - mm);
             a1 = ex2(m1 - mm);
           }
-          float l = a0 * tmem_ld1(u_col + dn);
-          if (has1) l += a1 * tmem_ld1(u1_col + dn);
           float* dst = p.part_u + (slot_row + row) * p.d;
 #pragma unroll 1
-          for (int c = 0; c < dn / 16; ++c) {
+          for (int c = hf; c < nch_u; c += 2) {
             float u[16];
             tmem_ld16(u_col + c * 16, u);
             if (has1) {
@@ -437,14 +441,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<float4*>(dst + c * 16 + e) =
                     make_float4(u[e], u[e + 1], u[e + 2], u[e + 3]);
           }
-          if (mine) {
+          if (hf == 0 && mine) {
+            float lt = a0 * (bars->l_x[0][0][row] + bars->l_x[0][1][row]);
+            if (has1) lt += a1 * (bars->l_x[1][0][row] + bars->l_x[1][1][row]);
             p.part_ml[(slot_row + row) * 2] = mm;
-            p.part_ml[(slot_row + row) * 2 + 1] = l;
+            p.part_ml[(slot_row + row) * 2 + 1] = lt;
           }
         }
         tc_fence_before();
         mbar_arrive(&bars->x_done);
       }
+      // the next segment's first writes to l_x / m_x come after the next
+      // segment's named barriers, which every thread of both groups reaches
       t = seg_end;
     }
     if (!ok) *abort = 1;
@@ -463,32 +471,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ================================================================ broadcast
 constexpr size_t kBcSmemBytes = 1024 + 2 * (size_t)kMaxAgents * kRowBytes +
                                 (size_t)kBcStages * kQTileBytes + 2 * (size_t)kQTileBytes +
-                                kOnesBytes + sizeof(BcBars);
+                                sizeof(BcBars);
 
-// Row max over the first kpad columns of a score row (columns >= k masked).
-// 64 columns per TMEM load; kpad (a multiple of 16) may end in a 32- or
-// 16-column remainder.
-__device__ __forceinline__ float bc_row_max(uint32_t s_col, int k, int kpad) {
+// Partial row max over score columns [c0, c1) (multiples of 16; columns >= k
+// masked), 32 columns per TMEM load with a 16-column remainder.
+__device__ __forceinline__ float bc_row_max(uint32_t s_col, int k, int c0, int c1) {
   float mx = -INFINITY;
-  int c = 0;
 #pragma unroll 1
-  for (; c + 64 <= kpad; c += 64) {
-    float v[64];
-    tmem_ld64(s_col + c, v);
-    if (c + 64 > k) {
-#pragma unroll
-      for (int e = 0; e < 64; ++e)
-        if (c + e >= k) v[e] = -INFINITY;
-    }
-    mx = max32(*reinterpret_cast<float(*)[32]>(&v[0]),
-               max32(*reinterpret_cast<float(*)[32]>(&v[32]), mx));
-  }
-#pragma unroll 1
-  for (; c < kpad; c += 32) {
+  for (int c = c0; c < c1; c += 32) {
     float v[32];
-    if (c + 32 <= kpad) {
+    if (c + 32 <= c1) {
       tmem_ld32(s_col + c, v);
-    } else {                      // a 16-column remainder
+    } else {
       float h[16];
       tmem_ld16(s_col + c, h);
 #pragma unroll
@@ -497,38 +491,28 @@ __device__ __forceinline__ float bc_row_max(uint32_t s_col, int k, int kpad) {
         v[16 + e] = -INFINITY;
       }
     }
+    if (c + 32 > k) {
 #pragma unroll
-    for (int e = 0; e < 32; ++e)
-      if (c + e >= k) v[e] = -INFINITY;
+      for (int e = 0; e < 32; ++e)
+        if (c + e >= k) v[e] = -INFINITY;
+    }
     mx = max32(v, mx);
   }
   return mx;
 }
 
-// P = 2^(S*c - m) as bf16 over the first kpad/2 columns (columns >= k give 0).
-__device__ __forceinline__ void bc_row_exp(uint32_t s_col, int k, int kpad, float c_scale,
-                                           float m) {
-  int c = 0;
+// P = 2^(S*c - m) as bf16 for score columns [c0, c1) (columns >= k give 0),
+// written over the same row at column p0 + (c - c0)/2 (inside [c0, c1)).
+// Returns the sum of the exponentials.
+__device__ __forceinline__ float bc_row_exp(uint32_t s_col, int k, int c0, int c1, int p0,
+                                            float c_scale, float m) {
+  float sum = 0.f;
 #pragma unroll 1
-  for (; c + 64 <= kpad; c += 64) {
-    float v[64];
-    tmem_ld64(s_col + c, v);
-    if (c + 64 > k) {
-#pragma unroll
-      for (int e = 0; e < 64; ++e)
-        if (c + e >= k) v[e] = -INFINITY;
-    }
-    uint32_t pk[16];
-    exp_pack32(*reinterpret_cast<float(*)[32]>(&v[0]), c_scale, -m, pk);
-    tmem_st16u(s_col + c / 2, pk);
-    exp_pack32(*reinterpret_cast<float(*)[32]>(&v[32]), c_scale, -m, pk);
-    tmem_st16u(s_col + c / 2 + 16, pk);
-  }
-#pragma unroll 1
-  for (; c < kpad; c += 32) {
+  for (int c = c0; c < c1; c += 32) {
     float v[32];
     uint32_t pk[16];
-    if (c + 32 <= kpad) {
+    const bool full = c + 32 <= c1;
+    if (full) {
       tmem_ld32(s_col + c, v);
     } else {
       float h[16];
@@ -539,19 +523,23 @@ __device__ __forceinline__ void bc_row_exp(uint32_t s_col, int k, int kpad, floa
         v[16 + e] = -INFINITY;
       }
     }
+    if (c + 32 > k) {
 #pragma unroll
-    for (int e = 0; e < 32; ++e)
-      if (c + e >= k) v[e] = -INFINITY;
-    exp_pack32(v, c_scale, -m, pk);
-    if (c + 32 <= kpad) {
-      tmem_st16u(s_col + c / 2, pk);
+      for (int e = 0; e < 32; ++e)
+        if (c + e >= k) v[e] = -INFINITY;
+    }
+    sum += exp_pack32(v, c_scale, -m, pk);
+    const int pc = p0 + (c - c0) / 2;
+    if (full) {
+      tmem_st16u(s_col + pc, pk);
     } else {
       uint32_t lo[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) lo[e] = pk[e];
-      tmem_st8(s_col + c / 2, lo);
+      tmem_st8(s_col + pc, lo);
     }
   }
+  return sum;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -566,8 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sVA = sA + kMaxAgents * kRowBytes;
   uint8_t* sQ = sVA + kMaxAgents * kRowBytes;
   uint8_t* sO = sQ + kBcStages * kQTileBytes;
-  uint8_t* sOnes = sO + 2 * kQTileBytes;
-  BcBars* bars = reinterpret_cast<BcBars*>(sOnes + kOnesBytes);
+  BcBars* bars = reinterpret_cast<BcBars*>(sO + 2 * kQTileBytes);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -579,7 +566,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kpad = round16(p.k);
   const int d16 = (p.d + 15) >> 4;
   const int dn = d16 * 16;
-  const int o_col = ((kpad / 2) + 31) & ~31;   // O accumulator column inside a 256-column buffer
+  // Columns of a 256-column TMEM buffer.  The two threads of a row split the
+  // kpad score columns at c_mid; each writes its bf16 P inside its own score
+  // columns (low half at c/2, high half at c_mid + (c - c_mid)/2), so neither
+  // overwrites scores the other still reads.  O (dn columns) goes to columns
+  // P does not use.
+  const int c_mid = (((kpad >> 4) + 1) >> 1) << 4;
+  const int p_hi_end = c_mid + (kpad - c_mid) / 2;
+  const int z2 = round16(p_hi_end);
+  const int o_col = (256 - z2 >= dn) ? z2 : c_mid / 2;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kBcStages; ++s) {
@@ -587,12 +582,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->q_empty[s], 1);
     }
     mbar_init(&bars->ag_full, 1);
-    mbar_init(&bars->ag_empty, 1);
+    mbar_init(&bars->ag_empty, 2);          // both issuers are done with the slice
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->p_full[i], kSoftmaxThreads);
       mbar_init(&bars->o_full[i], 1);
-      mbar_init(&bars->o_free[i], 128);
+      mbar_init(&bars->o_free[i], kSoftmaxThreads);
+      mbar_init(&bars->drain[i], 1);
     }
     bars->abort = 0;
     mbar_fence_init();
@@ -601,7 +597,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&map_va);
     prefetch_tensormap(&map_o);
   }
-  fill_ones(sOnes);
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
@@ -610,8 +605,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  // TMEM: buffer b at column b*256: S over [0, kpad), P (bf16) over [0, kpad/2),
-  // O over [o_col, o_col + dn), l at o_col + dn.
+  // TMEM: buffer g (tiles j with j % 2 == g) at column g*256 holds S, then P
+  // and O as laid out above.
 
   if (warp == 0) {
     if (lane == 0) {
@@ -649,79 +644,89 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp < kFirstSoftmaxWarp) {
     if (lane == 0) {
-      // ------------------------------------------------------- MMA issuer
+      // ----------------------------- MMA issuer of group g (tiles j % 2 == g)
+      const int g = warp - 1;
       const uint32_t idesc_s = idesc_bf16(128, kpad, 0, 0);
       const uint32_t idesc_pv = idesc_bf16(128, dn, 0, 1);
-      const uint32_t idesc_l = idesc_bf16(128, 16, 0, 1);
       const uint32_t sA_addr = smem_u32(sA), sVA_addr = smem_u32(sVA), sQ_addr = smem_u32(sQ);
-      const uint64_t ones_desc = sw128_desc(smem_u32(sOnes), 8192);
-      int n_slices = 0;
+      const uint32_t s_tm = tmem + g * 256;
+      const uint32_t o_tm = s_tm + o_col;
+      int n_slices = 0, u = 0;
       long long cur = -1;
-      auto slice_of = [&](int j) { return (t_begin + j) / tps; };
-      auto issue_s = [&](int j) -> bool {
-        const int b = j & 1;
-        if (slice_of(j) != cur) {
-          if (!mbar_wait(&bars->ag_full, n_slices & 1, abort)) return false;
-          cur = slice_of(j);
+      bool ok = true;
+      // walk every tile so that slice boundaries are seen by both issuers
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        const long long bh = (t_begin + j) / tps;
+        if (bh != cur) {
+          if (cur >= 0) mma_commit(&bars->ag_empty);   // done with the previous slice
+          if (!mbar_wait(&bars->ag_full, n_slices & 1, abort)) {
+            ok = false;
+            break;
+          }
+          cur = bh;
           ++n_slices;
         }
-        if (j >= 2 && !mbar_wait(&bars->o_free[b], ((j >> 1) - 1) & 1, abort)) return false;
+        if ((j & 1) != g) continue;
         const int s = j % kBcStages;
-        if (!mbar_wait(&bars->q_full[s], (j / kBcStages) & 1, abort)) return false;
+        // Start group 1 one softmax behind group 0, so that one group's
+        // exponentials overlap the other group's MMA and epilogue phases
+        // instead of both contending for the SFU at the same time.
+        if (g == 1 && u == 0 && !mbar_wait(&bars->p_full[0], 0, abort)) {
+          ok = false;
+          break;
+        }
+        // S = Q A^T into this group's buffer once its previous O has been read
+        if (u >= 1 && !mbar_wait(&bars->o_free[g], (u - 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(&bars->q_full[s], (j / kBcStages) & 1, abort)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         for (int kk = 0; kk < d16; ++kk) {
           const uint64_t da = sw128_desc(sQ_addr + s * kQTileBytes + kk * 32, 16);
           const uint64_t db = sw128_desc(sA_addr + kk * 32, 16);
-          mma_ss(tmem + b * 256, da, db, idesc_s, kk > 0);
+          mma_ss(s_tm, da, db, idesc_s, kk > 0);
         }
-        mma_commit(&bars->s_full[b]);
+        mma_commit(&bars->s_full[g]);
         mma_commit(&bars->q_empty[s]);
-        return true;
-      };
-      auto issue_pv = [&](int j) -> bool {
-        const int b = j & 1;
-        if (!mbar_wait(&bars->p_full[b], (j >> 1) & 1, abort)) return false;
+        // O = P V_A once the group has written P
+        if (!mbar_wait(&bars->p_full[g], u & 1, abort)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t o_tm = tmem + b * 256 + o_col;
         for (int kk = 0; kk < kpad / 16; ++kk) {
-          const uint32_t p_tm = tmem + b * 256 + kk * 8;
-          mma_ts(o_tm, p_tm, sw128_desc(sVA_addr + kk * 2048, 8192), idesc_pv, kk > 0);
-          mma_ts(o_tm + dn, p_tm, ones_desc, idesc_l, kk > 0);
+          // agents [16 kk, 16 kk + 16) sit in P column kk*8 (low half) or
+          // c_mid + (16 kk - c_mid)/2 (high half)
+          const int pc = (kk * 16 < c_mid) ? kk * 8 : c_mid + (kk * 16 - c_mid) / 2;
+          mma_ts(o_tm, s_tm + pc, sw128_desc(sVA_addr + kk * 2048, 8192), idesc_pv, kk > 0);
         }
-        mma_commit(&bars->o_full[b]);
-        if (j + 1 == n_tiles || slice_of(j + 1) != slice_of(j)) mma_commit(&bars->ag_empty);
-        return true;
-      };
-      bool ok = n_tiles > 0 ? issue_s(0) : true;
-      for (int j = 0; j < n_tiles && ok; ++j) {
-        const bool next_same = j + 1 < n_tiles && slice_of(j + 1) == slice_of(j);
-        if (next_same) {
-          ok = issue_s(j + 1);
-          if (ok) ok = issue_pv(j);
-        } else {
-          ok = issue_pv(j);
-          if (ok && j + 1 < n_tiles) ok = issue_s(j + 1);
-        }
+        mma_commit(&bars->o_full[g]);
+        ++u;
       }
-      // drain: all MMAs complete before TMEM is released
-      mma_commit(&bars->ag_full);
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(&bars->ag_full, (uint32_t)n_slices & 1) &&
-             globaltimer() - t0 < kWaitLimitNs) {
-      }
+      if (ok && cur >= 0) mma_commit(&bars->ag_empty);
+      drain_commits(&bars->drain[g]);
     }
   } else {
     // ------------------------------------------- softmax + epilogue groups
-    const int g = (warp - 2) >> 2;
+    const int sw = warp - kFirstSoftmaxWarp;
+    const int g = sw >> 3;
+    const int hf = (sw >> 2) & 1;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t s_col = tmem + lane_off + g * 256;
     const uint32_t o_tm = s_col + o_col;
     uint8_t* stage = sO + g * kQTileBytes;
-    const bool leader = (warp == 2 + 4 * g) && lane == 0;
+    const bool leader = (warp == kFirstSoftmaxWarp + 8 * g) && lane == 0;
+    // this thread's score columns: half 0 takes [0, c_mid), half 1 [c_mid, kpad)
+    const int c0 = hf ? c_mid : 0, c1 = hf ? kpad : c_mid;
+    const int p0 = hf ? c_mid : 0;
     bool ok = true;
     for (int j = g; j < n_tiles; j += 2) {
       const int u = j >> 1;
@@ -730,59 +735,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q0 = (int)(t - bh * tps) * kQTile;
       if (ok) ok = warp_wait(&bars->s_full[g], u & 1, abort);
       tc_fence_after();
+      if (ok) bars->xmax[g][hf][u & 1][row] = bc_row_max(s_col, p.k, c0, c1);   // -inf if empty
+      named_barrier(3 + g, kSoftmaxThreads);
+      float lsum = 0.f;
       if (ok) {
-        const float m = bc_row_max(s_col, p.k, kpad) * p.c;
-        bc_row_exp(s_col, p.k, kpad, p.c, m);
+        const float m =
+            fmaxf(bars->xmax[g][0][u & 1][row], bars->xmax[g][1][u & 1][row]) * p.c;
+        if (c1 > c0) lsum = bc_row_exp(s_col, p.k, c0, c1, p0, p.c, m);
         tmem_wait_st();
       }
+      bars->xsum[g][hf][u & 1][row] = lsum;
       tc_fence_before();
       mbar_arrive(&bars->p_full[g]);
-      // epilogue: O = (P V_A) / (P 1) -> bf16 -> swizzled staging tile -> TMA store
+      // epilogue: O = (P V_A) / l -> bf16 -> swizzled staging tile -> TMA store
       if (ok) ok = warp_wait(&bars->o_full[g], u & 1, abort);
       tc_fence_after();
-      float o[64];
-      float l = 1.f;
+      // this thread's 8-column output chunks: ch = hf, hf + 2, ... (at most 4)
+      float o[4][8];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        if (ok && c * 32 < dn) {
-          float v[32];
-          if (c * 32 + 32 <= dn) {
-            tmem_ld32(o_tm + c * 32, v);
-          } else {
-            float h[16];
-            tmem_ld16(o_tm + c * 32, h);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              v[e] = h[e];
-              v[16 + e] = 0.f;
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[c * 32 + e] = v[e];
+      for (int q = 0; q < 4; ++q) {
+        const int ch = 2 * q + hf;
+        if (ok && ch * 8 < p.d) {
+          tmem_ld8(o_tm + ch * 8, o[q]);
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[c * 32 + e] = 0.f;
+          for (int e = 0; e < 8; ++e) o[q][e] = 0.f;
         }
       }
-      if (ok) l = tmem_ld1(o_tm + dn);
       tc_fence_before();
-      mbar_arrive(&bars->o_free[g]);
-      const float inv = 1.f / l;
+      mbar_arrive(&bars->o_free[g]);           // the buffer may take the next S now
       if (leader) tma_store_wait_read();
-      named_barrier(3 + g, 128);
+      named_barrier(3 + g, kSoftmaxThreads);
+      const float inv = 1.f / (bars->xsum[g][0][u & 1][row] + bars->xsum[g][1][u & 1][row]);
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int q = 0; q < 4; ++q) {
+        const int ch = 2 * q + hf;
         if (ch * 8 < p.d) {
           uint4 w;
-          w.x = pack_bf16x2(o[ch * 8 + 0] * inv, o[ch * 8 + 1] * inv);
-          w.y = pack_bf16x2(o[ch * 8 + 2] * inv, o[ch * 8 + 3] * inv);
-          w.z = pack_bf16x2(o[ch * 8 + 4] * inv, o[ch * 8 + 5] * inv);
-          w.w = pack_bf16x2(o[ch * 8 + 6] * inv, o[ch * 8 + 7] * inv);
+          w.x = pack_bf16x2(o[q][0] * inv, o[q][1] * inv);
+          w.y = pack_bf16x2(o[q][2] * inv, o[q][3] * inv);
+          w.z = pack_bf16x2(o[q][4] * inv, o[q][5] * inv);
+          w.w = pack_bf16x2(o[q][6] * inv, o[q][7] * inv);
           *reinterpret_cast<uint4*>(stage + row * kRowBytes + ((ch ^ (row & 7)) << 4)) = w;
         }
       }
       fence_proxy_async_smem();
-      named_barrier(3 + g, 128);
+      named_barrier(3 + g, kSoftmaxThreads);
       if (leader && !*abort) {
         tma_store_3d(&map_o, stage, 0, q0, (int)bh);
         tma_store_commit();

@@ -314,6 +314,29 @@ __device__ __forceinline__ void fma2(float& a0, float& a1, float c, float b) {
       : "+f"(a0), "+f"(a1)
       : "f"(c), "f"(b));
 }
+// (a0, a1) + (b0, b1) on the paired FP32 datapath.
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y;\n\t"
+      "mov.b64 x, {%0, %1};\n\t"
+      "mov.b64 y, {%2, %3};\n\t"
+      "add.rn.f32x2 x, x, y;\n\t"
+      "mov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+// 8 consecutive 32-bit TMEM columns of this thread's lane -> registers.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
 // Row max of 32 values, seeded with m.
 __device__ __forceinline__ float max32(const float (&v)[32], float m) {
   float a = fmax3(m, v[0], v[1]), b = fmax3(v[2], v[3], v[4]), c = fmax3(v[5], v[6], v[7]);
@@ -328,14 +351,22 @@ __device__ __forceinline__ float max32(const float (&v)[32], float m) {
   return fmax3(fmax3(a, e, h), k, k);
 }
 // P = 2^(S*c - m) for 32 scores, packed to 16 bf16x2 words.
-__device__ __forceinline__ void exp_pack32(float (&v)[32], float c, float neg_m,
-                                           uint32_t (&pk)[16]) {
+// Returns the fp32 sum of the 32 exponentials (paired adds on the FMA pipe).
+__device__ __forceinline__ float exp_pack32(float (&v)[32], float c, float neg_m,
+                                            uint32_t (&pk)[16]) {
 #pragma unroll
   for (int e = 0; e < 32; e += 2) fma2(v[e], v[e + 1], c, neg_m);
 #pragma unroll
   for (int e = 0; e < 32; ++e) v[e] = ex2(v[e]);
 #pragma unroll
   for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+  float s0 = v[0], s1 = v[1], s2 = v[2], s3 = v[3];
+#pragma unroll
+  for (int e = 4; e < 32; e += 4) {
+    add2(s0, s1, v[e], v[e + 1]);
+    add2(s2, s3, v[e + 2], v[e + 3]);
+  }
+  return (s0 + s1) + (s2 + s3);
 }
 
 __device__ __forceinline__ void tmem_wait_st() {
