@@ -55,13 +55,6 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def dist_env():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return world, rank, local
-
-
 def workload_bytes(w, batch):
     """Algorithmic HBM bytes of one pass: Q, K, V read once and O written once."""
     return 4 * batch * w.H * w.N * w.d * w.elem_bytes
@@ -179,7 +172,17 @@ def cpu_baseline(w, target_s=12.0):
                       f"d={w.d}), fp64, {el:.1f} s"}
 
 
+def bench_config(w, world, set_bytes=None, n_sets=None):
+    cfg = w.describe()
+    cfg.update({"global_batch": world * w.B, "seq_len": w.N, "parallelism": f"replicas x{world}"})
+    if set_bytes is not None:
+        cfg["l2"] = (f"rotating {n_sets} input sets of {set_bytes / 2**20:.0f} MiB "
+                     f"(> 3x the 126 MB L2)")
+    return cfg
+
+
 def run_reference(args, w):
+    from efficient_vision_attention_b200.replicas import dist_env
     world, rank, _ = dist_env()
     if rank != 0:
         return
@@ -195,10 +198,10 @@ def run_reference(args, w):
     el = time.perf_counter() - t0
     value = statistics.median(v["value"] for v in vals)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": steps, "warmup": warm, "ms_per_step": 1e3 * el / max(1, steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": w.describe(),
+        "data": "synthetic", "config": bench_config(w, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": base["cores"], "kind": "oracle",
                          "sample": vals[-1]["sample"] + " per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -209,20 +212,15 @@ def run_reference(args, w):
 def run_native(args, w):
     import torch
     import efficient_vision_attention_b200 as eva
+    from efficient_vision_attention_b200 import replicas
     from efficient_vision_attention_b200.workloads import make_inputs
 
-    world, rank, local = dist_env()
+    world, rank, local = replicas.dist_env()
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-        pg = dist
+    pg = replicas.init("nccl", dev)
     eva.load_library()
     stream = torch.cuda.current_stream(dev)
     dt = eva.AA_FP32 if w.dtype == "fp32" else eva.AA_BF16
@@ -233,7 +231,7 @@ def run_native(args, w):
     n_sets = max(2, math.ceil(3 * L2_BYTES / set_bytes))
     sets = []
     for i in range(n_sets):
-        inp = make_inputs(w, seed=w.seed + 1000 * rank + i)
+        inp = make_inputs(w, seed=replicas.rank_seed(w.seed, rank) + i)
         s = {n: inp[n].to(dev) for n in "qkv"}
         s["agents"] = inp["agents"].to(dev) if inp["agents"] is not None else None
         s["out"] = torch.empty_like(s["q"])
@@ -272,10 +270,7 @@ def run_native(args, w):
     barrier()
     clk = clocks.stop()
     ms = ev0.elapsed_time(ev1) / args.steps
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if pg is not None:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = replicas.max_over_ranks(ms, pg, dev)
     units = world * B * H * N
     value = units / (ms_max * 1e-3)
 
@@ -342,7 +337,7 @@ def run_native(args, w):
 
     # End to end through the host-buffer entry point: pinned host inputs copied
     # in, result copied out, every step.
-    hin = make_inputs(w, seed=w.seed + 1000 * rank)
+    hin = make_inputs(w, seed=replicas.rank_seed(w.seed, rank))
     hq, hk, hv = (hin[n].pin_memory() for n in "qkv")
     hag = hin["agents"].pin_memory() if hin["agents"] is not None else None
     hout = torch.empty_like(hq).pin_memory()
@@ -366,29 +361,22 @@ def run_native(args, w):
             host_step()
         e1.record(stream)
         barrier()
-        e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev, dtype=torch.float64)
-        if pg is not None:
-            pg.all_reduce(e_ms, op=pg.ReduceOp.MAX)
+        e_ms = replicas.max_over_ranks(e0.elapsed_time(e1) / e2e_steps, pg, dev)
         in_bytes = 3 * B * H * N * d * w.elem_bytes + (hag.numel() * hag.element_size()
                                                        if hag is not None else 0)
-        e2e = {"value": units / (float(e_ms.item()) * 1e-3), "unit": UNIT,
+        e2e = {"value": units / (e_ms * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": in_bytes,
                "d2h_bytes_per_step": B * H * N * d * w.elem_bytes,
-               "ms_per_step": float(e_ms.item())}
+               "ms_per_step": e_ms}
 
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base = cpu_baseline(w)
 
-    if pg is not None:
-        pg.barrier()
-        pg.destroy_process_group()
+    replicas.finalize(pg)
     if rank != 0:
         return
-    cfg = w.describe()
-    cfg.update({"global_batch": world * B, "seq_len": N, "parallelism": f"replicas x{world}",
-                "l2": f"rotating {n_sets} input sets of {set_bytes / 2**20:.0f} MiB "
-                      f"(> 3x the 126 MB L2)"})
+    cfg = bench_config(w, world, set_bytes, n_sets)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
