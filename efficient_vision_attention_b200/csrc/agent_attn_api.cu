@@ -221,41 +221,43 @@ int launch_pool(const Problem& p, const void* q, float* a_f32, T* a_lowp, cudaSt
 }
 
 template <typename T>
-int launch_simt_attend(const SimtAttendArgs& args, long long BH, cudaStream_t st) {
+int launch_simt_attend(const SimtAttendArgs& args, long long BH, cudaStream_t st, bool pdl) {
   const size_t smem = simt_attend_smem_bytes(args.d);
   int rc = ensure_smem(simt_attend_kernel<T>, smem,
                        sizeof(T) == 4 ? g_simt_smem_f32 : g_simt_smem_bf16);
   if (rc != AA_OK) return rc;
   const long long blocks = BH * args.splits * args.row_blocks;
   if (blocks > 0x7fffffffLL) return AA_ERR_SHAPE;
-  simt_attend_kernel<T><<<(unsigned)blocks, kSimtThreads, smem, st>>>(args);
-  AA_CUDA(cudaGetLastError());
+  AA_CUDA(launch_kernel(simt_attend_kernel<T>, dim3((unsigned)blocks), dim3(kSimtThreads), smem, st,
+                        pdl, args));
   return AA_OK;
 }
 
 template <typename T>
 int launch_merge(const Problem& p, const Scratch& s, char* ws, float* va_f32, T* va_lowp,
-                 cudaStream_t st) {
+                 cudaStream_t st, bool pdl) {
   const long long work = p.BH() * p.k * (p.d / 4);
   const long long blocks = (work + kMergeThreads - 1) / kMergeThreads;
   if (blocks > 0x7fffffffLL) return AA_ERR_SHAPE;
-  agent_merge_kernel<T><<<(unsigned)blocks, kMergeThreads, 0, st>>>(
-      reinterpret_cast<const float*>(ws + s.pu_off), reinterpret_cast<const float*>(ws + s.pml_off),
-      s.plan, p.BH(), p.k, p.d, va_f32, va_lowp);
-  AA_CUDA(cudaGetLastError());
+  AA_CUDA(launch_kernel(agent_merge_kernel<T>, dim3((unsigned)blocks), dim3(kMergeThreads), 0, st,
+                        pdl, reinterpret_cast<const float*>(ws + s.pu_off),
+                        reinterpret_cast<const float*>(ws + s.pml_off), s.plan, p.BH(), p.k, p.d,
+                        va_f32, va_lowp));
   return AA_OK;
 }
 
-// Aggregation + merge.  agents are in the run dtype (fp32 path: float).
+// Aggregation + merge.  agents are in the run dtype (fp32 path: float).  With
+// pdl, the aggregation overlaps the tail of the previous kernel of the stream.
 template <typename T>
 int run_aggregate(const Problem& p, const Scratch& s, const AgentsRef& ag, const void* k,
-                  const void* v, char* ws, float* va_f32, T* va_lowp, cudaStream_t st) {
+                  const void* v, char* ws, float* va_f32, T* va_lowp, cudaStream_t st,
+                  bool pdl = false) {
   const long long qstride_h = (long long)p.N * p.d, qstride_b = qstride_h * p.H;
   if (use_tensor_cores(p)) {
     cudaError_t e = tc_launch_aggregate(ag.ptr, ag.bstride, ag.hstride, k, v, p.B, p.H, p.N, p.d,
                                         p.k, p.scale * kLog2e, s.plan,
                                         reinterpret_cast<float*>(ws + s.pu_off),
-                                        reinterpret_cast<float*>(ws + s.pml_off), st);
+                                        reinterpret_cast<float*>(ws + s.pml_off), st, pdl);
     if (e != cudaSuccess) return cuda_fail(e, "agent_aggregate (tensor cores) launch");
   } else {
     SimtAttendArgs a;
@@ -280,15 +282,15 @@ int run_aggregate(const Problem& p, const Scratch& s, const AgentsRef& ag, const
     a.part_u = reinterpret_cast<float*>(ws + s.pu_off);
     a.part_ml = reinterpret_cast<float*>(ws + s.pml_off);
     a.slots = s.plan.slots;
-    int rc = launch_simt_attend<T>(a, p.BH(), st);
+    int rc = launch_simt_attend<T>(a, p.BH(), st, pdl);
     if (rc != AA_OK) return rc;
   }
-  return launch_merge<T>(p, s, ws, va_f32, va_lowp, st);
+  return launch_merge<T>(p, s, ws, va_f32, va_lowp, st, true);
 }
 
 template <typename T>
 int run_broadcast(const Problem& p, const void* q, const AgentsRef& ag, const void* va,
-                  void* out, cudaStream_t st) {
+                  void* out, cudaStream_t st, bool pdl = false) {
   const long long qstride_h = (long long)p.N * p.d, qstride_b = qstride_h * p.H;
   const long long vstride_h = (long long)p.k * p.d, vstride_b = vstride_h * p.H;
   if (use_tensor_cores(p)) {
@@ -296,7 +298,7 @@ int run_broadcast(const Problem& p, const void* q, const AgentsRef& ag, const vo
     int rc = device_sm_count(&sms);
     if (rc != AA_OK) return rc;
     cudaError_t e = tc_launch_broadcast(q, ag.ptr, ag.bstride, va, out, p.B, p.H, p.N, p.d, p.k,
-                                        p.scale * kLog2e, sms, st);
+                                        p.scale * kLog2e, sms, st, pdl);
     if (e != cudaSuccess) return cuda_fail(e, "agent_broadcast (tensor cores) launch");
     return AA_OK;
   }
@@ -322,7 +324,7 @@ int run_broadcast(const Problem& p, const void* q, const AgentsRef& ag, const vo
   a.out = out;
   a.out_bstride = qstride_b;
   a.out_hstride = qstride_h;
-  return launch_simt_attend<T>(a, p.BH(), st);
+  return launch_simt_attend<T>(a, p.BH(), st, pdl);
 }
 
 template <typename T>
@@ -342,12 +344,17 @@ int run_forward(const Problem& p, const Scratch& s, const void* q, const void* k
     ag.bstride = ahs * p.H;
     ag.hstride = ahs;
   }
+  // The pool launches normally (it follows whatever the stream did before);
+  // the kernels after it overlap their predecessors' tails (programmatic
+  // dependent launch) and read their outputs only after a grid dependency wait.
+  const bool pdl_agg = learnable == nullptr;
   T* va_ws = reinterpret_cast<T*>(ws + s.va_off);
   int rc = (sizeof(T) == 4)
-               ? run_aggregate<T>(p, s, ag, k, v, ws, reinterpret_cast<float*>(va_ws), nullptr, st)
-               : run_aggregate<T>(p, s, ag, k, v, ws, nullptr, va_ws, st);
+               ? run_aggregate<T>(p, s, ag, k, v, ws, reinterpret_cast<float*>(va_ws), nullptr,
+                                  st, pdl_agg)
+               : run_aggregate<T>(p, s, ag, k, v, ws, nullptr, va_ws, st, pdl_agg);
   if (rc != AA_OK) return rc;
-  return run_broadcast<T>(p, q, ag, va_ws, out, st);
+  return run_broadcast<T>(p, q, ag, va_ws, out, st, true);
 }
 
 int forward_impl(const Problem& p, const void* q, const void* k, const void* v,

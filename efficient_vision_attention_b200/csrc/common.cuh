@@ -7,6 +7,16 @@
 
 namespace aa {
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream runs; it
+// must wait here before touching anything that kernel writes (a no-op when
+// the kernel was launched normally).  The trigger lets the next kernel of the
+// stream begin its own launch early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Element loads/stores for the two run dtypes, widened to / narrowed from fp32.
@@ -108,6 +118,25 @@ __host__ __device__ __forceinline__ int splits_of_slice(const SplitPlan& p, long
   long long t0 = bh * p.tiles_per_slice;
   long long t1 = t0 + p.tiles_per_slice - 1;
   return (int)(stream_cta_of_tile(p, t1) - stream_cta_of_tile(p, t0) + 1);
+}
+
+// Launches `kernel`; with pdl = true, with programmatic stream serialization
+// (the kernel may start before the previous kernel of the stream finishes and
+// synchronises with it through pdl_wait()).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t st, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 }  // namespace aa

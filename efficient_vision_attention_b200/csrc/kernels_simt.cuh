@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(kPoolThreads) agent_pool_kernel(const T* __res
                                                                   int pool_h, int pool_w,
                                                                   int px_per_cta) {
   extern __shared__ float colsum[];          // [token column of the window][group][8]
+  pdl_trigger();
   const int n_chunks = (pool_w + px_per_cta - 1) / px_per_cta;
   const int py = blockIdx.x / n_chunks;
   const int px0 = (blockIdx.x % n_chunks) * px_per_cta;
@@ -185,6 +186,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_attend_kernel(SimtAttendArg
   const T* vals = static_cast<const T*>(p.vals) +
                   agent_set_offset(bh, p.H, p.vals_bstride, p.vals_hstride);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_trigger();
 
   for (int e = tid; e < kSimtRows * d; e += kSimtThreads) {
     const int r = e / d, c = e % d;
@@ -282,6 +285,8 @@ __global__ void __launch_bounds__(kMergeThreads) agent_merge_kernel(
     long long BH, int n_agents, int d, float* __restrict__ va_f32, T* __restrict__ va_lowp) {
   const int quads = d >> 2;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (idx >= BH * n_agents * quads) return;
   const int cq = (int)(idx % quads);
   const long long row = idx / quads;              // bh * n_agents + j

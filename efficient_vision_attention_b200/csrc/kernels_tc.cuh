@@ -178,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_trigger();
   const uint32_t tmem = bars->tmem_base;
   // TMEM columns: score buffer b of group g at g*128 + b*64 (P over its first
   // 32 columns), U of group g at 256 + g*128 (dn columns).
@@ -188,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long it = 0;
       int seg = 0;
       const uint32_t a_bytes = (two ? 256 : 128) * kRowBytes;
+      pdl_wait();             // the agents may come from the previous kernel
       for (long long t = t_begin; t < t_end; ++seg) {
         const long long bh = t / tps;
         const long long seg_end = min(t_end, (bh + 1) * tps);
@@ -604,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_trigger();
   const uint32_t tmem = bars->tmem_base;
   // TMEM: buffer g (tiles j with j % 2 == g) at column g*256 holds S, then P
   // and O as laid out above.
@@ -614,6 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long cur = -1;
       int n_slices = 0;
       const uint32_t ag_bytes = 2u * kpad * kRowBytes;
+      pdl_wait();             // agents and V_A come from the previous kernels
       int j = 0;
       for (; j < n_tiles; ++j) {
         const long long t = t_begin + j;
@@ -897,7 +901,8 @@ inline cudaError_t ensure_tc_smem(const void* kernel, int bytes, std::atomic<int
 inline cudaError_t tc_launch_aggregate(const void* agents, long long a_bstride, long long a_hstride,
                                        const void* k, const void* v, int B, int H, int N, int d,
                                        int n_agents, float c, const SplitPlan& plan,
-                                       float* part_u, float* part_ml, cudaStream_t st) {
+                                       float* part_u, float* part_ml, cudaStream_t st,
+                                       bool pdl) {
   (void)a_hstride;
   using namespace tc;
   CUtensorMap mk, mv, ma;
@@ -922,13 +927,14 @@ inline cudaError_t tc_launch_aggregate(const void* agents, long long a_bstride, 
   p.slots = plan.slots;
   p.part_u = part_u;
   p.part_ml = part_ml;
-  agent_aggregate_tc_kernel<<<plan.ctas, kThreads, kAggSmemBytes, st>>>(mk, mv, ma, a_sets, p);
-  return cudaGetLastError();
+  return launch_kernel(agent_aggregate_tc_kernel, dim3(plan.ctas), dim3(kThreads), kAggSmemBytes,
+                       st, pdl, mk, mv, ma, a_sets, p);
 }
 
 inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long long a_bstride,
                                        const void* va, void* out, int B, int H, int N, int d,
-                                       int n_agents, float c, int sm_count, cudaStream_t st) {
+                                       int n_agents, float c, int sm_count, cudaStream_t st,
+                                       bool pdl) {
   using namespace tc;
   CUtensorMap mq, ma, mva, mo;
   int a_sets = 1;
@@ -950,8 +956,8 @@ inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long l
   p.tiles_per_slice = (N + kQTile - 1) / kQTile;
   p.total_tiles = BH * p.tiles_per_slice;
   p.ctas = (int)(p.total_tiles < sm_count ? p.total_tiles : sm_count);
-  agent_broadcast_tc_kernel<<<p.ctas, kThreads, kBcSmemBytes, st>>>(mq, ma, mva, mo, a_sets, p);
-  return cudaGetLastError();
+  return launch_kernel(agent_broadcast_tc_kernel, dim3(p.ctas), dim3(kThreads), kBcSmemBytes, st,
+                       pdl, mq, ma, mva, mo, a_sets, p);
 }
 
 }  // namespace aa
