@@ -102,7 +102,7 @@ class ClockSampler:
             except Exception as e:
                 self.error = repr(e)
                 return
-            self._stop.wait(0.02)
+            self._stop.wait(0.005)
 
     def stop(self):
         if self._thread is None:

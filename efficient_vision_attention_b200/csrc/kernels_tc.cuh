@@ -30,9 +30,11 @@
 // spends about 57 cycles per tcgen05.mma, so two issuers double the MMA rate
 // and keep the groups independent); warps 3-10 and 11-18 are the two softmax
 // groups, working on alternating tiles (or, for k > 128 in the aggregation,
-// on the two 128-agent halves).  In a group, TMEM lane = row, and each row
-// has two threads (two warps share a lane quadrant) that split its columns
-// and exchange partial row maxima and sums through shared memory.  Every wait
+// on the two 128-agent halves).  In a group, TMEM lane = row, and each warp
+// owns a 16-row slab of the 128 rows with all the columns of the tile (the
+// 16x256b TMEM access shape spreads a row over 4 threads, which combine row
+// maxima and sums with shuffles), so no warp waits for another inside the
+// softmax of a tile.  Every wait
 // is bounded; a wait that gives up makes its CTA skip the rest of its work
 // and raises the device watchdog.
 #pragma once
@@ -86,9 +88,8 @@ struct AggBars {
   uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
-  float m_x[128];
-  float l_x[2][2][128];      // [group][half][row]: partial row sums at a segment end
-  float xmax[2][2][2][128];  // [group][half][tile parity][row]: partial row maxima
+  float m_x[128];            // group 1's row maxima and sums at a segment end (k <= 128)
+  float l_x[128];
 };
 
 struct BcBars {
@@ -98,8 +99,6 @@ struct BcBars {
   uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
-  float xmax[2][2][2][128];  // [group][half][tile parity][row]: partial row maxima
-  float xsum[2][2][2][128];  // [group][half][tile parity][row]: partial row sums
 };
 
 __host__ __device__ constexpr int round16(int x) { return (x + 15) & ~15; }
@@ -302,16 +301,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------- softmax groups
     // Every thread walks the same segments and tiles whatever happens; after a
     // failed (timed-out) wait it only skips work, so no barrier is left short.
+    // A warp owns a 16-row slab of its group's 128 TMEM lanes with all 64
+    // columns of each score tile: the 4 threads of a row reduce its maximum
+    // and sum with shuffles, so the warps of a group never wait for each other
+    // inside a tile.
     const int sw = warp - kFirstSoftmaxWarp;  // 0..15
     const int g = sw >> 3;                    // group 0: warps 3-10, group 1: warps 11-18
-    const int hf = (sw >> 2) & 1;             // column half of the row this thread owns
     const int quad = warp & 3;                // TMEM lane quadrant this warp may access
-    const int row = quad * 32 + lane;         // TMEM lane = row of the 128-row tile
-    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t u_col = tmem + lane_off + 256 + g * 128;
-    const int agent = (two ? g * 128 : 0) + row;
-    const bool warp_active = (two ? g * 128 : 0) + quad * 32 < p.k;
-    const int nch_u = dn / 16;
+    const int slab = quad * 32 + ((sw >> 2) & 1) * 16;   // first lane (row) of the slab
+    const int j4 = lane & 3;
+    const int r0 = slab + (lane >> 2), r1 = r0 + 8;      // this thread's two rows
+    const uint32_t slab_off = (uint32_t)slab << 16;
+    const uint32_t u_col = tmem + slab_off + 256 + g * 128;
+    const int row_base = two ? g * 128 : 0;   // agent of TMEM lane 0 in this group
+    const bool warp_active = row_base + slab < p.k;
     int J = 0, seg = 0;
     bool ok = true;
     for (long long t = t_begin; t < t_end; ++seg) {
@@ -319,56 +322,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long seg_end = min(t_end, (bh + 1) * tps);
       const int n = (int)(seg_end - t);
       const int n_mine = two ? n : (g == 0 ? (n + 1) / 2 : n / 2);
-      float m = -INFINITY, l = 0.f;             // running max (log2 units) and this half's sum
+      // running maxima (log2 units) and this thread's partial sums of its rows
+      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
       bool first = true;
       for (int i = 0; i < n; ++i) {
         if (!two && (i & 1) != g) continue;
         const int b = J & 1;
-        const uint32_t s_col = tmem + lane_off + g * 128 + b * 64;
+        const uint32_t s_col = tmem + slab_off + g * 128 + b * 64;
         const int valid = min(kKeyTile, p.N - (int)(t + i - bh * tps) * kKeyTile);
         if (ok) ok = warp_wait(&bars->s_full[g][b], (uint32_t)(J >> 1) & 1, abort);
         tc_fence_after();
-        float v[32];
         if (ok && warp_active) {
-          tmem_ld32(s_col + hf * 32, v);
-          if (valid < kKeyTile) {               // ragged last tile: mask the missing keys
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (hf * 32 + e >= valid) v[e] = -INFINITY;
-          }
-          bars->xmax[g][hf][b][row] = max32(v, -INFINITY);
-        }
-        named_barrier(1 + g, kSoftmaxThreads);
-        if (ok && warp_active) {
-          const float mt =
-              fmaxf(bars->xmax[g][0][b][row], bars->xmax[g][1][b][row]) * p.c;
+          float v[32];
+          slab_ld64(s_col, v);
+          if (valid < kKeyTile) slab_mask<8>(v, 0, j4, valid);   // ragged last tile
+          float t0 = -INFINITY, t1 = -INFINITY;
+          slab_max<8>(v, t0, t1);
+          t0 = row4_max(t0) * p.c;
+          t1 = row4_max(t1) * p.c;
           if (first) {
-            m = mt;
+            m0 = t0;
+            m1 = t1;
             first = false;
-          } else if (__any_sync(0xffffffffu, mt > m + kRescaleThreshold)) {
-            // the running max grew a lot: once the previous P V has landed,
-            // rescale U and l by 2^(m_old - m_new) (each half takes alternate chunks)
+          } else if (__any_sync(0xffffffffu,
+                                t0 > m0 + kRescaleThreshold || t1 > m1 + kRescaleThreshold)) {
+            // a running max grew a lot: once the previous P V has landed,
+            // rescale the slab's U rows and sums by 2^(m_old - m_new)
             ok = warp_wait(&bars->pv_done[g][(J - 1) & 1], (uint32_t)((J - 1) >> 1) & 1, abort);
             tc_fence_after();
             if (ok) {
-              const float m_new = fmaxf(m, mt);
-              const float alpha = ex2(m - m_new);
-              m = m_new;
-              l *= alpha;
+              const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
+              const float a0 = ex2(m0 - n0), a1 = ex2(m1 - n1);
+              m0 = n0;
+              m1 = n1;
+              l0 *= a0;
+              l1 *= a1;
 #pragma unroll 1
-              for (int c = hf; c < nch_u; c += 2) {
-                float u[16];
-                tmem_ld16(u_col + c * 16, u);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) u[e] *= alpha;
-                tmem_st16(u_col + c * 16, u);
+              for (int c = 0; c < dn; c += 16) {
+                float u[8];
+                slab_ld16(u_col + c, u);
+                u[0] *= a0; u[1] *= a0; u[2] *= a1; u[3] *= a1;
+                u[4] *= a0; u[5] *= a0; u[6] *= a1; u[7] *= a1;
+                slab_st16(u_col + c, u);
               }
             }
           }
           if (ok) {
             uint32_t pk[16];
-            l += exp_pack32(v, p.c, -m, pk);
-            tmem_st16u(s_col + hf * 16, pk);
+            slab_exp<8>(v, p.c, -m0, -m1, pk, l0, l1);
+            slab_st_p32(s_col, pk);
             tmem_wait_st();
           }
         }
@@ -382,32 +384,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (n_mine > 0 && ok)
         ok = warp_wait(&bars->pv_done[g][(J - 1) & 1], (uint32_t)((J - 1) >> 1) & 1, abort);
       tc_fence_after();
-      bars->l_x[g][hf][row] = l;
-      if (hf == 0 && g == 1) bars->m_x[row] = m;
-      named_barrier(1 + g, kSoftmaxThreads);
+      l0 = row4_sum(l0);
+      l1 = row4_sum(l1);
       if (two) {
         if (ok && warp_active) {            // warp-uniform: the TMEM loads are warp-collective
-          const bool mine = agent < p.k;
-          float* dst = p.part_u + (slot_row + agent) * p.d;
+          const int a0 = row_base + r0, a1 = row_base + r1;
 #pragma unroll 1
-          for (int c = hf; c < nch_u; c += 2) {
-            float u[16];
-            tmem_ld16(u_col + c * 16, u);
+          for (int c = 0; c < dn; c += 16) {
+            float u[8];
+            slab_ld16(u_col + c, u);
 #pragma unroll
-            for (int e = 0; e < 16; e += 4)
-              if (mine && c * 16 + e < p.d)
-                *reinterpret_cast<float4*>(dst + c * 16 + e) =
-                    make_float4(u[e], u[e + 1], u[e + 2], u[e + 3]);
+            for (int h = 0; h < 2; ++h) {
+              const int col = c + 8 * h + 2 * j4;
+              if (c + 8 * h < p.d) {
+                if (a0 < p.k)
+                  *reinterpret_cast<float2*>(p.part_u + (slot_row + a0) * p.d + col) =
+                      make_float2(u[4 * h], u[4 * h + 1]);
+                if (a1 < p.k)
+                  *reinterpret_cast<float2*>(p.part_u + (slot_row + a1) * p.d + col) =
+                      make_float2(u[4 * h + 2], u[4 * h + 3]);
+              }
+            }
           }
-          if (hf == 0 && mine) {
-            p.part_ml[(slot_row + agent) * 2] = m;
-            p.part_ml[(slot_row + agent) * 2 + 1] = bars->l_x[g][0][row] + bars->l_x[g][1][row];
+          if (j4 == 0) {
+            if (a0 < p.k)
+              *reinterpret_cast<float2*>(p.part_ml + (slot_row + a0) * 2) = make_float2(m0, l0);
+            if (a1 < p.k)
+              *reinterpret_cast<float2*>(p.part_ml + (slot_row + a1) * 2) = make_float2(m1, l1);
           }
         }
       } else if (g == 1) {
         // both groups hold the same agent rows over different key tiles:
-        // group 1 has published (m, l) and waits until group 0 has read its
+        // group 1 publishes (m, l) and waits until group 0 has read its
         // accumulators
+        if (j4 == 0) {
+          bars->m_x[r0] = m0;
+          bars->m_x[r1] = m1;
+          bars->l_x[r0] = l0;
+          bars->l_x[r1] = l1;
+        }
         tc_fence_before();
         mbar_arrive(&bars->x_pub);
         if (ok) ok = warp_wait(&bars->x_done, (uint32_t)seg & 1, abort);
@@ -416,45 +431,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = warp_wait(&bars->x_pub, (uint32_t)seg & 1, abort);
         tc_fence_after();
         if (ok && warp_active) {            // warp-uniform: the TMEM loads are warp-collective
-          const bool mine = row < p.k;
           const bool has1 = (n / 2) > 0;
-          const uint32_t u1_col = tmem + lane_off + 256 + 128;
-          float mm = m, a0 = 1.f, a1 = 0.f;
-          if (has1 && mine) {
-            const float m1 = bars->m_x[row];
-            mm = fmaxf(m, m1);
-            a0 = ex2(m - mm);
-            a1 = ex2(m1 - mm);
+          const uint32_t u1_col = tmem + slab_off + 256 + 128;
+          float mm0 = m0, mm1 = m1, s0 = 1.f, s1 = 1.f, w0 = 0.f, w1 = 0.f;
+          if (has1) {
+            const float x0 = bars->m_x[r0], x1 = bars->m_x[r1];
+            mm0 = fmaxf(m0, x0);
+            mm1 = fmaxf(m1, x1);
+            s0 = ex2(m0 - mm0);
+            s1 = ex2(m1 - mm1);
+            w0 = ex2(x0 - mm0);
+            w1 = ex2(x1 - mm1);
           }
-          float* dst = p.part_u + (slot_row + row) * p.d;
 #pragma unroll 1
-          for (int c = hf; c < nch_u; c += 2) {
-            float u[16];
-            tmem_ld16(u_col + c * 16, u);
+          for (int c = 0; c < dn; c += 16) {
+            float u[8];
+            slab_ld16(u_col + c, u);
             if (has1) {
-              float w[16];
-              tmem_ld16(u1_col + c * 16, w);
+              float w[8];
+              slab_ld16(u1_col + c, w);
 #pragma unroll
-              for (int e = 0; e < 16; ++e) u[e] = a0 * u[e] + a1 * w[e];
+              for (int h = 0; h < 2; ++h) {
+                u[4 * h] = s0 * u[4 * h] + w0 * w[4 * h];
+                u[4 * h + 1] = s0 * u[4 * h + 1] + w0 * w[4 * h + 1];
+                u[4 * h + 2] = s1 * u[4 * h + 2] + w1 * w[4 * h + 2];
+                u[4 * h + 3] = s1 * u[4 * h + 3] + w1 * w[4 * h + 3];
+              }
             }
 #pragma unroll
-            for (int e = 0; e < 16; e += 4)
-              if (mine && c * 16 + e < p.d)
-                *reinterpret_cast<float4*>(dst + c * 16 + e) =
-                    make_float4(u[e], u[e + 1], u[e + 2], u[e + 3]);
+            for (int h = 0; h < 2; ++h) {
+              const int col = c + 8 * h + 2 * j4;
+              if (c + 8 * h < p.d) {
+                if (r0 < p.k)
+                  *reinterpret_cast<float2*>(p.part_u + (slot_row + r0) * p.d + col) =
+                      make_float2(u[4 * h], u[4 * h + 1]);
+                if (r1 < p.k)
+                  *reinterpret_cast<float2*>(p.part_u + (slot_row + r1) * p.d + col) =
+                      make_float2(u[4 * h + 2], u[4 * h + 3]);
+              }
+            }
           }
-          if (hf == 0 && mine) {
-            float lt = a0 * (bars->l_x[0][0][row] + bars->l_x[0][1][row]);
-            if (has1) lt += a1 * (bars->l_x[1][0][row] + bars->l_x[1][1][row]);
-            p.part_ml[(slot_row + row) * 2] = mm;
-            p.part_ml[(slot_row + row) * 2 + 1] = lt;
+          if (j4 == 0) {
+            const float lt0 = s0 * l0 + (has1 ? w0 * bars->l_x[r0] : 0.f);
+            const float lt1 = s1 * l1 + (has1 ? w1 * bars->l_x[r1] : 0.f);
+            if (r0 < p.k)
+              *reinterpret_cast<float2*>(p.part_ml + (slot_row + r0) * 2) = make_float2(mm0, lt0);
+            if (r1 < p.k)
+              *reinterpret_cast<float2*>(p.part_ml + (slot_row + r1) * 2) = make_float2(mm1, lt1);
           }
         }
         tc_fence_before();
         mbar_arrive(&bars->x_done);
       }
-      // the next segment's first writes to l_x / m_x come after the next
-      // segment's named barriers, which every thread of both groups reaches
+      // group 1 writes m_x / l_x again only after the next segment's x_done
+      // phase, which follows group 0's reads of this one
       t = seg_end;
     }
     if (!ok) *abort = 1;
@@ -475,73 +505,66 @@ constexpr size_t kBcSmemBytes = 1024 + 2 * (size_t)kMaxAgents * kRowBytes +
                                 (size_t)kBcStages * kQTileBytes + 2 * (size_t)kQTileBytes +
                                 sizeof(BcBars);
 
-// Partial row max over score columns [c0, c1) (multiples of 16; columns >= k
-// masked), 32 columns per TMEM load with a 16-column remainder.
-__device__ __forceinline__ float bc_row_max(uint32_t s_col, int k, int c0, int c1) {
-  float mx = -INFINITY;
+// Row maxima of a slab's two rows (this thread's columns) over score columns
+// [0, kpad), columns >= k masked; 64 columns per TMEM load, then 32 and 16.
+__device__ __forceinline__ void bc_slab_max(uint32_t s_col, int k, int kpad, int j4, float& t0,
+                                            float& t1) {
+  int c = 0;
 #pragma unroll 1
-  for (int c = c0; c < c1; c += 32) {
+  for (; c + 64 <= kpad; c += 64) {
     float v[32];
-    if (c + 32 <= c1) {
-      tmem_ld32(s_col + c, v);
-    } else {
-      float h[16];
-      tmem_ld16(s_col + c, h);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        v[e] = h[e];
-        v[16 + e] = -INFINITY;
-      }
-    }
-    if (c + 32 > k) {
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (c + e >= k) v[e] = -INFINITY;
-    }
-    mx = max32(v, mx);
+    slab_ld64(s_col + c, v);
+    if (c + 64 > k) slab_mask<8>(v, c, j4, k);
+    slab_max<8>(v, t0, t1);
   }
-  return mx;
+  if (c + 32 <= kpad) {
+    float v[16];
+    slab_ld32(s_col + c, v);
+    if (c + 32 > k) slab_mask<4>(v, c, j4, k);
+    slab_max<4>(v, t0, t1);
+    c += 32;
+  }
+  if (c < kpad) {
+    float v[8];
+    slab_ld16(s_col + c, v);
+    if (c + 16 > k) slab_mask<2>(v, c, j4, k);
+    slab_max<2>(v, t0, t1);
+  }
 }
 
-// P = 2^(S*c - m) as bf16 for score columns [c0, c1) (columns >= k give 0),
-// written over the same row at column p0 + (c - c0)/2 (inside [c0, c1)).
-// Returns the sum of the exponentials.
-__device__ __forceinline__ float bc_row_exp(uint32_t s_col, int k, int c0, int c1, int p0,
-                                            float c_scale, float m) {
-  float sum = 0.f;
+// P = 2^(S*c - m_row) as bf16 for score columns [0, kpad) (columns >= k give
+// 0), written over the same rows at packed column (score column)/2: a block's
+// P lands on columns this warp has already read.  Adds the exponentials to
+// the partial row sums l0, l1.
+__device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int j4, float c_scale,
+                                            float neg_m0, float neg_m1, float& l0, float& l1) {
+  int c = 0;
 #pragma unroll 1
-  for (int c = c0; c < c1; c += 32) {
+  for (; c + 64 <= kpad; c += 64) {
     float v[32];
     uint32_t pk[16];
-    const bool full = c + 32 <= c1;
-    if (full) {
-      tmem_ld32(s_col + c, v);
-    } else {
-      float h[16];
-      tmem_ld16(s_col + c, h);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        v[e] = h[e];
-        v[16 + e] = -INFINITY;
-      }
-    }
-    if (c + 32 > k) {
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (c + e >= k) v[e] = -INFINITY;
-    }
-    sum += exp_pack32(v, c_scale, -m, pk);
-    const int pc = p0 + (c - c0) / 2;
-    if (full) {
-      tmem_st16u(s_col + pc, pk);
-    } else {
-      uint32_t lo[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) lo[e] = pk[e];
-      tmem_st8(s_col + pc, lo);
-    }
+    slab_ld64(s_col + c, v);
+    if (c + 64 > k) slab_mask<8>(v, c, j4, k);
+    slab_exp<8>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
+    slab_st_p32(s_col + c / 2, pk);
   }
-  return sum;
+  if (c + 32 <= kpad) {
+    float v[16];
+    uint32_t pk[8];
+    slab_ld32(s_col + c, v);
+    if (c + 32 > k) slab_mask<4>(v, c, j4, k);
+    slab_exp<4>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
+    slab_st_p16(s_col + c / 2, pk);
+    c += 32;
+  }
+  if (c < kpad) {
+    float v[8];
+    uint32_t pk[4];
+    slab_ld16(s_col + c, v);
+    if (c + 16 > k) slab_mask<2>(v, c, j4, k);
+    slab_exp<2>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
+    slab_st_p8(s_col + c / 2, pk);
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -568,16 +591,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kpad = round16(p.k);
   const int d16 = (p.d + 15) >> 4;
   const int dn = d16 * 16;
-  // Columns of a 256-column TMEM buffer.  The two threads of a row split the
-  // kpad score columns at c_mid; each writes its bf16 P inside its own score
-  // columns (low half at c/2, high half at c_mid + (c - c_mid)/2), so neither
-  // overwrites scores the other still reads.  O (dn columns) goes to columns
-  // P does not use.
-  const int c_mid = (((kpad >> 4) + 1) >> 1) << 4;
-  const int p_hi_end = c_mid + (kpad - c_mid) / 2;
-  const int z2 = round16(p_hi_end);
-  const int o_col = (256 - z2 >= dn) ? z2 : c_mid / 2;
-
+  // Columns of a 256-column TMEM buffer: S over [0, kpad), then P (bf16x2)
+  // over [0, kpad/2), O (dn columns) after P.
+  const int o_col = round16(kpad / 2);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kBcStages; ++s) {
       mbar_init(&bars->q_full[s], 1);
@@ -609,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();
   const uint32_t tmem = bars->tmem_base;
   // TMEM: buffer g (tiles j with j % 2 == g) at column g*256 holds S, then P
-  // and O as laid out above.
+  // and O as laid out above (o_col + dn <= 128 + 64).
 
   if (warp == 0) {
     if (lane == 0) {
@@ -704,12 +720,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        for (int kk = 0; kk < kpad / 16; ++kk) {
-          // agents [16 kk, 16 kk + 16) sit in P column kk*8 (low half) or
-          // c_mid + (16 kk - c_mid)/2 (high half)
-          const int pc = (kk * 16 < c_mid) ? kk * 8 : c_mid + (kk * 16 - c_mid) / 2;
-          mma_ts(o_tm, s_tm + pc, sw128_desc(sVA_addr + kk * 2048, 8192), idesc_pv, kk > 0);
-        }
+        for (int kk = 0; kk < kpad / 16; ++kk)   // agents [16 kk, 16 kk + 16): P column 8 kk
+          mma_ts(o_tm, s_tm + kk * 8, sw128_desc(sVA_addr + kk * 2048, 8192), idesc_pv, kk > 0);
         mma_commit(&bars->o_full[g]);
         ++u;
       }
@@ -718,19 +730,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------- softmax + epilogue groups
+    // A warp owns a 16-row slab of the group's 128 query rows with all k
+    // score columns; the 4 threads of a row reduce its maximum and sum with
+    // shuffles, so within a tile the warps only meet at the output staging.
     const int sw = warp - kFirstSoftmaxWarp;
     const int g = sw >> 3;
-    const int hf = (sw >> 2) & 1;
     const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t s_col = tmem + lane_off + g * 256;
+    const int slab = quad * 32 + ((sw >> 2) & 1) * 16;
+    const int j4 = lane & 3;
+    const int r0 = slab + (lane >> 2), r1 = r0 + 8;
+    const uint32_t s_col = tmem + ((uint32_t)slab << 16) + g * 256;
     const uint32_t o_tm = s_col + o_col;
     uint8_t* stage = sO + g * kQTileBytes;
     const bool leader = (warp == kFirstSoftmaxWarp + 8 * g) && lane == 0;
-    // this thread's score columns: half 0 takes [0, c_mid), half 1 [c_mid, kpad)
-    const int c0 = hf ? c_mid : 0, c1 = hf ? kpad : c_mid;
-    const int p0 = hf ? c_mid : 0;
+    const int n_ch = dn / 16;                // 16-column chunks of O
     bool ok = true;
     for (int j = g; j < n_tiles; j += 2) {
       const int u = j >> 1;
@@ -739,28 +752,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q0 = (int)(t - bh * tps) * kQTile;
       if (ok) ok = warp_wait(&bars->s_full[g], u & 1, abort);
       tc_fence_after();
-      if (ok) bars->xmax[g][hf][u & 1][row] = bc_row_max(s_col, p.k, c0, c1);   // -inf if empty
-      named_barrier(3 + g, kSoftmaxThreads);
-      float lsum = 0.f;
+      float l0 = 0.f, l1 = 0.f;
       if (ok) {
-        const float m =
-            fmaxf(bars->xmax[g][0][u & 1][row], bars->xmax[g][1][u & 1][row]) * p.c;
-        if (c1 > c0) lsum = bc_row_exp(s_col, p.k, c0, c1, p0, p.c, m);
+        float t0 = -INFINITY, t1 = -INFINITY;
+        bc_slab_max(s_col, p.k, kpad, j4, t0, t1);
+        t0 = row4_max(t0) * p.c;
+        t1 = row4_max(t1) * p.c;
+        bc_slab_exp(s_col, p.k, kpad, j4, p.c, -t0, -t1, l0, l1);
         tmem_wait_st();
       }
-      bars->xsum[g][hf][u & 1][row] = lsum;
       tc_fence_before();
       mbar_arrive(&bars->p_full[g]);
+      const float inv0 = 1.f / row4_sum(l0), inv1 = 1.f / row4_sum(l1);
       // epilogue: O = (P V_A) / l -> bf16 -> swizzled staging tile -> TMA store
       if (ok) ok = warp_wait(&bars->o_full[g], u & 1, abort);
       tc_fence_after();
-      // this thread's 8-column output chunks: ch = hf, hf + 2, ... (at most 4)
       float o[4][8];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int ch = 2 * q + hf;
-        if (ok && ch * 8 < p.d) {
-          tmem_ld8(o_tm + ch * 8, o[q]);
+        if (ok && q < n_ch) {
+          slab_ld16(o_tm + q * 16, o[q]);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) o[q][e] = 0.f;
@@ -770,17 +781,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars->o_free[g]);           // the buffer may take the next S now
       if (leader) tma_store_wait_read();
       named_barrier(3 + g, kSoftmaxThreads);
-      const float inv = 1.f / (bars->xsum[g][0][u & 1][row] + bars->xsum[g][1][u & 1][row]);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int ch = 2 * q + hf;
-        if (ch * 8 < p.d) {
-          uint4 w;
-          w.x = pack_bf16x2(o[q][0] * inv, o[q][1] * inv);
-          w.y = pack_bf16x2(o[q][2] * inv, o[q][3] * inv);
-          w.z = pack_bf16x2(o[q][4] * inv, o[q][5] * inv);
-          w.w = pack_bf16x2(o[q][6] * inv, o[q][7] * inv);
-          *reinterpret_cast<uint4*>(stage + row * kRowBytes + ((ch ^ (row & 7)) << 4)) = w;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int ch = 2 * q + h;            // 16-byte chunk (8 columns) of the row
+          if (ch * 8 < p.d) {
+            *reinterpret_cast<uint32_t*>(stage + r0 * kRowBytes + ((ch ^ (r0 & 7)) << 4) +
+                                         j4 * 4) =
+                pack_bf16x2(o[q][4 * h] * inv0, o[q][4 * h + 1] * inv0);
+            *reinterpret_cast<uint32_t*>(stage + r1 * kRowBytes + ((ch ^ (r1 & 7)) << 4) +
+                                         j4 * 4) =
+                pack_bf16x2(o[q][4 * h + 2] * inv1, o[q][4 * h + 3] * inv1);
+          }
         }
       }
       fence_proxy_async_smem();

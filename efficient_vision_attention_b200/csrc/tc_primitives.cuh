@@ -369,6 +369,153 @@ __device__ __forceinline__ float exp_pack32(float (&v)[32], float c, float neg_m
   return (s0 + s1) + (s2 + s3);
 }
 
+// ------------------------------------------------- 16-lane slab access
+// The 16x256b / 16x128b shapes move 16 TMEM lanes (a 16-aligned base lane
+// inside the warp's quadrant).  Thread t holds rows t/4 and t/4 + 8 of the
+// slab, so each row is spread over the 4 consecutive threads of a lane group:
+//   16x256b, per 8 columns: registers (row t/4: columns 2(t%4), 2(t%4)+1),
+//                            (row t/4+8: the same two columns);
+//   16x128b, per 4 columns: (row t/4: column t%4), (row t/4+8: column t%4).
+// A bf16x2 word made from the first pair of a 16x256b group lands, through
+// 16x128b, in the packed column (column of the pair)/2: a score row turns
+// into its packed P row in place.
+__device__ __forceinline__ void slab_ld16(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void slab_ld32(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void slab_ld64(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 16 fp32 columns of the slab back to TMEM in the 16x256b layout (no wait).
+__device__ __forceinline__ void slab_st16(uint32_t taddr, const float (&v)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x2.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+          taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+      : "memory");
+}
+// Packed bf16x2 P words in the 16x128b layout: 8, 16 or 32 packed columns
+// (from 16, 32 or 64 score columns), no wait.
+__device__ __forceinline__ void slab_st_p8(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.16x128b.x2.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+__device__ __forceinline__ void slab_st_p16(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+__device__ __forceinline__ void slab_st_p32(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+// Columns of a 16x256b register block that lie at or beyond `valid` become
+// -inf; c0 is the block's first column, j4 = t % 4.
+template <int R>
+__device__ __forceinline__ void slab_mask(float (&v)[4 * R], int c0, int j4, int valid) {
+#pragma unroll
+  for (int g = 0; g < R; ++g) {
+    const int col = c0 + 8 * g + 2 * j4;
+    if (col >= valid) {
+      v[4 * g] = -INFINITY;
+      v[4 * g + 2] = -INFINITY;
+    }
+    if (col + 1 >= valid) {
+      v[4 * g + 1] = -INFINITY;
+      v[4 * g + 3] = -INFINITY;
+    }
+  }
+}
+// Running maxima of this thread's part of its two rows.
+template <int R>
+__device__ __forceinline__ void slab_max(const float (&v)[4 * R], float& t0, float& t1) {
+#pragma unroll
+  for (int g = 0; g < R; ++g) {
+    t0 = fmax3(t0, v[4 * g], v[4 * g + 1]);
+    t1 = fmax3(t1, v[4 * g + 2], v[4 * g + 3]);
+  }
+}
+// Reduction over the 4 threads that share a row.
+__device__ __forceinline__ float row4_max(float x) {
+  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
+  return fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
+}
+__device__ __forceinline__ float row4_sum(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  return x + __shfl_xor_sync(0xffffffffu, x, 2);
+}
+// P = 2^(S*c - m_row) for a 16x256b register block of both rows, packed to
+// bf16x2 words in the 16x128b order; the fp32 exponentials are added to the
+// rows' partial sums l0, l1.
+template <int R>
+__device__ __forceinline__ void slab_exp(float (&v)[4 * R], float c, float neg_m0, float neg_m1,
+                                         uint32_t (&pk)[2 * R], float& l0, float& l1) {
+#pragma unroll
+  for (int g = 0; g < R; ++g) {
+    fma2(v[4 * g], v[4 * g + 1], c, neg_m0);
+    fma2(v[4 * g + 2], v[4 * g + 3], c, neg_m1);
+  }
+#pragma unroll
+  for (int e = 0; e < 4 * R; ++e) v[e] = ex2(v[e]);
+  float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+  for (int g = 0; g < R; ++g) {
+    pk[2 * g] = pack_bf16x2(v[4 * g], v[4 * g + 1]);
+    pk[2 * g + 1] = pack_bf16x2(v[4 * g + 2], v[4 * g + 3]);
+    add2(a0, a1, v[4 * g], v[4 * g + 1]);
+    add2(b0, b1, v[4 * g + 2], v[4 * g + 3]);
+  }
+  l0 += a0 + a1;
+  l1 += b0 + b1;
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
