@@ -57,6 +57,7 @@ constexpr int kQTile = 128;                  // queries per broadcast tile (MMA 
 constexpr int kKTileBytes = kKeyTile * kRowBytes;
 constexpr int kQTileBytes = kQTile * kRowBytes;
 constexpr int kAggStages = 8;
+constexpr int kSBuf = 2;                     // score (and P) buffers per aggregation group
 constexpr int kBcStages = 4;
 constexpr int kMaxAgents = 256;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale only when the max grows by > 2^8
@@ -83,7 +84,8 @@ struct BcParams {
 struct AggBars {
   uint64_t full[kAggStages], empty[kAggStages];
   uint64_t a_full, a_empty;
-  uint64_t s_full[2][2], p_full[2][2], pv_done[2][2];   // [group][score buffer]
+  uint64_t s_full[2][kSBuf], s_free[2][kSBuf];    // [group][score buffer]
+  uint64_t p_full[2][kSBuf], pv_done[2][kSBuf];   // [group][P buffer]
   uint64_t x_pub, x_done;    // group 1 -> group 0 hand-over per segment (k <= 128)
   uint64_t drain[2];
   uint32_t tmem_base;
@@ -95,7 +97,8 @@ struct AggBars {
 struct BcBars {
   uint64_t q_full[kBcStages], q_empty[kBcStages];
   uint64_t ag_full, ag_empty;
-  uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+  uint64_t s_full[2], o_full[2], o_free[2];
+  uint64_t p_chunk[2][4];    // [group][64-column chunk of P]: written by the group
   uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
@@ -155,8 +158,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->a_full, 1);
     mbar_init(&bars->a_empty, 2);                 // both issuers finish the segment
     for (int g = 0; g < 2; ++g) {
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < kSBuf; ++b) {
         mbar_init(&bars->s_full[g][b], 1);
+        mbar_init(&bars->s_free[g][b], kSoftmaxThreads);
         mbar_init(&bars->p_full[g][b], kSoftmaxThreads);
         mbar_init(&bars->pv_done[g][b], 1);
       }
@@ -179,8 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   pdl_trigger();
   const uint32_t tmem = bars->tmem_base;
-  // TMEM columns: score buffer b of group g at g*128 + b*64 (P over its first
-  // 32 columns), U of group g at 256 + g*128 (dn columns).
+  // TMEM columns of group g: score buffers at g*256 + {0, 64}, bf16 P buffers
+  // at g*256 + {128, 160} (32 columns each), U at g*256 + 192 (dn <= 64).  A
+  // score buffer is free again once the softmax has loaded it; a P buffer
+  // once the P V that read it has completed.
 
   if (warp == 0) {
     if (lane == 0) {
@@ -230,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_pv = idesc_bf16(128, dn, 0, 1);
       const uint32_t sA_addr = smem_u32(sA) + (two ? g : 0) * 128 * kRowBytes;
       const uint32_t sK_addr = smem_u32(sK), sV_addr = smem_u32(sV);
-      const uint32_t u_tm = tmem + 256 + g * 128;
+      const uint32_t u_tm = tmem + g * 256 + 192;
       long long it0 = 0;
       int seg = 0;
       int cnt_s = 0, cnt_p = 0;
@@ -246,11 +252,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const long long itg = it0 + i;
           const int s = (int)(itg % kAggStages);
           if (!mbar_wait(&bars->full[s], (uint32_t)(itg / kAggStages) & 1, abort)) return false;
-          const int J = cnt_s, b = J & 1;
-          if (J >= 2 && !mbar_wait(&bars->pv_done[g][b], (uint32_t)((J >> 1) - 1) & 1, abort))
-            return false;           // the buffer's previous P has been consumed
+          const int J = cnt_s, b = J % kSBuf;
+          if (J >= kSBuf &&
+              !mbar_wait(&bars->s_free[g][b], (uint32_t)(J / kSBuf - 1) & 1, abort))
+            return false;           // the softmax has loaded the buffer's previous S
           tc_fence_after();
-          const uint32_t d_tm = tmem + g * 128 + b * 64;
+          const uint32_t d_tm = tmem + g * 256 + b * 64;
           for (int kk = 0; kk < d16; ++kk) {
             const uint64_t da = sw128_desc(sA_addr + kk * 32, 16);
             const uint64_t db = sw128_desc(sK_addr + s * kKTileBytes + kk * 32, 16);
@@ -263,10 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto issue_pv = [&](int i) -> bool {
           const long long itg = it0 + i;
           const int s = (int)(itg % kAggStages);
-          const int J = cnt_p, b = J & 1;
-          if (!mbar_wait(&bars->p_full[g][b], (uint32_t)(J >> 1) & 1, abort)) return false;
+          const int J = cnt_p, b = J % kSBuf;
+          if (!mbar_wait(&bars->p_full[g][b], (uint32_t)(J / kSBuf) & 1, abort)) return false;
           tc_fence_after();
-          const uint32_t p_tm = tmem + g * 128 + b * 64;
+          const uint32_t p_tm = tmem + g * 256 + 128 + b * 32;
           for (int kk = 0; kk < kKeyTile / 16; ++kk) {
             const uint64_t dv = sw128_desc(sV_addr + s * kKTileBytes + kk * 2048, 8192);
             mma_ts(u_tm, p_tm + kk * 8, dv, idesc_pv, (!first || kk > 0) ? 1u : 0u);
@@ -278,17 +285,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         // this group's tiles of the segment: all of them for two agent tiles,
-        // else every other one; one tile of look-ahead (S of the next tile is
-        // issued before P V of the current one)
+        // else every other one.  S of the tile two ahead is issued as soon as
+        // the softmax has loaded the current tile's scores, before P V of the
+        // current tile (which waits for the end of its softmax).
         const int i0 = two ? 0 : g, step = two ? 1 : 2;
         // In two-agent-tile mode both groups take every key tile; start group 1
         // one softmax behind group 0 so their SFU-bound phases interleave.
         if (two && g == 1 && seg == 0 && n > 0 &&
             !mbar_wait(&bars->p_full[0][0], 0, abort))
           ok = false;
-        if (ok && i0 < n) ok = issue_s(i0);
+        constexpr int kAhead = kSBuf;   // S(i + kAhead) reuses the buffer S(i) frees
+        for (int q = 0, i = i0; q < kAhead && i < n && ok; ++q, i += step) ok = issue_s(i);
         for (int i = i0; i < n && ok; i += step) {
-          if (i + step < n) ok = issue_s(i + step);
+          if (i + kAhead * step < n) ok = issue_s(i + kAhead * step);
           if (ok) ok = issue_pv(i);
         }
         mma_commit(&bars->a_empty);
@@ -312,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int j4 = lane & 3;
     const int r0 = slab + (lane >> 2), r1 = r0 + 8;      // this thread's two rows
     const uint32_t slab_off = (uint32_t)slab << 16;
-    const uint32_t u_col = tmem + slab_off + 256 + g * 128;
+    const uint32_t u_col = tmem + slab_off + g * 256 + 192;
     const int row_base = two ? g * 128 : 0;   // agent of TMEM lane 0 in this group
     const bool warp_active = row_base + slab < p.k;
     int J = 0, seg = 0;
@@ -327,14 +336,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool first = true;
       for (int i = 0; i < n; ++i) {
         if (!two && (i & 1) != g) continue;
-        const int b = J & 1;
-        const uint32_t s_col = tmem + slab_off + g * 128 + b * 64;
+        const int b = J % kSBuf;
+        const uint32_t s_col = tmem + slab_off + g * 256 + b * 64;
         const int valid = min(kKeyTile, p.N - (int)(t + i - bh * tps) * kKeyTile);
-        if (ok) ok = warp_wait(&bars->s_full[g][b], (uint32_t)(J >> 1) & 1, abort);
+        if (ok) ok = warp_wait(&bars->s_full[g][b], (uint32_t)(J / kSBuf) & 1, abort);
+        tc_fence_after();
+        float v[32];
+        if (ok && warp_active) slab_ld64(s_col, v);
+        tc_fence_before();
+        mbar_arrive(&bars->s_free[g][b]);       // the tensor core may overwrite S now
+        // The P buffer's previous contents (tile J-2) must have been read.
+        // Every warp waits, including one with no agent rows: its arrival on
+        // p_full for this tile must not come before that phase completed, or
+        // it would count towards tile J-2 (a score buffer is released as soon
+        // as it is loaded, so warps can be up to two tiles apart).
+        if (ok && J >= kSBuf)
+          ok = warp_wait(&bars->pv_done[g][b], (uint32_t)(J / kSBuf - 1) & 1, abort);
         tc_fence_after();
         if (ok && warp_active) {
-          float v[32];
-          slab_ld64(s_col, v);
           if (valid < kKeyTile) slab_mask<8>(v, 0, j4, valid);   // ragged last tile
           float t0 = -INFINITY, t1 = -INFINITY;
           slab_max<8>(v, t0, t1);
@@ -348,7 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 t0 > m0 + kRescaleThreshold || t1 > m1 + kRescaleThreshold)) {
             // a running max grew a lot: once the previous P V has landed,
             // rescale the slab's U rows and sums by 2^(m_old - m_new)
-            ok = warp_wait(&bars->pv_done[g][(J - 1) & 1], (uint32_t)((J - 1) >> 1) & 1, abort);
+            ok = warp_wait(&bars->pv_done[g][(J - 1) % kSBuf], (uint32_t)((J - 1) / kSBuf) & 1,
+                           abort);
             tc_fence_after();
             if (ok) {
               const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
@@ -370,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) {
             uint32_t pk[16];
             slab_exp<8>(v, p.c, -m0, -m1, pk, l0, l1);
-            slab_st_p32(s_col, pk);
+            slab_st_p32(tmem + slab_off + g * 256 + 128 + b * 32, pk);
             tmem_wait_st();
           }
         }
@@ -382,7 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int slot = (int)(cta - ((bh * tps + 1) * p.ctas - 1) / p.total_tiles);
       const long long slot_row = (bh * p.slots + slot) * (long long)p.k;
       if (n_mine > 0 && ok)
-        ok = warp_wait(&bars->pv_done[g][(J - 1) & 1], (uint32_t)((J - 1) >> 1) & 1, abort);
+        ok = warp_wait(&bars->pv_done[g][(J - 1) % kSBuf], (uint32_t)((J - 1) / kSBuf) & 1,
+                       abort);
       tc_fence_after();
       l0 = row4_sum(l0);
       l1 = row4_sum(l1);
@@ -432,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (ok && warp_active) {            // warp-uniform: the TMEM loads are warp-collective
           const bool has1 = (n / 2) > 0;
-          const uint32_t u1_col = tmem + slab_off + 256 + 128;
+          const uint32_t u1_col = tmem + slab_off + 256 + 192;
           float mm0 = m0, mm1 = m1, s0 = 1.f, s1 = 1.f, w0 = 0.f, w1 = 0.f;
           if (has1) {
             const float x0 = bars->m_x[r0], x1 = bars->m_x[r1];
@@ -532,38 +553,62 @@ __device__ __forceinline__ void bc_slab_max(uint32_t s_col, int k, int kpad, int
   }
 }
 
+// TMEM column (within a 256-column buffer) of the bf16 P of 64-score-column
+// chunk ch.  "Packed" layout (S and O fit side by side, kpad + dn <= 256):
+// chunk ch's P at 32 ch, i.e. each score column's P at half its column, and
+// O at kpad.  "Wide" layout (kpad + dn > 256): chunks 0 and 1 pack into
+// [0, 64), O takes [64, 128) once chunk 1 has been read, and every later
+// chunk's P stays at the start of its own score columns.  Either way a P
+// store only lands on score columns its warp has already read and never on
+// O, so P V can run while later chunks are still being computed.
+__device__ __forceinline__ int bc_p_col(int ch, bool wide) { return (wide && ch >= 2) ? 64 * ch : 32 * ch; }
+
 // P = 2^(S*c - m_row) as bf16 for score columns [0, kpad) (columns >= k give
-// 0), written over the same rows at packed column (score column)/2: a block's
-// P lands on columns this warp has already read.  Adds the exponentials to
-// the partial row sums l0, l1.
-__device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int j4, float c_scale,
-                                            float neg_m0, float neg_m1, float& l0, float& l1) {
-  int c = 0;
+// 0), placed by bc_p_col.  Adds the exponentials to the partial row sums l0,
+// l1.  After each 64-column chunk the thread arrives on that chunk's barrier
+// (whether or not it did the work).
+__device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int j4, bool wide,
+                                            float c_scale, float neg_m0, float neg_m1, float& l0,
+                                            float& l1, bool run, uint64_t* chunk_bar) {
+  int c = 0, ch = 0;
 #pragma unroll 1
-  for (; c + 64 <= kpad; c += 64) {
-    float v[32];
-    uint32_t pk[16];
-    slab_ld64(s_col + c, v);
-    if (c + 64 > k) slab_mask<8>(v, c, j4, k);
-    slab_exp<8>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
-    slab_st_p32(s_col + c / 2, pk);
-  }
-  if (c + 32 <= kpad) {
-    float v[16];
-    uint32_t pk[8];
-    slab_ld32(s_col + c, v);
-    if (c + 32 > k) slab_mask<4>(v, c, j4, k);
-    slab_exp<4>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
-    slab_st_p16(s_col + c / 2, pk);
-    c += 32;
+  for (; c + 64 <= kpad; c += 64, ++ch) {
+    if (run) {
+      float v[32];
+      uint32_t pk[16];
+      slab_ld64(s_col + c, v);
+      if (c + 64 > k) slab_mask<8>(v, c, j4, k);
+      slab_exp<8>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
+      slab_st_p32(s_col + bc_p_col(ch, wide), pk);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    mbar_arrive(&chunk_bar[ch]);
   }
   if (c < kpad) {
-    float v[8];
-    uint32_t pk[4];
-    slab_ld16(s_col + c, v);
-    if (c + 16 > k) slab_mask<2>(v, c, j4, k);
-    slab_exp<2>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
-    slab_st_p8(s_col + c / 2, pk);
+    if (run) {
+      const uint32_t pc = s_col + bc_p_col(ch, wide);
+      if (c + 32 <= kpad) {
+        float v[16];
+        uint32_t pk[8];
+        slab_ld32(s_col + c, v);
+        if (c + 32 > k) slab_mask<4>(v, c, j4, k);
+        slab_exp<4>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
+        slab_st_p16(pc, pk);
+      }
+      const int c16 = c + ((kpad - c) & 32);
+      if (c16 < kpad) {
+        float v[8];
+        uint32_t pk[4];
+        slab_ld16(s_col + c16, v);
+        if (c16 + 16 > k) slab_mask<2>(v, c16, j4, k);
+        slab_exp<2>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
+        slab_st_p8(pc + (c16 - c) / 2, pk);
+      }
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    mbar_arrive(&chunk_bar[ch]);
   }
 }
 
@@ -591,9 +636,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kpad = round16(p.k);
   const int d16 = (p.d + 15) >> 4;
   const int dn = d16 * 16;
-  // Columns of a 256-column TMEM buffer: S over [0, kpad), then P (bf16x2)
-  // over [0, kpad/2), O (dn columns) after P.
-  const int o_col = round16(kpad / 2);
+  // Columns of a 256-column TMEM buffer: S over [0, kpad); P and O placed as
+  // bc_p_col describes.
+  const bool wide = kpad + dn > 256;
+  const int o_col = wide ? 64 : kpad;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kBcStages; ++s) {
       mbar_init(&bars->q_full[s], 1);
@@ -603,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->ag_empty, 2);          // both issuers are done with the slice
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], kSoftmaxThreads);
+      for (int c = 0; c < 4; ++c) mbar_init(&bars->p_chunk[i][c], kSoftmaxThreads);
       mbar_init(&bars->o_full[i], 1);
       mbar_init(&bars->o_free[i], kSoftmaxThreads);
       mbar_init(&bars->drain[i], 1);
@@ -625,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();
   const uint32_t tmem = bars->tmem_base;
   // TMEM: buffer g (tiles j with j % 2 == g) at column g*256 holds S, then P
-  // and O as laid out above (o_col + dn <= 128 + 64).
+  // and O as laid out above.
 
   if (warp == 0) {
     if (lane == 0) {
@@ -693,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Start group 1 one softmax behind group 0, so that one group's
         // exponentials overlap the other group's MMA and epilogue phases
         // instead of both contending for the SFU at the same time.
-        if (g == 1 && u == 0 && !mbar_wait(&bars->p_full[0], 0, abort)) {
+        if (g == 1 && u == 0 && !mbar_wait(&bars->p_chunk[0][(kpad - 1) / 64], 0, abort)) {
           ok = false;
           break;
         }
@@ -714,14 +760,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bars->s_full[g]);
         mma_commit(&bars->q_empty[s]);
-        // O = P V_A once the group has written P
-        if (!mbar_wait(&bars->p_full[g], u & 1, abort)) {
-          ok = false;
-          break;
+        // O = P V_A, 64 agents at a time as the group writes P (in the wide
+        // layout O's columns are free only once chunk 1 has been read)
+        int kk = 0;
+        for (int ch = 0; ch * 64 < kpad && ok; ++ch) {
+          if (!mbar_wait(&bars->p_chunk[g][ch], u & 1, abort)) {
+            ok = false;
+            break;
+          }
+          if (wide && ch == 0) continue;
+          tc_fence_after();
+          const int kk_end = min(kpad / 16, 4 * ch + 4);
+          for (; kk < kk_end; ++kk)   // agents [16 kk, 16 kk + 16)
+            mma_ts(o_tm, s_tm + bc_p_col(kk >> 2, wide) + (kk & 3) * 8,
+                   sw128_desc(sVA_addr + kk * 2048, 8192), idesc_pv, kk > 0);
         }
-        tc_fence_after();
-        for (int kk = 0; kk < kpad / 16; ++kk)   // agents [16 kk, 16 kk + 16): P column 8 kk
-          mma_ts(o_tm, s_tm + kk * 8, sw128_desc(sVA_addr + kk * 2048, 8192), idesc_pv, kk > 0);
+        if (!ok) break;
         mma_commit(&bars->o_full[g]);
         ++u;
       }
@@ -752,17 +806,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q0 = (int)(t - bh * tps) * kQTile;
       if (ok) ok = warp_wait(&bars->s_full[g], u & 1, abort);
       tc_fence_after();
-      float l0 = 0.f, l1 = 0.f;
+      float l0 = 0.f, l1 = 0.f, t0 = -INFINITY, t1 = -INFINITY;
       if (ok) {
-        float t0 = -INFINITY, t1 = -INFINITY;
         bc_slab_max(s_col, p.k, kpad, j4, t0, t1);
         t0 = row4_max(t0) * p.c;
         t1 = row4_max(t1) * p.c;
-        bc_slab_exp(s_col, p.k, kpad, j4, p.c, -t0, -t1, l0, l1);
-        tmem_wait_st();
       }
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[g]);
+      bc_slab_exp(s_col, p.k, kpad, j4, wide, p.c, -t0, -t1, l0, l1, ok, bars->p_chunk[g]);
       const float inv0 = 1.f / row4_sum(l0), inv1 = 1.f / row4_sum(l1);
       // epilogue: O = (P V_A) / l -> bf16 -> swizzled staging tile -> TMA store
       if (ok) ok = warp_wait(&bars->o_full[g], u & 1, abort);

@@ -123,6 +123,35 @@ def test_stage_broadcast(dtype, N, n_agents, d):
     assert_close(f64(out.cpu()), ref, dtype, "O")
 
 
+@pytest.mark.parametrize("B,H,N,n_agents,d", [(16, 2, 3136, 49, 32), (2, 4, 8192, 144, 64),
+                                              (2, 8, 16384, 256, 40), (64, 3, 196, 49, 64)])
+def test_tensor_core_stages_are_repeatable(B, H, N, n_agents, d):
+    """Repeated launches of the bf16 aggregation and broadcast give bit-identical
+    results: many key tiles per CTA, agent counts that leave some softmax warps
+    without rows (49, 144) and both agent-tile modes.  A missing dependency
+    between the softmax warps, the MMA issuers and the TMEM buffers shows up
+    as run-to-run drift even when each run stays inside the tolerance."""
+    q, k, v = (t.cuda() for t in random_qkv((B, H, N, d), seed=N + d, dtype=torch.bfloat16))
+    g = torch.Generator().manual_seed(17)
+    agents = (torch.randn((B, H, n_agents, d), generator=g) * 0.5).to(torch.bfloat16).cuda()
+    scale = 1 / math.sqrt(d)
+    vas, outs = [], []
+    for _ in range(6):
+        va = torch.full((B, H, n_agents, d), 3.0, dtype=torch.bfloat16, device="cuda")
+        eva.agent_attn_stage_aggregate(agents, H * n_agents * d, k, v, None, va, B, H, N, d,
+                                       n_agents, scale, eva.AA_BF16)
+        out = torch.full_like(q, 3.0)
+        eva.agent_attn_stage_broadcast(q, agents, H * n_agents * d, va, out, B, H, N, d,
+                                       n_agents, scale, eva.AA_BF16)
+        torch.cuda.synchronize()
+        vas.append(va)
+        outs.append(out)
+    assert eva.agent_attn_check_device_error(check=False) == 0
+    for r in range(1, 6):
+        assert torch.equal(vas[r], vas[0]), f"V_A differs in run {r}"
+        assert torch.equal(outs[r], outs[0]), f"O differs in run {r}"
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_learnable_agents_batch_stride_and_permutation(dtype):
     B, H, gh, gw, d, n_ag = 2, 2, 20, 20, 32, 40
