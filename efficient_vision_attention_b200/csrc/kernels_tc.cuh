@@ -57,7 +57,7 @@ constexpr int kQTile = 128;                  // queries per broadcast tile (MMA 
 constexpr int kKTileBytes = kKeyTile * kRowBytes;
 constexpr int kQTileBytes = kQTile * kRowBytes;
 constexpr int kAggStages = 8;
-constexpr int kSBuf = 2;                     // score (and P) buffers per aggregation group
+constexpr int kSBuf = 3;                     // score buffers per aggregation group
 constexpr int kBcStages = 4;
 constexpr int kMaxAgents = 256;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale only when the max grows by > 2^8
@@ -84,8 +84,7 @@ struct BcParams {
 struct AggBars {
   uint64_t full[kAggStages], empty[kAggStages];
   uint64_t a_full, a_empty;
-  uint64_t s_full[2][kSBuf], s_free[2][kSBuf];    // [group][score buffer]
-  uint64_t p_full[2][kSBuf], pv_done[2][kSBuf];   // [group][P buffer]
+  uint64_t s_full[2][kSBuf], p_full[2][kSBuf], pv_done[2][kSBuf];   // [group][score buffer]
   uint64_t x_pub, x_done;    // group 1 -> group 0 hand-over per segment (k <= 128)
   uint64_t drain[2];
   uint32_t tmem_base;
@@ -160,7 +159,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = 0; g < 2; ++g) {
       for (int b = 0; b < kSBuf; ++b) {
         mbar_init(&bars->s_full[g][b], 1);
-        mbar_init(&bars->s_free[g][b], kSoftmaxThreads);
         mbar_init(&bars->p_full[g][b], kSoftmaxThreads);
         mbar_init(&bars->pv_done[g][b], 1);
       }
@@ -183,10 +181,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   pdl_trigger();
   const uint32_t tmem = bars->tmem_base;
-  // TMEM columns of group g: score buffers at g*256 + {0, 64}, bf16 P buffers
-  // at g*256 + {128, 160} (32 columns each), U at g*256 + 192 (dn <= 64).  A
-  // score buffer is free again once the softmax has loaded it; a P buffer
-  // once the P V that read it has completed.
+  // TMEM columns of group g: score buffers at g*256 + {0, 64, 128} (the bf16
+  // P of a tile is written over the first 32 columns of its scores), U at
+  // g*256 + 192 (dn <= 64).  A score buffer is free again once the P V that
+  // read its P has completed.
 
   if (warp == 0) {
     if (lane == 0) {
@@ -254,8 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&bars->full[s], (uint32_t)(itg / kAggStages) & 1, abort)) return false;
           const int J = cnt_s, b = J % kSBuf;
           if (J >= kSBuf &&
-              !mbar_wait(&bars->s_free[g][b], (uint32_t)(J / kSBuf - 1) & 1, abort))
-            return false;           // the softmax has loaded the buffer's previous S
+              !mbar_wait(&bars->pv_done[g][b], (uint32_t)(J / kSBuf - 1) & 1, abort))
+            return false;           // the buffer's previous P has been consumed
           tc_fence_after();
           const uint32_t d_tm = tmem + g * 256 + b * 64;
           for (int kk = 0; kk < d16; ++kk) {
@@ -273,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int J = cnt_p, b = J % kSBuf;
           if (!mbar_wait(&bars->p_full[g][b], (uint32_t)(J / kSBuf) & 1, abort)) return false;
           tc_fence_after();
-          const uint32_t p_tm = tmem + g * 256 + 128 + b * 32;
+          const uint32_t p_tm = tmem + g * 256 + b * 64;
           for (int kk = 0; kk < kKeyTile / 16; ++kk) {
             const uint64_t dv = sw128_desc(sV_addr + s * kKTileBytes + kk * 2048, 8192);
             mma_ts(u_tm, p_tm + kk * 8, dv, idesc_pv, (!first || kk > 0) ? 1u : 0u);
@@ -285,16 +283,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         // this group's tiles of the segment: all of them for two agent tiles,
-        // else every other one.  S of the tile two ahead is issued as soon as
-        // the softmax has loaded the current tile's scores, before P V of the
-        // current tile (which waits for the end of its softmax).
+        // else every other one; two tiles of look-ahead (S of the tile after
+        // next is issued before P V of the current one, into the buffer whose
+        // P V has completed)
         const int i0 = two ? 0 : g, step = two ? 1 : 2;
         // In two-agent-tile mode both groups take every key tile; start group 1
         // one softmax behind group 0 so their SFU-bound phases interleave.
         if (two && g == 1 && seg == 0 && n > 0 &&
             !mbar_wait(&bars->p_full[0][0], 0, abort))
           ok = false;
-        constexpr int kAhead = kSBuf;   // S(i + kAhead) reuses the buffer S(i) frees
+        constexpr int kAhead = kSBuf - 1;
         for (int q = 0, i = i0; q < kAhead && i < n && ok; ++q, i += step) ok = issue_s(i);
         for (int i = i0; i < n && ok; i += step) {
           if (i + kAhead * step < n) ok = issue_s(i + kAhead * step);
@@ -341,19 +339,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int valid = min(kKeyTile, p.N - (int)(t + i - bh * tps) * kKeyTile);
         if (ok) ok = warp_wait(&bars->s_full[g][b], (uint32_t)(J / kSBuf) & 1, abort);
         tc_fence_after();
-        float v[32];
-        if (ok && warp_active) slab_ld64(s_col, v);
-        tc_fence_before();
-        mbar_arrive(&bars->s_free[g][b]);       // the tensor core may overwrite S now
-        // The P buffer's previous contents (tile J-2) must have been read.
-        // Every warp waits, including one with no agent rows: its arrival on
-        // p_full for this tile must not come before that phase completed, or
-        // it would count towards tile J-2 (a score buffer is released as soon
-        // as it is loaded, so warps can be up to two tiles apart).
-        if (ok && J >= kSBuf)
-          ok = warp_wait(&bars->pv_done[g][b], (uint32_t)(J / kSBuf - 1) & 1, abort);
-        tc_fence_after();
+        // A tile's scores are only written after the P V of the buffer's
+        // previous tile (which needed every warp's P) has completed, so the
+        // warps of a group are never more than kSBuf - 1 tiles apart and a
+        // barrier phase only ever collects arrivals of one tile.
         if (ok && warp_active) {
+          float v[32];
+          slab_ld64(s_col, v);
           if (valid < kKeyTile) slab_mask<8>(v, 0, j4, valid);   // ragged last tile
           float t0 = -INFINITY, t1 = -INFINITY;
           slab_max<8>(v, t0, t1);
@@ -390,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) {
             uint32_t pk[16];
             slab_exp<8>(v, p.c, -m0, -m1, pk, l0, l1);
-            slab_st_p32(tmem + slab_off + g * 256 + 128 + b * 32, pk);
+            slab_st_p32(s_col, pk);
             tmem_wait_st();
           }
         }
