@@ -52,6 +52,7 @@ def _load():
         lib.oracle_agent_broadcast.argtypes = [dp, dp, dp, i64, i64, i64, i64, ctypes.c_double, dp]
         lib.oracle_agent_attn.argtypes = [dp, dp, dp, dp, i64, i64, i64, i64, i64, i64, i64, i64,
                                           ctypes.c_double, dp, dp, dp]
+        lib.oracle_dwc.argtypes = [dp, dp, dp, i64, i64, i64, i64, i64, dp]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -145,3 +146,30 @@ def agent_attn(q, k, v, grid_h: int, grid_w: int, pool_h: int, pool_w: int,
                           bh, n, d, grid_h, grid_w, pool_h, pool_w, n_agents, float(scale),
                           _ptr(scratch_a), _ptr(scratch_va), _ptr(o))
     return o.reshape(lead + o.shape[1:])
+
+
+def dwc(v, w, bias, grid_h: int, grid_w: int) -> np.ndarray:
+    """Depth-wise 3x3 convolution of V [B, H, N, d] over its token grid with
+    per-(head, channel) kernels w [H, d, 3, 3] and optional bias [H, d]
+    (zero padding, output on the same grid)."""
+    v = _f64(v)
+    B, H, n, d = v.shape
+    if n != grid_h * grid_w:
+        raise ValueError("N must equal grid_h * grid_w")
+    w = _f64(w)
+    assert w.shape == (H, d, 3, 3)
+    b = None if bias is None else _f64(bias)
+    if b is not None:
+        assert b.shape == (H, d)
+    out = np.empty_like(v)
+    _load().oracle_dwc(_ptr(v), _ptr(w), _ptr(b) if b is not None else None, B * H, H, grid_h,
+                       grid_w, d, _ptr(out))
+    return out
+
+
+def agent_attn_dwc(q, k, v, grid_h: int, grid_w: int, pool_h: int, pool_w: int, scale: float,
+                   w, bias=None, agents=None) -> np.ndarray:
+    """The full module's output: the Agent Attention forward pass plus the
+    depth-wise convolution term of V."""
+    return (agent_attn(q, k, v, grid_h, grid_w, pool_h, pool_w, scale, agents=agents)
+            + dwc(v, w, bias, grid_h, grid_w))

@@ -144,6 +144,40 @@ void oracle_agent_attn(const double* q, const double* k, const double* v,
   oracle_agent_broadcast(q, a, scratch_va, BH, N, d, n_agents, scale, o);
 }
 
+/* Depth-wise 3x3 convolution of V over its token grid: the DWC term that the
+ * full module adds to the attention output.
+ * [Agent Attention: On the Integration of Softmax and Linear Attention
+ *  (arXiv:2312.08874v3 summary), §4 "Module Enhancements": the full module
+ *  adds a depth-wise convolution term whose cost is k^2 N C with k = 3.]
+ * Each channel c of each head h has its own 3x3 kernel w[h][c][ty][tx] and an
+ * optional bias[h][c]; positions outside the grid contribute zero (padding 1,
+ * stride 1, so the output keeps the grid):
+ *   out[bh][y*gw + x][c] = bias[h][c]
+ *       + sum_{ty,tx in 0..2} w[h][c][ty][tx] * V[bh][(y+ty-1)*gw + (x+tx-1)][c]
+ * with h = bh % H.  v, out: [BH][grid_h*grid_w][d]; w: [H][d][3][3];
+ * bias_or_null: [H][d] or NULL. */
+void oracle_dwc(const double* v, const double* w, const double* bias_or_null, int64_t BH,
+                int64_t H, int64_t grid_h, int64_t grid_w, int64_t d, double* out) {
+  const int64_t N = grid_h * grid_w;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    for (int64_t n = 0; n < N; ++n) {
+      const int64_t h = bh % H, y = n / grid_w, x = n % grid_w;
+      for (int64_t c = 0; c < d; ++c) {
+        double acc = bias_or_null ? bias_or_null[h * d + c] : 0.0;
+        for (int64_t ty = 0; ty < 3; ++ty) {
+          for (int64_t tx = 0; tx < 3; ++tx) {
+            const int64_t yy = y + ty - 1, xx = x + tx - 1;
+            if (yy < 0 || yy >= grid_h || xx < 0 || xx >= grid_w) continue;
+            acc += w[(h * d + c) * 9 + ty * 3 + tx] * v[(bh * N + yy * grid_w + xx) * d + c];
+          }
+        }
+        out[(bh * N + n) * d + c] = acc;
+      }
+    }
+  }
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -232,3 +232,79 @@ def test_oracle_is_fp64_and_deterministic():
     o2 = oracle.agent_attn(q, k, v, 8, 8, 2, 2, 0.2)
     assert o1.dtype == np.float64
     np.testing.assert_array_equal(o1, o2)
+
+
+# ---------------------------------------------------------------- DWC term
+def torch_dwc(v, w, bias, gh, gw):
+    """Library depth-wise convolution (float64 conv2d, one group per channel)."""
+    B, H, N, d = v.shape
+    t = torch.from_numpy(v).reshape(B, H, gh, gw, d).permute(0, 1, 4, 2, 3).reshape(B, H * d, gh, gw)
+    wt = torch.from_numpy(w).reshape(H * d, 1, 3, 3)
+    bt = None if bias is None else torch.from_numpy(bias).reshape(H * d)
+    o = F.conv2d(t, wt, bt, padding=1, groups=H * d)
+    return o.reshape(B, H, d, gh, gw).permute(0, 1, 3, 4, 2).reshape(B, H, N, d).numpy()
+
+
+@pytest.mark.parametrize("gh,gw,d", [(5, 7, 3), (1, 9, 2), (6, 1, 4), (8, 8, 8)])
+def test_dwc_matches_library_depthwise_conv(gh, gw, d):
+    B, H = 2, 3
+    v = rnd((B, H, gh * gw, d), 31)
+    w = rnd((H, d, 3, 3), 32)
+    bias = rnd((H, d), 33)
+    np.testing.assert_allclose(oracle.dwc(v, w, bias, gh, gw), torch_dwc(v, w, bias, gh, gw),
+                               rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(oracle.dwc(v, w, None, gh, gw), torch_dwc(v, w, None, gh, gw),
+                               rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("ty,tx", [(0, 0), (0, 1), (0, 2), (1, 0), (1, 1), (1, 2), (2, 0), (2, 1),
+                                   (2, 2)])
+def test_dwc_single_tap_is_a_zero_filled_shift(ty, tx):
+    """A kernel with one unit tap at (ty, tx) reads V at (y + ty - 1, x + tx - 1)."""
+    gh, gw, d = 4, 6, 2
+    v = rnd((1, 2, gh * gw, d), 34)
+    w = np.zeros((2, d, 3, 3))
+    w[:, :, ty, tx] = 1.0
+    grid = v.reshape(1, 2, gh, gw, d)
+    want = np.zeros_like(grid)
+    dy, dx = ty - 1, tx - 1
+    ys, xs = slice(max(0, -dy), gh - max(0, dy)), slice(max(0, -dx), gw - max(0, dx))
+    ys2, xs2 = slice(max(0, dy), gh - max(0, -dy)), slice(max(0, dx), gw - max(0, -dx))
+    want[:, :, ys, xs] = grid[:, :, ys2, xs2]
+    np.testing.assert_array_equal(oracle.dwc(v, w, None, gh, gw), want.reshape(v.shape))
+
+
+def test_dwc_constant_values_count_the_taps_inside_the_grid():
+    gh, gw, d, c = 5, 4, 3, 1.75
+    v = np.full((1, 1, gh * gw, d), c)
+    w = rnd((1, d, 3, 3), 35)
+    out = oracle.dwc(v, w, None, gh, gw).reshape(gh, gw, d)
+    for y in range(gh):
+        for x in range(gw):
+            inside = np.zeros((3, 3))
+            for ty in range(3):
+                for tx in range(3):
+                    inside[ty, tx] = 0 <= y + ty - 1 < gh and 0 <= x + tx - 1 < gw
+            want = c * (w[0] * inside).sum(axis=(1, 2))
+            np.testing.assert_allclose(out[y, x], want, rtol=1e-14, atol=1e-14)
+
+
+def test_dwc_is_linear_and_bias_only_is_a_broadcast():
+    gh, gw, d = 3, 5, 4
+    v1, v2 = rnd((2, 2, gh * gw, d), 36), rnd((2, 2, gh * gw, d), 37)
+    w = rnd((2, d, 3, 3), 38)
+    lhs = oracle.dwc(2.5 * v1 + v2, w, None, gh, gw)
+    rhs = 2.5 * oracle.dwc(v1, w, None, gh, gw) + oracle.dwc(v2, w, None, gh, gw)
+    np.testing.assert_allclose(lhs, rhs, rtol=1e-12, atol=1e-12)
+    bias = rnd((2, d), 39)
+    out = oracle.dwc(v1, np.zeros((2, d, 3, 3)), bias, gh, gw)
+    np.testing.assert_array_equal(out, np.broadcast_to(bias[None, :, None, :], out.shape))
+
+
+def test_full_module_output_is_attention_plus_dwc():
+    gh, gw, d = 6, 6, 4
+    q, k, v = (rnd((1, 2, gh * gw, d), s) for s in (40, 41, 42))
+    w = rnd((2, d, 3, 3), 43)
+    full = oracle.agent_attn_dwc(q, k, v, gh, gw, 3, 3, 0.5, w)
+    np.testing.assert_allclose(full - oracle.agent_attn(q, k, v, gh, gw, 3, 3, 0.5),
+                               torch_dwc(v, w, None, gh, gw), rtol=1e-12, atol=1e-12)
