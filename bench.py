@@ -328,7 +328,7 @@ def run_native(args, w):
     dom = "aggregate" if stage_ms["aggregate"] >= stage_ms["broadcast"] else "broadcast"
     achieved = half_bytes / (stage_ms[dom] * 1e-3) / 1e9
     both = 2 * half_bytes / ((stage_ms["aggregate"] + stage_ms["broadcast"]) * 1e-3) / 1e9
-    kernel_name = {"aggregate": "agent_aggregate", "broadcast": "agent_broadcast"}[dom]
+    kernel_name = {"aggregate": "agent_aggregate+agent_merge", "broadcast": "agent_broadcast"}[dom]
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_kind": f"of {peak_kind}",
                 "kernel": kernel_name,
