@@ -335,6 +335,32 @@ def run_native(args, w):
                 "algorithmic_bytes_per_launch": half_bytes,
                 "traffic": recorded_traffic(kernel_name, w.name)}
 
+    # The DWC term of the full module (depth-wise 3x3 convolution of V added to
+    # O) on the same workload: its own kernel, HBM-bound (V read, O read and
+    # written), timed with back-to-back launches like the stages above.
+    gw_ = torch.Generator().manual_seed(w.seed + 77)
+    dwc_w = (torch.randn((H, d, 3, 3), generator=gw_) * 0.3).to(dev)
+    dwc_b = (torch.randn((H, d), generator=gw_) * 0.1).to(dev)
+
+    def run_dwc(s):
+        eva.agent_attn_dwc(s["v"], dwc_w, dwc_b, s["out"], B, H, w.grid_h, w.grid_w, d, dt, True,
+                           stream)
+
+    for r in range(3):
+        run_dwc(sets[r % n_sets])
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for r in range(reps):
+        run_dwc(sets[r % n_sets])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dwc_ms = e0.elapsed_time(e1) / reps
+    dwc_bytes = 3 * B * H * N * d * w.elem_bytes
+    dwc = {"kernel": "dwc", "ms": dwc_ms, "algorithmic_bytes_per_launch": dwc_bytes,
+           "achieved_gbs": dwc_bytes / (dwc_ms * 1e-3) / 1e9,
+           "frac": dwc_bytes / (dwc_ms * 1e-3) / 1e9 / peak}
+
     # End to end through the host-buffer entry point: pinned host inputs copied
     # in, result copied out, every step.
     hin = make_inputs(w, seed=replicas.rank_seed(w.seed, rank))
@@ -386,6 +412,7 @@ def run_native(args, w):
         "hbm_frac_aggregate_plus_broadcast": both / peak,
         "stage_ms": stage_ms,
         "roofline": roofline,
+        "dwc_term": dwc,
         "cpu_baseline": base,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,

@@ -13,6 +13,8 @@ from .binding import (  # noqa: F401
     agent_attn_forward_agents,
     agent_attn_forward_host,
     agent_attn_check_device_error,
+    agent_attn_dwc,
+    agent_attn_forward_dwc,
     agent_attn_forward_ws,
     agent_attn_stage_pool,
     agent_attn_stage_aggregate,

@@ -49,6 +49,9 @@ _SIGNATURES = {
     "agent_attn_check_device_error": (_i, []),
     "agent_attn_stage_aggregate_static": (_i, [_vp, _ll, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                                _f, _i, _vp]),
+    "agent_attn_dwc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "agent_attn_forward_dwc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                    _i, _f, _i, _vp]),
 }
 
 # Size of the library's fixed scratch array (AA_STATIC_SCRATCH_BYTES in the header).
@@ -195,4 +198,24 @@ def agent_attn_stage_aggregate_static(agents, agents_batch_stride, k, v, va_f32,
     st = load_library().agent_attn_stage_aggregate_static(
         _ptr(agents), agents_batch_stride, _ptr(k), _ptr(v), _ptr(va_f32), _ptr(va_lowp), B, H, N,
         d, n_agents, scale, dtype, _stream(stream))
+    return _finish(st, check)
+
+
+def agent_attn_dwc(v, w, bias_or_null, out, B, H, grid_h, grid_w, d, dtype, accumulate=False,
+                   stream=None, check=True):
+    """out (+)= depth-wise 3x3 convolution of v over its token grid; w is
+    [H, d, 3, 3] fp32, bias [H, d] fp32 or None."""
+    st = load_library().agent_attn_dwc(_ptr(v), _ptr(w), _ptr(bias_or_null), _ptr(out), B, H,
+                                       grid_h, grid_w, d, dtype, 1 if accumulate else 0,
+                                       _stream(stream))
+    return _finish(st, check)
+
+
+def agent_attn_forward_dwc(q, k, v, agents_or_null, dwc_w, dwc_bias_or_null, out, B, H, N, d,
+                           grid_h, grid_w, pool_h, pool_w, scale, dtype, stream=None, check=True):
+    """The full module output: the forward pass plus the depth-wise convolution of v."""
+    st = load_library().agent_attn_forward_dwc(_ptr(q), _ptr(k), _ptr(v), _ptr(agents_or_null),
+                                               _ptr(dwc_w), _ptr(dwc_bias_or_null), _ptr(out), B,
+                                               H, N, d, grid_h, grid_w, pool_h, pool_w, scale,
+                                               dtype, _stream(stream))
     return _finish(st, check)

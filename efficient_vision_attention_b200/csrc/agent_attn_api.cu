@@ -15,6 +15,7 @@
 
 #include "agent_attn.h"
 #include "common.cuh"
+#include "kernels_dwc.cuh"
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
 
@@ -411,6 +412,40 @@ int pooled_forward(const void* q, const void* k, const void* v, const void* agen
                       static_cast<cudaStream_t>(stream));
 }
 
+// Depth-wise 3x3 term: out (+)= DWConv3x3(v) over the grid, per (head, channel).
+int dwc_impl(const void* v, const float* w, const float* bias, void* out, int B, int H,
+             int grid_h, int grid_w, int d, int dtype, int accumulate, cudaStream_t st, bool pdl) {
+  const long long BH = (long long)B * H;
+  const long long N = (long long)grid_h * grid_w;
+  const long long items = N * (d / 8);
+  if (items >= (1LL << 31)) return AA_ERR_SHAPE;       // per-slice index math is 32-bit
+  const long long blocks = (items + kDwcThreads - 1) / kDwcThreads;
+  const dim3 grid((unsigned)blocks, (unsigned)(BH < 65535 ? BH : 65535));
+  const size_t smem = (size_t)10 * d * sizeof(float);
+  cudaError_t e;
+  if (dtype == AA_FP32)
+    e = launch_kernel(dwc_kernel<float>, grid, dim3(kDwcThreads), smem, st, pdl,
+                      static_cast<const float*>(v), w, bias, static_cast<float*>(out), H, grid_h,
+                      grid_w, d, BH, accumulate);
+  else
+    e = launch_kernel(dwc_kernel<__nv_bfloat16>, grid, dim3(kDwcThreads), smem, st, pdl,
+                      static_cast<const __nv_bfloat16*>(v), w, bias,
+                      static_cast<__nv_bfloat16*>(out), H, grid_h, grid_w, d, BH, accumulate);
+  if (e != cudaSuccess) return cuda_fail(e, "dwc_kernel launch");
+  return AA_OK;
+}
+
+int validate_dwc(const void* v, const float* w, const void* out, int B, int H, int grid_h,
+                 int grid_w, int d, int dtype) {
+  if (dtype != AA_FP32 && dtype != AA_BF16) return AA_ERR_UNSUPPORTED;
+  if (B < 1 || H < 1 || grid_h < 1 || grid_w < 1) return AA_ERR_SHAPE;
+  if (d < 8 || d > 128 || (d % 8) != 0) return AA_ERR_UNSUPPORTED;
+  if ((long long)B * H * grid_h * (long long)grid_w > (1LL << 40)) return AA_ERR_SHAPE;
+  if (!v || !w || !out) return AA_ERR_NULL;
+  if (!aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(w) & 3u)) return AA_ERR_ALIGN;
+  return AA_OK;
+}
+
 // Fixed scratch of agent_attn_stage_aggregate_static: a file-scope device
 // array, so that entry point needs no allocation at all.  Its device address
 // is looked up once per device (with that device current) and cached.
@@ -645,6 +680,31 @@ const char* agent_attn_status_string(int status) {
 }
 
 const char* agent_attn_version(void) { return "0.1.0"; }
+
+int agent_attn_dwc(const void* v, const float* w, const float* bias_or_null, void* out, int B,
+                   int H, int grid_h, int grid_w, int d, int dtype, int accumulate, void* stream) {
+  int rc = validate_dwc(v, w, out, B, H, grid_h, grid_w, d, dtype);
+  if (rc != AA_OK) return rc;
+  if (bias_or_null && (reinterpret_cast<uintptr_t>(bias_or_null) & 3u)) return AA_ERR_ALIGN;
+  return dwc_impl(v, w, bias_or_null, out, B, H, grid_h, grid_w, d, dtype, accumulate ? 1 : 0,
+                  static_cast<cudaStream_t>(stream), false);
+}
+
+int agent_attn_forward_dwc(const void* q, const void* k, const void* v, const void* agents_or_null,
+                           const float* dwc_w, const float* dwc_bias_or_null, void* out, int B,
+                           int H, int N, int d, int grid_h, int grid_w, int pool_h, int pool_w,
+                           float scale, int dtype, void* stream) {
+  int rc = validate_grid(N, grid_h, grid_w, pool_h, pool_w);
+  if (rc != AA_OK) return rc;
+  rc = validate_dwc(v, dwc_w, out, B, H, grid_h, grid_w, d, dtype);
+  if (rc != AA_OK) return rc;
+  if (dwc_bias_or_null && (reinterpret_cast<uintptr_t>(dwc_bias_or_null) & 3u)) return AA_ERR_ALIGN;
+  rc = pooled_forward(q, k, v, agents_or_null, out, B, H, N, d, grid_h, grid_w, pool_h, pool_w,
+                      scale, dtype, nullptr, 0, false, stream);
+  if (rc != AA_OK) return rc;
+  return dwc_impl(v, dwc_w, dwc_bias_or_null, out, B, H, grid_h, grid_w, d, dtype, 1,
+                  static_cast<cudaStream_t>(stream), true);
+}
 
 int agent_attn_check_device_error(void) {
   unsigned int word = 0, zero = 0;

@@ -297,28 +297,32 @@ __global__ void __launch_bounds__(kMergeThreads) agent_merge_kernel(
   const long long split_stride = (long long)n_agents;      // rows between consecutive splits
   const float* ml0 = part_ml + ((slot0)*n_agents + j) * 2;
   const float* u0 = part_u + ((slot0)*n_agents + j) * (long long)d + cq * 4;
-  float mx = -INFINITY;
-  for (int s0 = 0; s0 < n_splits; s0 += kMergeUnroll) {
-    float m[kMergeUnroll];
-#pragma unroll
-    for (int a = 0; a < kMergeUnroll; ++a)
-      m[a] = (s0 + a < n_splits) ? ml0[(s0 + a) * split_stride * 2] : -INFINITY;
-#pragma unroll
-    for (int a = 0; a < kMergeUnroll; ++a) mx = fmaxf(mx, m[a]);
-  }
+  // One pass over the splits, kMergeUnroll at a time: every load of a batch
+  // (running max, running sum and 4 accumulator columns of each split) is in
+  // flight together; the batch's maximum rescales what was combined so far.
+  float mx = -INFINITY, den = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float den = 0.f;
   for (int s0 = 0; s0 < n_splits; s0 += kMergeUnroll) {
     float2 ml[kMergeUnroll];
     float4 u[kMergeUnroll];
 #pragma unroll
     for (int a = 0; a < kMergeUnroll; ++a) {
       const bool ok = s0 + a < n_splits;
-      ml[a] = ok ? *reinterpret_cast<const float2*>(ml0 + (s0 + a) * split_stride * 2)
+      ml[a] = ok ? __ldg(reinterpret_cast<const float2*>(ml0 + (s0 + a) * split_stride * 2))
                  : make_float2(-INFINITY, 0.f);
-      u[a] = ok ? *reinterpret_cast<const float4*>(u0 + (s0 + a) * split_stride * d)
+      u[a] = ok ? __ldg(reinterpret_cast<const float4*>(u0 + (s0 + a) * split_stride * d))
                 : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    float mb = mx;
+#pragma unroll
+    for (int a = 0; a < kMergeUnroll; ++a) mb = fmaxf(mb, ml[a].x);
+    const float r = (mx == -INFINITY) ? 0.f : exp2f(mx - mb);   // rescale of earlier batches
+    den *= r;
+    acc.x *= r;
+    acc.y *= r;
+    acc.z *= r;
+    acc.w *= r;
+    mx = mb;
 #pragma unroll
     for (int a = 0; a < kMergeUnroll; ++a) {
       const float w = (s0 + a < n_splits) ? exp2f(ml[a].x - mx) : 0.f;

@@ -171,6 +171,41 @@ AA_API int agent_attn_stage_aggregate_static(const void* agents, long long agent
                                              void* va_lowp, int B, int H, int N, int d,
                                              int n_agents, float scale, int dtype, void* stream);
 
+/* ---- the depth-wise convolution term of the full module ----
+ *
+ * The full Agent Attention module adds a depth-wise convolution term to the
+ * attention output (arXiv:2312.08874v3 summary, §4 "Module Enhancements": the
+ * full module adds a depth-wise convolution term, cost k^2 N C with k = 3).
+ * Read here as a 3x3 depth-wise convolution of V over the token grid, one
+ * kernel per (head, channel), zero padding, output on the same grid:
+ *   DWC(V)[b,h,y*grid_w+x,c] = bias[h,c]
+ *       + sum_{ty,tx in 0..2} w[h,c,ty,tx] * V[b,h,(y+ty-1)*grid_w+(x+tx-1),c]
+ * (positions outside the grid contribute zero).
+ *
+ * agent_attn_dwc: out (+)= DWC(v).
+ *   v, out        : [B, H, grid_h*grid_w, d] device buffers of `dtype`
+ *                   (16-byte aligned); out may not alias v.
+ *   w             : [H, d, 3, 3] fp32 device buffer (4-byte aligned).
+ *   bias_or_null  : [H, d] fp32 device buffer, or NULL for no bias.
+ *   accumulate    : 0 -> out = DWC(v); non-zero -> out = out + DWC(v)
+ *                   (computed in fp32, rounded once to `dtype`).
+ * Same d / dtype rules as the forward pass, and grid_h*grid_w*d/8 < 2^31
+ * (else AA_ERR_SHAPE); asynchronous on `stream`. */
+AA_API int agent_attn_dwc(const void* v, const float* w, const float* bias_or_null, void* out,
+                          int B, int H, int grid_h, int grid_w, int d, int dtype, int accumulate,
+                          void* stream);
+
+/* The full module output: out = AgentAttention(q, k, v) + DWC(v), i.e.
+ * agent_attn_forward followed by agent_attn_dwc(accumulate = 1) on the same
+ * stream (the convolution kernel reads its V taps while the broadcast is
+ * still running and waits for it only before touching out).  Arguments as
+ * in agent_attn_forward and agent_attn_dwc. */
+AA_API int agent_attn_forward_dwc(const void* q, const void* k, const void* v,
+                                  const void* agents_or_null, const float* dwc_w,
+                                  const float* dwc_bias_or_null, void* out, int B, int H, int N,
+                                  int d, int grid_h, int grid_w, int pool_h, int pool_w,
+                                  float scale, int dtype, void* stream);
+
 /* Human-readable text for a status code (for AA_ERR_CUDA, includes the last
  * CUDA error text seen on the calling thread).  Never NULL. */
 AA_API const char* agent_attn_status_string(int status);

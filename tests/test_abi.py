@@ -130,3 +130,23 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     with pytest.raises(binding.AgentAttnError, match="missing"):
         binding.load_library()
     monkeypatch.setattr(binding, "_lib", None)
+
+
+def test_dwc_validation():
+    base = dict(v=A16, w=A16, bias_or_null=None, out=A16, B=1, H=2, grid_h=8, grid_w=8, d=32,
+                dtype=eva.AA_BF16, accumulate=True, stream=0, check=False)
+    f = eva.agent_attn_dwc
+    assert f(**{**base, "v": None}) == 1
+    assert f(**{**base, "w": None}) == 1
+    assert f(**{**base, "out": ODD}) == 4
+    assert f(**{**base, "d": 36}) == 3
+    assert f(**{**base, "d": 136}) == 3
+    assert f(**{**base, "dtype": 5}) == 3
+    assert f(**{**base, "grid_w": 0}) == 2
+    g = eva.agent_attn_forward_dwc
+    full = dict(q=A16, k=A16, v=A16, agents_or_null=None, dwc_w=A16, dwc_bias_or_null=None,
+                out=A16, B=1, H=1, N=64, d=32, grid_h=8, grid_w=8, pool_h=2, pool_w=2, scale=0.1,
+                dtype=eva.AA_BF16, stream=0, check=False)
+    assert g(**{**full, "dwc_w": None}) == 1
+    assert g(**{**full, "N": 63}) == 2
+    assert g(**{**full, "pool_h": 9}) == 2
