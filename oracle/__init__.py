@@ -53,6 +53,8 @@ def _load():
         lib.oracle_agent_attn.argtypes = [dp, dp, dp, dp, i64, i64, i64, i64, i64, i64, i64, i64,
                                           ctypes.c_double, dp, dp, dp]
         lib.oracle_dwc.argtypes = [dp, dp, dp, i64, i64, i64, i64, i64, dp]
+        lib.oracle_agent_attn_bias.argtypes = [dp, dp, dp, dp, dp, dp, i64, i64, i64, i64, i64,
+                                               i64, i64, i64, i64, ctypes.c_double, dp, dp, dp]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -173,3 +175,62 @@ def agent_attn_dwc(q, k, v, grid_h: int, grid_w: int, pool_h: int, pool_w: int, 
     depth-wise convolution term of V."""
     return (agent_attn(q, k, v, grid_h, grid_w, pool_h, pool_w, scale, agents=agents)
             + dwc(v, w, bias, grid_h, grid_w))
+
+
+def agent_bias(row, col, block, grid_h: int, grid_w: int, pool_h: int, pool_w: int) -> np.ndarray:
+    """Full agent-bias matrix [H, k, N] from its components (the reading of the
+    pages' "column, row and block components"): for agent j and token
+    n = y*grid_w + x,
+        B[h, j, n] = row[h, j, y] + col[h, j, x] + block[h, j, b(y, x)],
+    where b(y, x) = floor(y*pool_h/grid_h)*pool_w + floor(x*pool_w/grid_w) is
+    the cell of the pool_h x pool_w partition of the grid holding the token.
+    row: [H, k, grid_h], col: [H, k, grid_w], block: [H, k, pool_h*pool_w];
+    a component given as None contributes zero (at least one is required)."""
+    parts = [x for x in (row, col, block) if x is not None]
+    H, k = _f64(parts[0]).shape[:2]
+    out = np.zeros((H, k, grid_h, grid_w))
+    if row is not None:
+        out += _f64(row)[:, :, :, None]
+    if col is not None:
+        out += _f64(col)[:, :, None, :]
+    if block is not None:
+        by = (np.arange(grid_h) * pool_h) // grid_h
+        bx = (np.arange(grid_w) * pool_w) // grid_w
+        cell = by[:, None] * pool_w + bx[None, :]
+        out += _f64(block)[:, :, cell]
+    return out.reshape(H, k, grid_h * grid_w)
+
+
+def agent_attn_bias(q, k, v, grid_h: int, grid_w: int, pool_h: int, pool_w: int, scale: float,
+                    b1=None, b2=None, agents=None) -> np.ndarray:
+    """Forward pass with agent bias: b1 [H, k, N] is added to the aggregation
+    logits (agent j, key n), b2 [H, k, N] to the broadcast logits (query n,
+    agent j); either may be None.  Inputs [B, H, N, d]."""
+    q = _f64(q)
+    B, H, n, d = q.shape
+    k3 = _f64(k).reshape(B * H, n, d)
+    v3 = _f64(v).reshape(B * H, n, d)
+    q3 = q.reshape(B * H, n, d)
+    if agents is None:
+        n_agents = pool_h * pool_w
+        a3 = None
+    else:
+        ag = _f64(agents)
+        n_agents = ag.shape[-2]
+        if ag.ndim == 3:
+            ag = np.broadcast_to(ag[None], (B,) + ag.shape)
+        a3 = np.ascontiguousarray(ag.reshape(B * H, n_agents, d))
+    b1 = None if b1 is None else np.ascontiguousarray(_f64(b1))
+    b2 = None if b2 is None else np.ascontiguousarray(_f64(b2))
+    for b in (b1, b2):
+        if b is not None:
+            assert b.shape == (H, n_agents, n)
+    scratch_a = np.empty((B * H, n_agents, d))
+    scratch_va = np.empty((B * H, n_agents, d))
+    o = np.empty_like(q3)
+    _load().oracle_agent_attn_bias(
+        _ptr(q3), _ptr(k3), _ptr(v3), _ptr(a3) if a3 is not None else None,
+        _ptr(b1) if b1 is not None else None, _ptr(b2) if b2 is not None else None,
+        B * H, H, n, d, grid_h, grid_w, pool_h, pool_w, n_agents, float(scale),
+        _ptr(scratch_a), _ptr(scratch_va), _ptr(o))
+    return o.reshape(B, H, n, d)

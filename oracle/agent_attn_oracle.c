@@ -144,6 +144,71 @@ void oracle_agent_attn(const double* q, const double* k, const double* v,
   oracle_agent_broadcast(q, a, scratch_va, BH, N, d, n_agents, scale, o);
 }
 
+/* Agent bias: the logits of both softmaxes get an additive bias.
+ * [Agent Attention: On the Integration of Softmax and Linear Attention
+ *  (arXiv:2312.08874v3 summary), §4 "Module Enhancements": the bias terms B1
+ *  and B2 are incorporated into both attention operations; §6
+ *  "Implementation Details": column, row and block components build the
+ *  full bias.]
+ *   aggregate: V_A[j] = softmax_n(scale * A_j . K_n + b1[h][j][n]) @ V
+ *   broadcast: O[i]   = softmax_j(scale * Q_i . A_j + b2[h][j][i]) @ V_A
+ * b1, b2: [H][n_agents][N] full bias matrices shared over the batch
+ * (h = bh % H), either may be NULL for no bias.  How the full matrices are
+ * built from their components is the caller's (oracle/__init__.py). */
+static void softmax_attend_row_biased(const double* x_row, const double* keys,
+                                      const double* vals, int64_t n_keys, int64_t d,
+                                      double scale, const double* bias, int64_t bias_stride,
+                                      double* work, double* out) {
+  double mx = -INFINITY;
+  for (int64_t n = 0; n < n_keys; ++n) {
+    double s = 0.0;
+    for (int64_t c = 0; c < d; ++c) s += x_row[c] * keys[n * d + c];
+    s = s * scale + (bias ? bias[n * bias_stride] : 0.0);
+    work[n] = s;
+    if (s > mx) mx = s;
+  }
+  double total = 0.0;
+  for (int64_t n = 0; n < n_keys; ++n) {
+    work[n] = exp(work[n] - mx);
+    total += work[n];
+  }
+  for (int64_t c = 0; c < d; ++c) out[c] = 0.0;
+  for (int64_t n = 0; n < n_keys; ++n) {
+    double p = work[n] / total;
+    for (int64_t c = 0; c < d; ++c) out[c] += p * vals[n * d + c];
+  }
+}
+
+void oracle_agent_attn_bias(const double* q, const double* k, const double* v,
+                            const double* agents_or_null, const double* b1, const double* b2,
+                            int64_t BH, int64_t H, int64_t N, int64_t d, int64_t grid_h,
+                            int64_t grid_w, int64_t pool_h, int64_t pool_w, int64_t n_agents,
+                            double scale, double* scratch_a, double* scratch_va, double* o) {
+  const double* a = agents_or_null;
+  if (a == NULL) {
+    oracle_agent_pool(q, BH, N, d, grid_h, grid_w, pool_h, pool_w, scratch_a);
+    a = scratch_a;
+  }
+#pragma omp parallel
+  {
+    double* work = (double*)malloc(sizeof(double) * (size_t)(N > n_agents ? N : n_agents));
+#pragma omp for collapse(2) schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh)
+      for (int64_t j = 0; j < n_agents; ++j)
+        softmax_attend_row_biased(a + (bh * n_agents + j) * d, k + bh * N * d, v + bh * N * d, N,
+                                  d, scale, b1 ? b1 + ((bh % H) * n_agents + j) * N : NULL, 1,
+                                  work, scratch_va + (bh * n_agents + j) * d);
+#pragma omp for collapse(2) schedule(static)
+    for (int64_t bh = 0; bh < BH; ++bh)
+      for (int64_t i = 0; i < N; ++i)
+        softmax_attend_row_biased(q + (bh * N + i) * d, a + bh * n_agents * d,
+                                  scratch_va + bh * n_agents * d, n_agents, d, scale,
+                                  b2 ? b2 + (bh % H) * n_agents * N + i : NULL, N, work,
+                                  o + (bh * N + i) * d);
+    free(work);
+  }
+}
+
 /* Depth-wise 3x3 convolution of V over its token grid: the DWC term that the
  * full module adds to the attention output.
  * [Agent Attention: On the Integration of Softmax and Linear Attention

@@ -34,3 +34,18 @@ def agent_attn_brute(q, a, k, v, scale: float):
     """Returns (O, M) for one slice; O = M @ V."""
     m = mixing_matrix(q, a, k, scale)
     return m @ np.asarray(v, np.float64), m
+
+
+def agent_attn_brute_bias(q, a, k, v, scale: float, b1=None, b2=None):
+    """Biased twin for one slice: M = softmax_rows(Q A^T s + B2^T) @
+    softmax_rows(A K^T s + B1) with b1, b2 given as [n_agents, N]; O = M @ V."""
+    q = np.asarray(q, np.float64)
+    a = np.asarray(a, np.float64)
+    k = np.asarray(k, np.float64)
+    n_agents, n = a.shape[0], q.shape[0]
+    b1 = np.zeros((n_agents, n)) if b1 is None else np.asarray(b1, np.float64)
+    b2 = np.zeros((n_agents, n)) if b2 is None else np.asarray(b2, np.float64)
+    left = _softmax_rows(scale * q @ a.T + b2.T)
+    right = _softmax_rows(scale * a @ k.T + b1)
+    m = left @ right
+    return m @ np.asarray(v, np.float64), m

@@ -308,3 +308,79 @@ def test_full_module_output_is_attention_plus_dwc():
     full = oracle.agent_attn_dwc(q, k, v, gh, gw, 3, 3, 0.5, w)
     np.testing.assert_allclose(full - oracle.agent_attn(q, k, v, gh, gw, 3, 3, 0.5),
                                torch_dwc(v, w, None, gh, gw), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- agent bias
+def bias_parts(H, k, gh, gw, nb, seed, scale=1.0):
+    return (rnd((H, k, gh), seed, scale), rnd((H, k, gw), seed + 1, scale),
+            rnd((H, k, nb), seed + 2, scale))
+
+
+def test_bias_components_build_the_full_matrix_by_grid_cell():
+    """Row, column and block components land on the token's grid row, grid
+    column and cell of the floor partition into pool_h x pool_w blocks."""
+    H, k, gh, gw, ph, pw = 2, 3, 7, 5, 3, 2
+    row, col, block = bias_parts(H, k, gh, gw, ph * pw, 50)
+    full = oracle.agent_bias(row, col, block, gh, gw, ph, pw)
+    for y in range(gh):
+        for x in range(gw):
+            cell = (y * ph // gh) * pw + (x * pw // gw)
+            np.testing.assert_array_equal(full[:, :, y * gw + x],
+                                          row[:, :, y] + col[:, :, x] + block[:, :, cell])
+    # a one-hot block component marks exactly the tokens of that block
+    onehot = np.zeros((1, 1, ph * pw))
+    onehot[0, 0, 4] = 1.0
+    marked = oracle.agent_bias(None, None, onehot, gh, gw, ph, pw).reshape(gh, gw)
+    ys, xs = np.nonzero(marked)
+    assert set(ys * ph // gh) == {4 // pw} and set(xs * pw // gw) == {4 % pw}
+
+
+def test_zero_bias_is_the_plain_forward_pass():
+    q, k, v = (rnd((2, 2, 30, 4), s) for s in (51, 52, 53))
+    z = np.zeros((2, 4, 30))
+    np.testing.assert_array_equal(oracle.agent_attn_bias(q, k, v, 5, 6, 2, 2, 0.4, z, z),
+                                  oracle.agent_attn(q, k, v, 5, 6, 2, 2, 0.4))
+
+
+def test_bias_matches_the_brute_force_mixing_matrix():
+    gh, gw, ph, pw, d = 4, 5, 2, 2, 3
+    q, k, v = (rnd((1, 2, gh * gw, d), s) for s in (54, 55, 56))
+    b1 = oracle.agent_bias(*bias_parts(2, 4, gh, gw, 4, 57), gh, gw, ph, pw)
+    b2 = oracle.agent_bias(*bias_parts(2, 4, gh, gw, 4, 60), gh, gw, ph, pw)
+    got = oracle.agent_attn_bias(q, k, v, gh, gw, ph, pw, 0.7, b1, b2)
+    a = torch_pool(q[0], gh, gw, ph, pw)
+    for h in range(2):
+        o, m = brute.agent_attn_brute_bias(q[0, h], a[h], k[0, h], v[0, h], 0.7, b1[h], b2[h])
+        np.testing.assert_allclose(m.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(got[0, h], o, rtol=1e-11, atol=1e-12)
+
+
+def test_bias_constant_along_the_softmax_axis_changes_nothing():
+    """A per-agent constant in B1 (over keys) and a per-query constant in B2
+    (over agents) cancel in their softmaxes."""
+    gh, gw, ph, pw = 6, 6, 3, 3
+    q, k, v = (rnd((2, 2, 36, 4), s) for s in (63, 64, 65))
+    row1 = np.broadcast_to(rnd((2, 9, 1), 66), (2, 9, gh))           # depends on the agent only
+    b1 = oracle.agent_bias(row1, None, None, gh, gw, ph, pw)
+    row2 = np.broadcast_to(rnd((2, 1, gh), 67), (2, 9, gh))          # depends on the query only
+    col2 = np.broadcast_to(rnd((2, 1, gw), 68), (2, 9, gw))
+    b2 = oracle.agent_bias(row2, col2, None, gh, gw, ph, pw)
+    np.testing.assert_allclose(oracle.agent_attn_bias(q, k, v, gh, gw, ph, pw, 0.5, b1, b2),
+                               oracle.agent_attn(q, k, v, gh, gw, ph, pw, 0.5),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_bias_that_admits_one_token_selects_its_value():
+    """B1 = -1e4 everywhere except token (y*, x*): every agent aggregates exactly
+    V[n*], so every query reads V[n*] whatever B2 is."""
+    gh, gw, ph, pw, ys, xs = 5, 4, 2, 2, 3, 1
+    q, k, v = (rnd((1, 2, gh * gw, 3), s) for s in (69, 70, 71))
+    row = np.full((2, 4, gh), -1e4)
+    row[:, :, ys] = 0.0
+    col = np.full((2, 4, gw), -1e4)
+    col[:, :, xs] = 0.0
+    b1 = oracle.agent_bias(row, col, None, gh, gw, ph, pw)
+    b2 = oracle.agent_bias(*bias_parts(2, 4, gh, gw, 4, 72), gh, gw, ph, pw)
+    got = oracle.agent_attn_bias(q, k, v, gh, gw, ph, pw, 0.5, b1, b2)
+    want = np.broadcast_to(v[:, :, ys * gw + xs][:, :, None, :], got.shape)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
