@@ -361,6 +361,36 @@ def run_native(args, w):
            "achieved_gbs": dwc_bytes / (dwc_ms * 1e-3) / 1e9,
            "frac": dwc_bytes / (dwc_ms * 1e-3) / 1e9 / peak}
 
+    # The forward pass with agent bias (row, column and block components in
+    # both softmaxes) on the same workload; it runs the SIMT kernels.
+    gb_ = torch.Generator().manual_seed(w.seed + 78)
+    nb_ = w.pool_h * w.pool_w
+
+    def bias_triple():
+        return [(torch.randn((H, nk, n_), generator=gb_) * 0.5).to(dev)
+                for n_ in (w.grid_h, w.grid_w, nb_)]
+
+    b1_, b2_ = bias_triple(), bias_triple()
+
+    def run_bias(s):
+        eva.agent_attn_forward_bias(s["q"], s["k"], s["v"], None, b1_, b2_, s["out"], B, H, N, d,
+                                    w.grid_h, w.grid_w, w.pool_h, w.pool_w, w.scale, dt, stream)
+
+    bias_fwd = None
+    if not w.learnable_agents:
+        run_bias(sets[0])
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for r in range(3):
+            run_bias(sets[r % n_sets])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        b_ms = e0.elapsed_time(e1) / 3
+        bias_fwd = {"ms_per_forward": b_ms, "value": B * H * N / (b_ms * 1e-3), "unit": UNIT,
+                    "path": "simt"}
+
     # End to end through the host-buffer entry point: pinned host inputs copied
     # in, result copied out, every step.
     hin = make_inputs(w, seed=replicas.rank_seed(w.seed, rank))
@@ -413,6 +443,7 @@ def run_native(args, w):
         "stage_ms": stage_ms,
         "roofline": roofline,
         "dwc_term": dwc,
+        "agent_bias_forward": bias_fwd,
         "cpu_baseline": base,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,

@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     AgentAttnError,
     agent_attn_forward,
     agent_attn_forward_agents,
+    agent_attn_forward_bias,
     agent_attn_forward_host,
     agent_attn_check_device_error,
     agent_attn_dwc,

@@ -49,6 +49,8 @@ _SIGNATURES = {
     "agent_attn_check_device_error": (_i, []),
     "agent_attn_stage_aggregate_static": (_i, [_vp, _ll, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                                _f, _i, _vp]),
+    "agent_attn_forward_bias": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
+                                     _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "agent_attn_dwc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "agent_attn_forward_dwc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                     _i, _f, _i, _vp]),
@@ -218,4 +220,18 @@ def agent_attn_forward_dwc(q, k, v, agents_or_null, dwc_w, dwc_bias_or_null, out
                                                _ptr(dwc_w), _ptr(dwc_bias_or_null), _ptr(out), B,
                                                H, N, d, grid_h, grid_w, pool_h, pool_w, scale,
                                                dtype, _stream(stream))
+    return _finish(st, check)
+
+
+def agent_attn_forward_bias(q, k, v, agents_or_null, b1, b2, out, B, H, N, d, grid_h, grid_w,
+                            pool_h, pool_w, scale, dtype, stream=None, check=True):
+    """Forward pass with agent bias.  b1, b2: (row, col, block) triples of fp32
+    device tensors [H, k, grid_h], [H, k, grid_w], [H, k, pool_h*pool_w]
+    (entries may be None), or None for no bias on that softmax."""
+    r1, c1, k1 = b1 if b1 is not None else (None, None, None)
+    r2, c2, k2 = b2 if b2 is not None else (None, None, None)
+    st = load_library().agent_attn_forward_bias(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(agents_or_null), _ptr(r1), _ptr(c1), _ptr(k1), _ptr(r2),
+        _ptr(c2), _ptr(k2), _ptr(out), B, H, N, d, grid_h, grid_w, pool_h, pool_w, scale, dtype,
+        _stream(stream))
     return _finish(st, check)

@@ -106,11 +106,22 @@ int scratch_alloc(void** ptr, size_t bytes, cudaStream_t st) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Components of one agent bias (fp32 device pointers, any may be null):
+// row [H][k][grid_h], col [H][k][grid_w], block [H][k][pool_h*pool_w].
+struct AgentBiasRef {
+  const float* row;
+  const float* col;
+  const float* block;
+  bool any() const { return row || col || block; }
+};
+
 struct Problem {
   int B, H, N, d, k;
   int grid_h, grid_w, pool_h, pool_w;  // pool_h == 0: learnable agents
   float scale;
   int dtype;
+  const AgentBiasRef* b1 = nullptr;    // agent bias of the aggregation (agents x tokens)
+  const AgentBiasRef* b2 = nullptr;    // agent bias of the broadcast (tokens x agents)
   long long BH() const { return (long long)B * H; }
   size_t elem() const { return dtype == AA_FP32 ? 4 : 2; }
 };
@@ -131,7 +142,24 @@ int validate_grid(int N, int grid_h, int grid_w, int pool_h, int pool_w) {
   return AA_OK;
 }
 
-bool use_tensor_cores(const Problem& p) { return p.dtype == AA_BF16 && tc_supported(p.d, p.k); }
+bool has_bias(const Problem& p) { return (p.b1 && p.b1->any()) || (p.b2 && p.b2->any()); }
+// The agent bias runs on the SIMT kernels only (no tensor-core variant yet).
+bool use_tensor_cores(const Problem& p) {
+  return p.dtype == AA_BF16 && tc_supported(p.d, p.k) && !has_bias(p);
+}
+
+void set_bias(SimtAttendArgs& a, const Problem& p, const AgentBiasRef* b, bool tok_is_col) {
+  if (!b || !b->any()) return;
+  a.bias_row = b->row;
+  a.bias_col = b->col;
+  a.bias_block = b->block;
+  a.bias_tok_is_col = tok_is_col ? 1 : 0;
+  a.grid_h = p.grid_h;
+  a.grid_w = p.grid_w;
+  a.pool_h = p.pool_h;
+  a.pool_w = p.pool_w;
+  a.n_agents = p.k;
+}
 
 // Scratch layout.  Every region starts on a 256-byte boundary.
 struct Scratch {
@@ -283,6 +311,7 @@ int run_aggregate(const Problem& p, const Scratch& s, const AgentsRef& ag, const
     a.part_u = reinterpret_cast<float*>(ws + s.pu_off);
     a.part_ml = reinterpret_cast<float*>(ws + s.pml_off);
     a.slots = s.plan.slots;
+    set_bias(a, p, p.b1, true);
     int rc = launch_simt_attend<T>(a, p.BH(), st, pdl);
     if (rc != AA_OK) return rc;
   }
@@ -325,6 +354,7 @@ int run_broadcast(const Problem& p, const void* q, const AgentsRef& ag, const vo
   a.out = out;
   a.out_bstride = qstride_b;
   a.out_hstride = qstride_h;
+  set_bias(a, p, p.b2, false);
   return launch_simt_attend<T>(a, p.BH(), st, pdl);
 }
 
@@ -704,6 +734,31 @@ int agent_attn_forward_dwc(const void* q, const void* k, const void* v, const vo
   if (rc != AA_OK) return rc;
   return dwc_impl(v, dwc_w, dwc_bias_or_null, out, B, H, grid_h, grid_w, d, dtype, 1,
                   static_cast<cudaStream_t>(stream), true);
+}
+
+int agent_attn_forward_bias(const void* q, const void* k, const void* v, const void* agents_or_null,
+                            const float* b1_row, const float* b1_col, const float* b1_block,
+                            const float* b2_row, const float* b2_col, const float* b2_block,
+                            void* out, int B, int H, int N, int d, int grid_h, int grid_w,
+                            int pool_h, int pool_w, float scale, int dtype, void* stream) {
+  int rc = validate_grid(N, grid_h, grid_w, pool_h, pool_w);
+  if (rc != AA_OK) return rc;
+  const int kk = pool_h * pool_w;
+  rc = validate_common(B, H, N, d, kk, scale, dtype);
+  if (rc != AA_OK) return rc;
+  rc = check_tensor_ptrs(q, k, v, out);
+  if (rc != AA_OK) return rc;
+  if (agents_or_null && !aligned16(agents_or_null)) return AA_ERR_ALIGN;
+  const float* parts[6] = {b1_row, b1_col, b1_block, b2_row, b2_col, b2_block};
+  for (const float* b : parts)
+    if (b && (reinterpret_cast<uintptr_t>(b) & 3u)) return AA_ERR_ALIGN;
+  AgentBiasRef bias1{b1_row, b1_col, b1_block}, bias2{b2_row, b2_col, b2_block};
+  Problem p{B, H, N, d, kk, grid_h, grid_w, pool_h, pool_w, scale, dtype};
+  p.b1 = &bias1;
+  p.b2 = &bias2;
+  AgentsRef learn{agents_or_null, 0, (long long)kk * d};
+  return forward_impl(p, q, k, v, agents_or_null ? &learn : nullptr, out, nullptr, 0, false,
+                      static_cast<cudaStream_t>(stream));
 }
 
 int agent_attn_check_device_error(void) {

@@ -148,6 +148,16 @@ struct SimtAttendArgs {
   // normalised output (part_u == nullptr): out[bh][row][c] = U / l
   void* out;
   long long out_bstride, out_hstride;
+  // optional agent bias added to the logits: for agent a and grid token
+  // (y, x), row[h][a][y] + col[h][a][x] + block[h][a][cell(y, x)] (fp32,
+  // each component may be null); cell = floor(y*pool_h/grid_h)*pool_w +
+  // floor(x*pool_w/grid_w).  tok_is_col: columns are tokens (aggregation),
+  // else rows are tokens (broadcast).
+  const float* bias_row;
+  const float* bias_col;
+  const float* bias_block;
+  int bias_tok_is_col;
+  int grid_h, grid_w, pool_h, pool_w, n_agents;
 };
 
 __host__ __forceinline__ size_t simt_attend_smem_bytes(int d) {
@@ -209,13 +219,30 @@ __global__ void __launch_bounds__(kSimtThreads) simt_attend_kernel(SimtAttendArg
       s_vals[e] = ok ? to_f32(vals[(long long)(c0 + j) * d + c]) : 0.f;
     }
     __syncthreads();
+    const bool biased = p.bias_row || p.bias_col || p.bias_block;
     for (int e = tid; e < kSimtRows * kSimtCols; e += kSimtThreads) {
       const int r = e / kSimtCols, j = e % kSimtCols;
       const float* a = s_rows + r * dp;
       const float* b = s_cols + j * dp;
       float acc = 0.f;
       for (int c = 0; c < d; ++c) acc = fmaf(a[c], b[c], acc);
-      s_p[r * (kSimtCols + 1) + j] = acc * p.scale_log2;
+      float logit = acc * p.scale_log2;
+      if (biased && r0 + r < p.n_rows && j < valid) {
+        const int tok = p.bias_tok_is_col ? c0 + j : r0 + r;
+        const int ag = p.bias_tok_is_col ? r0 + r : c0 + j;
+        const int y = tok / p.grid_w, x = tok - y * p.grid_w;
+        const long long base = (long long)(bh % p.H) * p.n_agents + ag;
+        float bias = 0.f;
+        if (p.bias_row) bias += p.bias_row[base * p.grid_h + y];
+        if (p.bias_col) bias += p.bias_col[base * p.grid_w + x];
+        if (p.bias_block) {
+          const int cell = (int)(((long long)y * p.pool_h) / p.grid_h) * p.pool_w +
+                           (int)(((long long)x * p.pool_w) / p.grid_w);
+          bias += p.bias_block[base * ((long long)p.pool_h * p.pool_w) + cell];
+        }
+        logit = fmaf(bias, kLog2e, logit);
+      }
+      s_p[r * (kSimtCols + 1) + j] = logit;
     }
     __syncthreads();
     for (int r = warp; r < kSimtRows; r += kSimtThreads / 32) {

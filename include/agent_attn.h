@@ -171,6 +171,31 @@ AA_API int agent_attn_stage_aggregate_static(const void* agents, long long agent
                                              void* va_lowp, int B, int H, int N, int d,
                                              int n_agents, float scale, int dtype, void* stream);
 
+/* ---- agent bias ----
+ *
+ * Bias terms added to the logits of both softmaxes (arXiv:2312.08874v3
+ * summary, §4 "Module Enhancements": B1 and B2 enter both attention
+ * operations; §6 "Implementation Details": column, row and block components
+ * build the full bias).  Read here, per head h, agent a and grid token
+ * n = y*grid_w + x, as
+ *   bias[h, a, n] = row[h, a, y] + col[h, a, x] + block[h, a, cell(y, x)],
+ *   cell(y, x) = floor(y*pool_h/grid_h)*pool_w + floor(x*pool_w/grid_w)
+ * (the floor partition of the grid into the pool_h x pool_w agent cells).
+ *   aggregation: V_A[a] = softmax_n(scale * A_a . K_n + B1[h, a, n]) V
+ *   broadcast:   O[n]   = softmax_a(scale * Q_n . A_a + B2[h, a, n]) V_A
+ * Components are fp32 device buffers shared over the batch (4-byte aligned):
+ *   *_row [H, k, grid_h], *_col [H, k, grid_w], *_block [H, k, pool_h*pool_w],
+ * k = pool_h*pool_w; each may be NULL (contributes zero).  Other arguments as
+ * in agent_attn_forward.  With any bias present the aggregation and the
+ * broadcast run on the SIMT kernels (fp32 arithmetic, either dtype). */
+AA_API int agent_attn_forward_bias(const void* q, const void* k, const void* v,
+                                   const void* agents_or_null, const float* b1_row,
+                                   const float* b1_col, const float* b1_block,
+                                   const float* b2_row, const float* b2_col,
+                                   const float* b2_block, void* out, int B, int H, int N, int d,
+                                   int grid_h, int grid_w, int pool_h, int pool_w, float scale,
+                                   int dtype, void* stream);
+
 /* ---- the depth-wise convolution term of the full module ----
  *
  * The full Agent Attention module adds a depth-wise convolution term to the

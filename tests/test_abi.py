@@ -150,3 +150,15 @@ def test_dwc_validation():
     assert g(**{**full, "dwc_w": None}) == 1
     assert g(**{**full, "N": 63}) == 2
     assert g(**{**full, "pool_h": 9}) == 2
+
+
+def test_bias_validation():
+    base = dict(q=A16, k=A16, v=A16, agents_or_null=None, b1=(A16, None, None), b2=None, out=A16,
+                B=1, H=1, N=64, d=32, grid_h=8, grid_w=8, pool_h=2, pool_w=2, scale=0.1,
+                dtype=eva.AA_BF16, stream=0, check=False)
+    f = eva.agent_attn_forward_bias
+    assert f(**{**base, "b1": (A16 + 2, None, None)}) == 4
+    assert f(**{**base, "b2": (None, None, A16 + 1)}) == 4
+    assert f(**{**base, "N": 65}) == 2
+    assert f(**{**base, "q": None}) == 1
+    assert f(**{**base, "scale": -1.0}) == 7

@@ -1,0 +1,71 @@
+"""GPU parity of the forward pass with agent bias (row, column and block
+components in both softmaxes) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import efficient_vision_attention_b200 as eva
+import oracle
+from efficient_vision_attention_b200.workloads import random_qkv
+from gpu_helpers import assert_close, dtype_code, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def parts(H, k, gh, gw, seed, scale=0.5, drop=()):
+    g = torch.Generator().manual_seed(seed)
+    out = []
+    for name, n in (("row", gh), ("col", gw), ("block", k)):
+        t = torch.randn((H, k, n), generator=g) * scale
+        out.append(None if name in drop else t)
+    return out
+
+
+def run(q, k, v, gh, gw, ph, pw, scale, b1, b2, dtype):
+    B, H, N, d = q.shape
+    out = torch.empty((B, H, N, d), dtype=dtype, device="cuda")
+    dev = lambda t: None if t is None else t.cuda()
+    eva.agent_attn_forward_bias(q.cuda(), k.cuda(), v.cuda(), None,
+                                None if b1 is None else [dev(t) for t in b1],
+                                None if b2 is None else [dev(t) for t in b2], out, B, H, N, d,
+                                gh, gw, ph, pw, scale, dtype_code(dtype))
+    torch.cuda.synchronize()
+    return out
+
+
+def full(b, gh, gw, ph, pw):
+    if b is None:
+        return None
+    return oracle.agent_bias(*[None if t is None else f64(t) for t in b], gh, gw, ph, pw)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("B,H,gh,gw,ph,pw,d", [(2, 2, 8, 8, 2, 2, 32), (2, 3, 14, 14, 7, 7, 64),
+                                               (1, 2, 32, 32, 8, 8, 40), (1, 2, 13, 11, 4, 3, 16)])
+@pytest.mark.parametrize("drop1,drop2", [((), ()), (("col",), ("row", "block")),
+                                         (("row", "col", "block"), ())])
+def test_bias_matches_oracle(dtype, B, H, gh, gw, ph, pw, d, drop1, drop2):
+    N, k = gh * gw, ph * pw
+    q, kk, v = random_qkv((B, H, N, d), seed=N + d, dtype=dtype)
+    b1 = parts(H, k, gh, gw, 21, drop=drop1)
+    b2 = parts(H, k, gh, gw, 22, drop=drop2)
+    b1 = None if all(t is None for t in b1) else b1
+    scale = 1 / math.sqrt(d)
+    out = run(q, kk, v, gh, gw, ph, pw, scale, b1, b2, dtype)
+    ref = oracle.agent_attn_bias(f64(q), f64(kk), f64(v), gh, gw, ph, pw, scale,
+                                 full(b1, gh, gw, ph, pw), full(b2, gh, gw, ph, pw))
+    assert_close(f64(out), ref, dtype, "biased O")
+
+
+def test_bias_admitting_one_token_selects_its_value_on_gpu():
+    gh, gw, ph, pw, d, ys, xs = 9, 7, 3, 3, 16, 4, 2
+    q, kk, v = random_qkv((1, 2, gh * gw, d), seed=3)
+    row = torch.full((2, 9, gh), -1e4)
+    row[:, :, ys] = 0.0
+    col = torch.full((2, 9, gw), -1e4)
+    col[:, :, xs] = 0.0
+    out = run(q, kk, v, gh, gw, ph, pw, 0.25, [row, col, None], parts(2, 9, gh, gw, 5), torch.float32)
+    want = v[:, :, ys * gw + xs][:, :, None, :].expand_as(out.cpu())
+    assert torch.allclose(out.cpu(), want, atol=1e-6, rtol=0)
