@@ -16,6 +16,7 @@
 #include "agent_attn.h"
 #include "common.cuh"
 #include "kernels_dwc.cuh"
+#include "kernels_pool.cuh"
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
 
@@ -222,8 +223,33 @@ struct AgentsRef {
   long long bstride, hstride;  // elements
 };
 
+std::atomic<int> g_pool_tma_smem_f32[kMaxDevices], g_pool_tma_smem_bf16[kMaxDevices];
+
 template <typename T>
 int launch_pool(const Problem& p, const void* q, float* a_f32, T* a_lowp, cudaStream_t st) {
+  const PoolTmaPlan tp = pool_tma_plan(p.grid_h, p.grid_w, p.pool_h, p.pool_w, p.d, (int)sizeof(T));
+  if (tp.ok) {
+    int rc = ensure_smem(agent_pool_tma_kernel<T>, tp.smem,
+                         sizeof(T) == 4 ? g_pool_tma_smem_f32 : g_pool_tma_smem_bf16);
+    if (rc != AA_OK) return rc;
+    const int n_chunks = (p.pool_w + tp.px_per_cta - 1) / tp.px_per_cta;
+    const long long grid_x = (long long)p.pool_h * n_chunks;
+    if (grid_x > 0x7fffffffLL) return AA_ERR_SHAPE;
+    const int tile_region =
+        (int)((((size_t)tp.rows_max * tp.cols_max * p.d * sizeof(T)) + 127) & ~(size_t)127);
+    for (long long b0 = 0; b0 < p.BH(); b0 += 65535) {   // grid.y limit: slices in chunks
+      const long long nb = (p.BH() - b0 < 65535) ? p.BH() - b0 : 65535;
+      const long long qoff = b0 * (long long)p.N * p.d;
+      const long long aoff = b0 * (long long)p.k * p.d;
+      agent_pool_tma_kernel<T><<<dim3((unsigned)grid_x, (unsigned)nb), kPoolTmaThreads, tp.smem,
+                                 st>>>(
+          static_cast<const T*>(q) + qoff, a_f32 ? a_f32 + aoff : nullptr,
+          a_lowp ? a_lowp + aoff : nullptr, p.N, p.d, p.grid_h, p.grid_w, p.pool_h, p.pool_w,
+          tp.px_per_cta, tp.cols_max, tile_region);
+      AA_CUDA(cudaGetLastError());
+    }
+    return AA_OK;
+  }
   const int per = pool_px_per_cta(p.grid_w, p.pool_w, p.d);
   const int n_chunks = (p.pool_w + per - 1) / per;
   const int groups = p.d / 8;
