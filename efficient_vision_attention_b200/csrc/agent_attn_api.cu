@@ -473,8 +473,8 @@ int dwc_impl(const void* v, const float* w, const float* bias, void* out, int B,
              int grid_h, int grid_w, int d, int dtype, int accumulate, cudaStream_t st, bool pdl) {
   const long long BH = (long long)B * H;
   const long long N = (long long)grid_h * grid_w;
-  const long long items = N * (d / 8);
-  if (items >= (1LL << 31)) return AA_ERR_SHAPE;       // per-slice index math is 32-bit
+  const long long items = (long long)grid_h * ((grid_w + kDwcSpan - 1) / kDwcSpan) * (d / 8);
+  if (N * (d / 8) >= (1LL << 31)) return AA_ERR_SHAPE;   // per-slice index math is 32-bit
   const long long blocks = (items + kDwcThreads - 1) / kDwcThreads;
   const dim3 grid((unsigned)blocks, (unsigned)(BH < 65535 ? BH : 65535));
   const size_t smem = (size_t)10 * d * sizeof(float);

@@ -3,13 +3,14 @@
 // 2312.08874v3 summary, §4 "Module Enhancements": a depth-wise convolution
 // term of cost k^2 N C with k = 3).
 //
-// Each thread owns one (token, 8-channel group) of one (batch, head) slice:
-// it reads the 9 neighbouring 8-channel groups of V (zero outside the grid),
-// applies the head's per-channel 3x3 kernels (staged in shared memory as
-// [tap][channel]), adds the bias and, when accumulating, the value already in
-// `out`, and writes 8 channels.  Consecutive threads cover consecutive
-// channel groups of consecutive tokens, so every tap is a coalesced row read
-// and the 9 taps of a block hit L1/L2 for the rows they share.  HBM-bound:
+// Each thread owns a run of kDwcSpan neighbouring tokens of one grid row and
+// one 8-channel group of a (batch, head) slice: it reads the 3 x (kDwcSpan+2)
+// neighbouring 8-channel groups of V once (zero outside the grid), applies the
+// head's per-channel 3x3 kernels (staged in shared memory as [tap][channel],
+// each weight vector read once for the whole run), adds the bias and, when
+// accumulating, the value already in `out`, and writes the run.  Consecutive
+// threads cover consecutive channel groups of consecutive runs, so every tap
+// row is a coalesced read and blocks share rows through L1/L2.  HBM-bound:
 // V read once, out read (when accumulating) and written once.
 #pragma once
 
@@ -31,31 +32,16 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
   *reinterpret_cast<uint4*>(p) = raw;
 }
 
-// The 9 taps of one (token, 8-channel group): raw 16-byte bf16 rows (zero
-// outside the grid), loaded before anything else so that their trip to
-// memory overlaps the staging of the kernel weights.
-struct DwcTaps {
-  uint4 raw[9];
-};
-__device__ __forceinline__ void dwc_load_taps(const __nv_bfloat16* vs, int y, int x, int grid_h,
-                                              int grid_w, int d, DwcTaps& t) {
-#pragma unroll
-  for (int ty = 0; ty < 3; ++ty) {
-#pragma unroll
-    for (int tx = 0; tx < 3; ++tx) {
-      const int yy = y + ty - 1, xx = x + tx - 1;
-      const bool in = yy >= 0 && yy < grid_h && xx >= 0 && xx < grid_w;
-      t.raw[ty * 3 + tx] =
-          in ? __ldg(reinterpret_cast<const uint4*>(vs + (size_t)((unsigned)yy * grid_w + xx) * d))
-             : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-}
+// Tokens per thread along x: neighbouring outputs share 2 of their 3 tap
+// columns and every weight vector.
+constexpr int kDwcSpan = 2;
 
 // v, out: [BH][grid_h*grid_w][d] of T; w: [H][d][3][3] fp32; bias: [H][d] fp32
-// or null.  Grid: (ceil(N*d/8 / kDwcThreads), min(BH, 65535)), N*d/8 < 2^31.
-// With programmatic dependent launch the V taps are read and convolved before
-// waiting for the previous kernel of the stream (which writes `out`, not V).
+// or null.  Thread = (grid row y, run of kDwcSpan tokens along x, 8-channel
+// group); grid: (ceil(items / kDwcThreads), min(BH, 65535)) with
+// items = grid_h * ceil(grid_w / kDwcSpan) * d/8 < 2^31.  With programmatic
+// dependent launch the convolution is computed before waiting for the
+// previous kernel of the stream (which writes `out`, not V).
 template <typename T>
 __global__ void __launch_bounds__(kDwcThreads)
     dwc_kernel(const T* __restrict__ v, const float* __restrict__ w,
@@ -64,20 +50,17 @@ __global__ void __launch_bounds__(kDwcThreads)
   extern __shared__ float s_w[];   // [9][d] kernel taps, then [d] bias
   pdl_trigger();
   const unsigned nch = (unsigned)d / 8u;
+  const unsigned xruns = ((unsigned)grid_w + kDwcSpan - 1) / kDwcSpan;
   const unsigned N = (unsigned)grid_h * (unsigned)grid_w;
+  const unsigned items = (unsigned)grid_h * xruns * nch;
   const unsigned item = blockIdx.x * blockDim.x + threadIdx.x;
-  const bool mine = item < N * nch;
-  const unsigned n = mine ? item / nch : 0u;
-  const unsigned ch = item - n * nch;
-  const int y = (int)(n / (unsigned)grid_w), x = (int)(n - (unsigned)y * grid_w);
+  const bool mine = item < items;
+  const unsigned ch = mine ? item % nch : 0u;
+  const unsigned run = mine ? item / nch : 0u;
+  const int y = (int)(run / xruns);
+  const int x0 = (int)(run - (unsigned)y * xruns) * kDwcSpan;
   for (long long bh = blockIdx.y; bh < BH; bh += gridDim.y) {
     const int h = (int)(bh % H);
-    const T* vs = v + bh * (long long)N * d + ch * 8;
-    DwcTaps taps;
-    constexpr bool kPreload = false;   // preloading the 9 taps (93 registers) measured slower
-    if constexpr (kPreload) {
-      if (mine) dwc_load_taps(vs, y, x, grid_h, grid_w, d, taps);
-    }
     __syncthreads();   // the previous slice's weights are no longer read
     for (int i = threadIdx.x; i < 9 * d; i += blockDim.x) {
       const int tap = i / d, c = i - tap * d;
@@ -85,35 +68,59 @@ __global__ void __launch_bounds__(kDwcThreads)
     }
     for (int i = threadIdx.x; i < d; i += blockDim.x) s_w[9 * d + i] = bias ? bias[h * d + i] : 0.f;
     __syncthreads();
-    float acc[8];
+    float acc[kDwcSpan][8];
+    const T* vs = v + bh * (long long)N * d + ch * 8;
     if (mine) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = s_w[9 * d + ch * 8 + e];
+      for (int t = 0; t < kDwcSpan; ++t)
 #pragma unroll
-      for (int tap = 0; tap < 9; ++tap) {
-        float t[8];
-        if constexpr (kPreload) {
-          unpack8(taps.raw[tap], reinterpret_cast<const __nv_bfloat16*>(vs), t);
-        } else {
-          const int yy = y + tap / 3 - 1, xx = x + tap % 3 - 1;
-          if (yy < 0 || yy >= grid_h || xx < 0 || xx >= grid_w) continue;
-          load8(vs + (size_t)((unsigned)yy * grid_w + xx) * d, t);
+        for (int e = 0; e < 8; ++e) acc[t][e] = s_w[9 * d + ch * 8 + e];
+#pragma unroll
+      for (int ty = 0; ty < 3; ++ty) {
+        const int yy = y + ty - 1;
+        if (yy < 0 || yy >= grid_h) continue;
+        // the kDwcSpan + 2 tap columns x0-1 .. x0+kDwcSpan of row yy, kept as
+        // raw 16-byte rows and widened at each use (fewer live registers)
+        uint4 raw[kDwcSpan + 2];
+        const T* cp[kDwcSpan + 2];
+        bool cin[kDwcSpan + 2];
+#pragma unroll
+        for (int c = 0; c < kDwcSpan + 2; ++c) {
+          const int xx = x0 + c - 1;
+          cin[c] = xx >= 0 && xx < grid_w;
+          cp[c] = vs + (size_t)((unsigned)yy * grid_w + (cin[c] ? xx : 0)) * d;
+          raw[c] = cin[c] ? load16(cp[c]) : make_uint4(0u, 0u, 0u, 0u);
         }
-        const float* wt = s_w + tap * d + ch * 8;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = fmaf(wt[e], t[e], acc[e]);
+        for (int tx = 0; tx < 3; ++tx) {
+          float wt[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) wt[e] = s_w[(ty * 3 + tx) * d + ch * 8 + e];
+#pragma unroll
+          for (int t = 0; t < kDwcSpan; ++t) {
+            if (!cin[t + tx]) continue;
+            float cv[8];
+            unpack8(raw[t + tx], cp[t + tx], cv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[t][e] = fmaf(wt[e], cv[e], acc[t][e]);
+          }
+        }
       }
     }
     pdl_wait();   // `out` may be written by the previous kernel of the stream
     if (mine) {
-      T* o = out + (bh * (long long)N + n) * d + ch * 8;
-      if (accumulate) {
-        float prev[8];
-        load8(o, prev);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] += prev[e];
+      for (int t = 0; t < kDwcSpan; ++t) {
+        if (x0 + t >= grid_w) continue;
+        T* o = out + (bh * (long long)N + (long long)y * grid_w + x0 + t) * d + ch * 8;
+        if (accumulate) {
+          float prev[8];
+          load8(o, prev);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[t][e] += prev[e];
+        }
+        store8(o, acc[t]);
       }
-      store8(o, acc);
     }
   }
 }
