@@ -53,6 +53,9 @@ def _load():
         lib.oracle_agent_attn.argtypes = [dp, dp, dp, dp, i64, i64, i64, i64, i64, i64, i64, i64,
                                           ctypes.c_double, dp, dp, dp]
         lib.oracle_dwc.argtypes = [dp, dp, dp, i64, i64, i64, i64, i64, dp]
+        lib.oracle_agent_attn_backward.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, i64,
+                                                   i64, i64, i64, ctypes.c_double, dp, dp, dp,
+                                                   dp]
         lib.oracle_agent_attn_bias.argtypes = [dp, dp, dp, dp, dp, dp, i64, i64, i64, i64, i64,
                                                i64, i64, i64, i64, ctypes.c_double, dp, dp, dp]
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -234,3 +237,32 @@ def agent_attn_bias(q, k, v, grid_h: int, grid_w: int, pool_h: int, pool_w: int,
         B * H, H, n, d, grid_h, grid_w, pool_h, pool_w, n_agents, float(scale),
         _ptr(scratch_a), _ptr(scratch_va), _ptr(o))
     return o.reshape(B, H, n, d)
+
+
+def agent_attn_backward(q, k, v, dout, grid_h: int, grid_w: int, pool_h: int, pool_w: int,
+                        scale: float, agents=None):
+    """Gradients (dq, dk, dv, dagents) of the forward pass for the output
+    gradient dout; inputs [B, H, N, d].  agents: None (pooled from Q; dq then
+    includes the pooling adjoint) or [H, k, d] / [B, H, k, d] given agents.
+    dagents is [B, H, k, d] (per slice, before any sum over a shared batch)."""
+    q = _f64(q)
+    B, H, n, d = q.shape
+    k3, v3, do3 = (_f64(t).reshape(B * H, n, d) for t in (k, v, dout))
+    q3 = q.reshape(B * H, n, d)
+    if agents is None:
+        n_agents = pool_h * pool_w
+        a3 = None
+    else:
+        ag = _f64(agents)
+        n_agents = ag.shape[-2]
+        if ag.ndim == 3:
+            ag = np.broadcast_to(ag[None], (B,) + ag.shape)
+        a3 = np.ascontiguousarray(ag.reshape(B * H, n_agents, d))
+    dq, dk, dv = (np.empty((B * H, n, d)) for _ in range(3))
+    da = np.empty((B * H, n_agents, d))
+    _load().oracle_agent_attn_backward(
+        _ptr(q3), _ptr(k3), _ptr(v3), _ptr(a3) if a3 is not None else None, _ptr(do3), B * H, n,
+        d, grid_h, grid_w, pool_h, pool_w, n_agents, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(da))
+    shape = (B, H, n, d)
+    return dq.reshape(shape), dk.reshape(shape), dv.reshape(shape), da.reshape(B, H, n_agents, d)

@@ -243,6 +243,133 @@ void oracle_dwc(const double* v, const double* w, const double* bias_or_null, in
   }
 }
 
+/* Backward pass of the forward pass above (pooled or given agents), for
+ * finetuning.  [arXiv:2312.08874v3 summary, C.4 "AgentSD for finetuning":
+ * agent attention is used during DreamBooth finetuning, i.e. gradients flow
+ * through both softmax stages.]  The pages give no formulas; these are the
+ * derivatives of the definition, written per stage:
+ *   P1 = softmax_rows(s A K^T)  (k x N),  V_A = P1 V
+ *   P2 = softmax_rows(s Q A^T)  (N x k),  O   = P2 V_A
+ * given dO:
+ *   dV_A = P2^T dO;  dP2 = dO V_A^T;  dS2 = P2 .* (dP2 - rowsum(dP2 .* P2))
+ *   dQ  = s dS2 A;   dA  = s dS2^T Q
+ *   dV  = P1^T dV_A; dP1 = dV_A V^T;  dS1 = P1 .* (dP1 - rowsum(dP1 .* P1))
+ *   dK  = s dS1^T A; dA += s dS1 K
+ *   pooled agents: dQ[n] += sum over the bins j holding token n of dA[j] / |bin j|
+ * Outputs dq, dk, dv [BH][N][d]; dagents [BH][n_agents][d] (the gradient of
+ * the agents themselves, before the pooling adjoint; may be NULL). */
+void oracle_agent_attn_backward(const double* q, const double* k, const double* v,
+                                const double* agents_or_null, const double* dout, int64_t BH,
+                                int64_t N, int64_t d, int64_t grid_h, int64_t grid_w,
+                                int64_t pool_h, int64_t pool_w, int64_t n_agents, double scale,
+                                double* dq, double* dk, double* dv, double* dagents) {
+  const int64_t K_ = n_agents;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    const double* Q = q + bh * N * d;
+    const double* Kt = k + bh * N * d;
+    const double* V = v + bh * N * d;
+    const double* dO = dout + bh * N * d;
+    double* A = (double*)malloc(sizeof(double) * (size_t)(K_ * d));
+    double* VA = (double*)calloc((size_t)(K_ * d), sizeof(double));
+    double* P1 = (double*)malloc(sizeof(double) * (size_t)(K_ * N));
+    double* P2 = (double*)malloc(sizeof(double) * (size_t)(N * K_));
+    double* dVA = (double*)calloc((size_t)(K_ * d), sizeof(double));
+    double* dA = (double*)calloc((size_t)(K_ * d), sizeof(double));
+    double* dS = (double*)malloc(sizeof(double) * (size_t)(N > K_ ? N : K_));
+    if (agents_or_null) {
+      for (int64_t i = 0; i < K_ * d; ++i) A[i] = agents_or_null[bh * K_ * d + i];
+    } else {
+      oracle_agent_pool(Q, 1, N, d, grid_h, grid_w, pool_h, pool_w, A);
+    }
+    /* forward: P1, V_A, P2 */
+    for (int64_t j = 0; j < K_; ++j) {
+      double mx = -INFINITY, tot = 0.0;
+      for (int64_t n = 0; n < N; ++n) {
+        double z = 0.0;
+        for (int64_t c = 0; c < d; ++c) z += A[j * d + c] * Kt[n * d + c];
+        P1[j * N + n] = z * scale;
+        if (P1[j * N + n] > mx) mx = P1[j * N + n];
+      }
+      for (int64_t n = 0; n < N; ++n) tot += (P1[j * N + n] = exp(P1[j * N + n] - mx));
+      for (int64_t n = 0; n < N; ++n) {
+        P1[j * N + n] /= tot;
+        for (int64_t c = 0; c < d; ++c) VA[j * d + c] += P1[j * N + n] * V[n * d + c];
+      }
+    }
+    for (int64_t i = 0; i < N; ++i) {
+      double mx = -INFINITY, tot = 0.0;
+      for (int64_t j = 0; j < K_; ++j) {
+        double t = 0.0;
+        for (int64_t c = 0; c < d; ++c) t += Q[i * d + c] * A[j * d + c];
+        P2[i * K_ + j] = t * scale;
+        if (P2[i * K_ + j] > mx) mx = P2[i * K_ + j];
+      }
+      for (int64_t j = 0; j < K_; ++j) tot += (P2[i * K_ + j] = exp(P2[i * K_ + j] - mx));
+      for (int64_t j = 0; j < K_; ++j) P2[i * K_ + j] /= tot;
+    }
+    /* broadcast stage */
+    double* dQs = dq + bh * N * d;
+    for (int64_t i = 0; i < N * d; ++i) dQs[i] = 0.0;
+    for (int64_t i = 0; i < N; ++i) {
+      double dot = 0.0;
+      for (int64_t j = 0; j < K_; ++j) {
+        double dp = 0.0;
+        for (int64_t c = 0; c < d; ++c) dp += dO[i * d + c] * VA[j * d + c];
+        dS[j] = dp;
+        dot += dp * P2[i * K_ + j];
+      }
+      for (int64_t j = 0; j < K_; ++j) {
+        const double p = P2[i * K_ + j];
+        const double ds = p * (dS[j] - dot);
+        for (int64_t c = 0; c < d; ++c) {
+          dVA[j * d + c] += p * dO[i * d + c];
+          dQs[i * d + c] += scale * ds * A[j * d + c];
+          dA[j * d + c] += scale * ds * Q[i * d + c];
+        }
+      }
+    }
+    /* aggregation stage */
+    double* dKs = dk + bh * N * d;
+    double* dVs = dv + bh * N * d;
+    for (int64_t i = 0; i < N * d; ++i) dKs[i] = dVs[i] = 0.0;
+    for (int64_t j = 0; j < K_; ++j) {
+      double dot = 0.0;
+      for (int64_t n = 0; n < N; ++n) {
+        double dp = 0.0;
+        for (int64_t c = 0; c < d; ++c) dp += dVA[j * d + c] * V[n * d + c];
+        dS[n] = dp;
+        dot += dp * P1[j * N + n];
+      }
+      for (int64_t n = 0; n < N; ++n) {
+        const double p = P1[j * N + n];
+        const double ds = p * (dS[n] - dot);
+        for (int64_t c = 0; c < d; ++c) {
+          dVs[n * d + c] += p * dVA[j * d + c];
+          dKs[n * d + c] += scale * ds * A[j * d + c];
+          dA[j * d + c] += scale * ds * Kt[n * d + c];
+        }
+      }
+    }
+    if (dagents)
+      for (int64_t i = 0; i < K_ * d; ++i) dagents[bh * K_ * d + i] = dA[i];
+    /* pooling adjoint: each token of bin j receives dA[j] / |bin j| */
+    if (!agents_or_null) {
+      for (int64_t j = 0; j < K_; ++j) {
+        const int64_t py = j / pool_w, px = j % pool_w;
+        const int64_t y0 = bin_start(py, grid_h, pool_h), y1 = bin_end(py, grid_h, pool_h);
+        const int64_t x0 = bin_start(px, grid_w, pool_w), x1 = bin_end(px, grid_w, pool_w);
+        const double inv = 1.0 / (double)((y1 - y0) * (x1 - x0));
+        for (int64_t y = y0; y < y1; ++y)
+          for (int64_t x = x0; x < x1; ++x)
+            for (int64_t c = 0; c < d; ++c)
+              dQs[(y * grid_w + x) * d + c] += dA[j * d + c] * inv;
+      }
+    }
+    free(A); free(VA); free(P1); free(P2); free(dVA); free(dA); free(dS);
+  }
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

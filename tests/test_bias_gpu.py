@@ -69,3 +69,23 @@ def test_bias_admitting_one_token_selects_its_value_on_gpu():
     out = run(q, kk, v, gh, gw, ph, pw, 0.25, [row, col, None], parts(2, 9, gh, gw, 5), torch.float32)
     want = v[:, :, ys * gw + xs][:, :, None, :].expand_as(out.cpu())
     assert torch.allclose(out.cpu(), want, atol=1e-6, rtol=0)
+
+
+def test_bias_at_the_sd_latent_size_on_sampled_slices():
+    """The SD-latent workload (B=2, H=8, N=16384, d=40, k=256) with all six bias
+    components, checked on two sampled (b, h) slices."""
+    from efficient_vision_attention_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS["sd_latent_1024"]
+    inp = make_inputs(w)
+    q, kk, v = inp["q"], inp["k"], inp["v"]
+    b1 = parts(w.H, w.n_agents, w.grid_h, w.grid_w, 31)
+    b2 = parts(w.H, w.n_agents, w.grid_h, w.grid_w, 32)
+    out = run(q, kk, v, w.grid_h, w.grid_w, w.pool_h, w.pool_w, w.scale, b1, b2, w.torch_dtype)
+    for (b, h) in [(0, 0), (1, 7)]:
+        sl = lambda t: t[b:b + 1, h:h + 1]
+        hb = lambda trip: [t[h:h + 1] for t in trip]
+        ref = oracle.agent_attn_bias(f64(sl(q)), f64(sl(kk)), f64(sl(v)), w.grid_h, w.grid_w,
+                                     w.pool_h, w.pool_w, w.scale,
+                                     full(hb(b1), w.grid_h, w.grid_w, w.pool_h, w.pool_w),
+                                     full(hb(b2), w.grid_h, w.grid_w, w.pool_h, w.pool_w))
+        assert_close(f64(out[b, h]), ref[0, 0], w.torch_dtype, f"biased O slice {(b, h)}")

@@ -384,3 +384,62 @@ def test_bias_that_admits_one_token_selects_its_value():
     got = oracle.agent_attn_bias(q, k, v, gh, gw, ph, pw, 0.5, b1, b2)
     want = np.broadcast_to(v[:, :, ys * gw + xs][:, :, None, :], got.shape)
     np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- backward
+def torch_forward(q, k, v, gh, gw, ph, pw, scale, agents=None):
+    """The forward pass written with torch library ops (float64), for autograd."""
+    B, H, N, d = q.shape
+    if agents is None:
+        t = q.reshape(B * H, gh, gw, d).permute(0, 3, 1, 2)
+        a = F.adaptive_avg_pool2d(t, (ph, pw)).permute(0, 2, 3, 1).reshape(B, H, ph * pw, d)
+    else:
+        a = agents
+    va = torch.softmax(scale * a @ k.transpose(-1, -2), dim=-1) @ v
+    return torch.softmax(scale * q @ a.transpose(-1, -2), dim=-1) @ va
+
+
+@pytest.mark.parametrize("learnable", [False, True])
+def test_backward_matches_autograd_of_library_ops(learnable):
+    B, H, gh, gw, ph, pw, d, scale = 2, 2, 5, 6, 2, 3, 4, 0.6
+    q, k, v, do = (rnd((B, H, gh * gw, d), s) for s in (80, 81, 82, 83))
+    ag = rnd((B, H, ph * pw, d), 84) if learnable else None
+    tq, tk, tv = (torch.from_numpy(x).requires_grad_() for x in (q, k, v))
+    ta = torch.from_numpy(ag).requires_grad_() if learnable else None
+    out = torch_forward(tq, tk, tv, gh, gw, ph, pw, scale, ta)
+    out.backward(torch.from_numpy(do))
+    dq, dk, dv, da = oracle.agent_attn_backward(q, k, v, do, gh, gw, ph, pw, scale, agents=ag)
+    for got, want in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(got, want.numpy(), rtol=1e-10, atol=1e-12)
+    if learnable:
+        np.testing.assert_allclose(da, ta.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_matches_central_differences():
+    """<dO, O(x + eU)> - <dO, O(x - eU)> over 2e equals <grad, U>, for random
+    directions U of q, k and v, with the oracle's own forward pass."""
+    B, H, gh, gw, ph, pw, d, scale = 1, 2, 4, 5, 2, 2, 3, 0.8
+    x = {n: rnd((B, H, gh * gw, d), s) for n, s in (("q", 90), ("k", 91), ("v", 92))}
+    do = rnd((B, H, gh * gw, d), 93)
+    grads = dict(zip("qkv", oracle.agent_attn_backward(x["q"], x["k"], x["v"], do, gh, gw, ph,
+                                                        pw, scale)[:3]))
+    eps = 1e-5
+    for name, s in (("q", 94), ("k", 95), ("v", 96)):
+        u = rnd(x[name].shape, s)
+
+        def loss(sign):
+            y = dict(x)
+            y[name] = x[name] + sign * eps * u
+            return float((do * oracle.agent_attn(y["q"], y["k"], y["v"], gh, gw, ph, pw,
+                                                 scale)).sum())
+        fd = (loss(1) - loss(-1)) / (2 * eps)
+        assert abs(fd - float((grads[name] * u).sum())) < 1e-7 * max(1.0, abs(fd))
+
+
+def test_backward_sums_follow_the_forward_invariances():
+    """O(K + u) = O(K) gives sum_n dK_n = 0; O(V + c) = O(V) + c gives
+    sum_n dV_n = sum_n dO_n."""
+    q, k, v, do = (rnd((2, 3, 24, 5), s) for s in (97, 98, 99, 100))
+    _, dk, dv, _ = oracle.agent_attn_backward(q, k, v, do, 4, 6, 2, 3, 0.5)
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
+    np.testing.assert_allclose(dv.sum(axis=2), do.sum(axis=2), rtol=1e-12, atol=1e-12)
