@@ -391,6 +391,32 @@ def run_native(args, w):
         bias_fwd = {"ms_per_forward": b_ms, "value": B * H * N / (b_ms * 1e-3), "unit": UNIT,
                     "path": "simt"}
 
+    # The backward pass (gradients of Q, K, V for an output gradient) on the
+    # same workload; it runs SIMT kernels with fp32 arithmetic.
+    bwd = None
+    if not w.learnable_agents:
+        dout_ = torch.randn(sets[0]["q"].shape, generator=torch.Generator().manual_seed(5)).to(
+            w.torch_dtype).to(dev)
+        gq_, gk_, gv_ = (torch.empty_like(sets[0]["q"]) for _ in range(3))
+
+        def run_bwd(s):
+            eva.agent_attn_backward(s["q"], s["k"], s["v"], None, dout_, gq_, gk_, gv_, None, B, H,
+                                    N, d, w.grid_h, w.grid_w, w.pool_h, w.pool_w, w.scale, dt,
+                                    stream)
+
+        run_bwd(sets[0])
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for r in range(2):
+            run_bwd(sets[r % n_sets])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        bwd_ms = e0.elapsed_time(e1) / 2
+        bwd = {"ms_per_backward": bwd_ms, "value": B * H * N / (bwd_ms * 1e-3), "unit": UNIT,
+               "path": "simt"}
+
     # End to end through the host-buffer entry point: pinned host inputs copied
     # in, result copied out, every step.
     hin = make_inputs(w, seed=replicas.rank_seed(w.seed, rank))
@@ -444,6 +470,7 @@ def run_native(args, w):
         "roofline": roofline,
         "dwc_term": dwc,
         "agent_bias_forward": bias_fwd,
+        "backward": bwd,
         "cpu_baseline": base,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,

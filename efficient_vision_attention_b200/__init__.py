@@ -13,6 +13,7 @@ from .binding import (  # noqa: F401
     agent_attn_forward_agents,
     agent_attn_forward_bias,
     agent_attn_forward_host,
+    agent_attn_backward,
     agent_attn_check_device_error,
     agent_attn_dwc,
     agent_attn_forward_dwc,

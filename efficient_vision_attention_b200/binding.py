@@ -51,6 +51,8 @@ _SIGNATURES = {
                                                _f, _i, _vp]),
     "agent_attn_forward_bias": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
                                      _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
+    "agent_attn_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                 _i, _i, _i, _f, _i, _vp]),
     "agent_attn_dwc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "agent_attn_forward_dwc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                     _i, _f, _i, _vp]),
@@ -233,5 +235,16 @@ def agent_attn_forward_bias(q, k, v, agents_or_null, b1, b2, out, B, H, N, d, gr
     st = load_library().agent_attn_forward_bias(
         _ptr(q), _ptr(k), _ptr(v), _ptr(agents_or_null), _ptr(r1), _ptr(c1), _ptr(k1), _ptr(r2),
         _ptr(c2), _ptr(k2), _ptr(out), B, H, N, d, grid_h, grid_w, pool_h, pool_w, scale, dtype,
+        _stream(stream))
+    return _finish(st, check)
+
+
+def agent_attn_backward(q, k, v, agents_or_null, dout, dq, dk, dv, dagents_or_null, B, H, N, d,
+                        grid_h, grid_w, pool_h, pool_w, scale, dtype, stream=None, check=True):
+    """Gradients dq, dk, dv (and the agents' own gradient, fp32 [B, H, k, d],
+    when dagents_or_null is given) of the forward pass for dout."""
+    st = load_library().agent_attn_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(agents_or_null), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(dagents_or_null), B, H, N, d, grid_h, grid_w, pool_h, pool_w, scale, dtype,
         _stream(stream))
     return _finish(st, check)

@@ -15,6 +15,7 @@
 
 #include "agent_attn.h"
 #include "common.cuh"
+#include "kernels_bwd.cuh"
 #include "kernels_dwc.cuh"
 #include "kernels_pool.cuh"
 #include "kernels_simt.cuh"
@@ -28,6 +29,9 @@ thread_local char g_cuda_err[384] = "AA_ERR_CUDA: no CUDA error recorded on this
 int cuda_fail(cudaError_t e, const char* what) {
   snprintf(g_cuda_err, sizeof(g_cuda_err), "AA_ERR_CUDA: %s: %s (%s)", what, cudaGetErrorName(e),
            cudaGetErrorString(e));
+  // a launch error is also left as the thread's last error; clear it (it is
+  // reported here) so that the next call's launch checks do not see it again
+  (void)cudaGetLastError();
   return AA_ERR_CUDA;
 }
 #define AA_CUDA(call)                                   \
@@ -123,6 +127,7 @@ struct Problem {
   int dtype;
   const AgentBiasRef* b1 = nullptr;    // agent bias of the aggregation (agents x tokens)
   const AgentBiasRef* b2 = nullptr;    // agent bias of the broadcast (tokens x agents)
+  bool force_simt = false;             // plan the SIMT kernels whatever the dtype
   long long BH() const { return (long long)B * H; }
   size_t elem() const { return dtype == AA_FP32 ? 4 : 2; }
 };
@@ -146,7 +151,7 @@ int validate_grid(int N, int grid_h, int grid_w, int pool_h, int pool_w) {
 bool has_bias(const Problem& p) { return (p.b1 && p.b1->any()) || (p.b2 && p.b2->any()); }
 // The agent bias runs on the SIMT kernels only (no tensor-core variant yet).
 bool use_tensor_cores(const Problem& p) {
-  return p.dtype == AA_BF16 && tc_supported(p.d, p.k) && !has_bias(p);
+  return p.dtype == AA_BF16 && tc_supported(p.d, p.k) && !has_bias(p) && !p.force_simt;
 }
 
 void set_bias(SimtAttendArgs& a, const Problem& p, const AgentBiasRef* b, bool tok_is_col) {
@@ -290,14 +295,14 @@ int launch_simt_attend(const SimtAttendArgs& args, long long BH, cudaStream_t st
 
 template <typename T>
 int launch_merge(const Problem& p, const Scratch& s, char* ws, float* va_f32, T* va_lowp,
-                 cudaStream_t st, bool pdl) {
+                 cudaStream_t st, bool pdl, float* ml_out = nullptr) {
   const long long work = p.BH() * p.k * (p.d / 4);
   const long long blocks = (work + kMergeThreads - 1) / kMergeThreads;
   if (blocks > 0x7fffffffLL) return AA_ERR_SHAPE;
   AA_CUDA(launch_kernel(agent_merge_kernel<T>, dim3((unsigned)blocks), dim3(kMergeThreads), 0, st,
                         pdl, reinterpret_cast<const float*>(ws + s.pu_off),
                         reinterpret_cast<const float*>(ws + s.pml_off), s.plan, p.BH(), p.k, p.d,
-                        va_f32, va_lowp));
+                        va_f32, va_lowp, ml_out));
   return AA_OK;
 }
 
@@ -500,6 +505,144 @@ int validate_dwc(const void* v, const float* w, const void* out, int B, int H, i
   if (!v || !w || !out) return AA_ERR_NULL;
   if (!aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(w) & 3u)) return AA_ERR_ALIGN;
   return AA_OK;
+}
+
+// ------------------------------------------------------------ backward pass
+std::atomic<int> g_bwd_q_f32[kMaxDevices], g_bwd_q_bf16[kMaxDevices];
+std::atomic<int> g_bwd_k_f32[kMaxDevices], g_bwd_k_bf16[kMaxDevices];
+std::atomic<int> g_simt_f32rows_f32[kMaxDevices], g_simt_f32rows_bf16[kMaxDevices];
+
+// Learnable agents [H][k][d] of T (shared over the batch) -> fp32 [BH][k][d].
+template <typename T>
+__global__ void expand_agents_f32_kernel(const T* __restrict__ ag, float* __restrict__ out,
+                                         long long BH, int H, long long kd) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= BH * kd) return;
+  const long long bh = e / kd, r = e - bh * kd;
+  out[e] = to_f32(ag[(bh % H) * kd + r]);
+}
+
+template <typename T>
+int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
+                  const void* agents, const void* dout, void* dq, void* dk, void* dv,
+                  float* dagents, cudaStream_t st) {
+  int sms = 0;
+  int rc = device_sm_count(&sms);
+  if (rc != AA_OK) return rc;
+  Scratch s;
+  plan_scratch(p, sms, &s);            // p.force_simt: SIMT aggregation plan
+  const long long BH = p.BH();
+  const size_t kd = (size_t)p.k * p.d;
+  const size_t nd = (size_t)p.N * p.d;
+  // workspace: plan regions (partials) + fp32 agents, V_A, (max, sum), dV_A, dA, dQ
+  size_t off = s.total;
+  const size_t a32_off = off;   off += round256(BH * kd * 4);
+  const size_t va32_off = off;  off += round256(BH * kd * 4);
+  const size_t ml_off = off;    off += round256(BH * (size_t)p.k * 2 * 4);
+  const size_t dva_off = off;   off += round256(BH * kd * 4);
+  const size_t da_off = off;    off += round256(BH * kd * 4);
+  const size_t dq_off = off;    off += round256(BH * nd * 4);
+  char* ws = nullptr;
+  rc = scratch_alloc(reinterpret_cast<void**>(&ws), off, st);
+  if (rc != AA_OK) return rc;
+  float* a32 = reinterpret_cast<float*>(ws + a32_off);
+  float* va32 = reinterpret_cast<float*>(ws + va32_off);
+  float* ml = reinterpret_cast<float*>(ws + ml_off);
+  float* dva = reinterpret_cast<float*>(ws + dva_off);
+  float* da = reinterpret_cast<float*>(ws + da_off);
+  float* dqa = reinterpret_cast<float*>(ws + dq_off);
+  auto run = [&]() -> int {
+    // 1. fp32 agents
+    if (agents == nullptr) {
+      int r = launch_pool<T>(p, q, a32, nullptr, st);
+      if (r != AA_OK) return r;
+    } else {
+      const long long n = BH * (long long)kd;
+      expand_agents_f32_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+          static_cast<const T*>(agents), a32, BH, p.H, (long long)kd);
+      AA_CUDA(cudaGetLastError());
+    }
+    // 2. forward aggregation with fp32 agent rows: V_A and each row's max and sum
+    SimtAttendArgs a;
+    memset(&a, 0, sizeof(a));
+    const long long qstride_h = (long long)nd, qstride_b = qstride_h * p.H;
+    a.rows = a32;
+    a.rows_bstride = (long long)kd * p.H;
+    a.rows_hstride = (long long)kd;
+    a.cols = k;
+    a.cols_bstride = qstride_b;
+    a.cols_hstride = qstride_h;
+    a.vals = v;
+    a.vals_bstride = qstride_b;
+    a.vals_hstride = qstride_h;
+    a.H = p.H;
+    a.n_rows = p.k;
+    a.n_cols = p.N;
+    a.d = p.d;
+    a.scale_log2 = p.scale * kLog2e;
+    a.row_blocks = s.simt_row_blocks;
+    a.splits = s.plan.fixed;
+    a.cols_per_split = s.simt_cols_per_split;
+    a.part_u = reinterpret_cast<float*>(ws + s.pu_off);
+    a.part_ml = reinterpret_cast<float*>(ws + s.pml_off);
+    a.slots = s.plan.slots;
+    const size_t smem_a = simt_attend_smem_bytes(p.d);
+    int r = ensure_smem(simt_attend_kernel<T, float>, smem_a,
+                        sizeof(T) == 4 ? g_simt_f32rows_f32 : g_simt_f32rows_bf16);
+    if (r != AA_OK) return r;
+    const long long blocks = BH * a.splits * a.row_blocks;
+    if (blocks > 0x7fffffffLL) return AA_ERR_SHAPE;
+    AA_CUDA(launch_kernel(simt_attend_kernel<T, float>, dim3((unsigned)blocks), dim3(kSimtThreads),
+                          smem_a, st, false, a));
+    r = launch_merge<T>(p, s, ws, va32, nullptr, st, false, ml);
+    if (r != AA_OK) return r;
+    // 3. broadcast-stage gradients
+    AA_CUDA(cudaMemsetAsync(dva, 0, BH * kd * 4, st));
+    AA_CUDA(cudaMemsetAsync(da, 0, BH * kd * 4, st));
+    BwdArgs g;
+    memset(&g, 0, sizeof(g));
+    g.x = q;
+    g.y = dout;
+    g.a = a32;
+    g.va = va32;
+    g.dq = dqa;
+    g.dva_acc = dva;
+    g.da_acc = da;
+    g.N = p.N;
+    g.n_agents = p.k;
+    g.d = p.d;
+    g.scale = p.scale;
+    g.scale_log2 = p.scale * kLog2e;
+    const size_t smem_b = bwd_smem_bytes(p.d);
+    const dim3 grid_b((unsigned)((p.N + kBwdRows - 1) / kBwdRows), (unsigned)BH);
+    r = ensure_smem(bwd_query_kernel<T>, smem_b, sizeof(T) == 4 ? g_bwd_q_f32 : g_bwd_q_bf16);
+    if (r != AA_OK) return r;
+    bwd_query_kernel<T><<<grid_b, kBwdThreads, smem_b, st>>>(g);
+    AA_CUDA(cudaGetLastError());
+    // 4. aggregation-stage gradients
+    g.x = k;
+    g.y = v;
+    g.dva = dva;
+    g.ml = ml;
+    g.dk = dk;
+    g.dv = dv;
+    r = ensure_smem(bwd_key_kernel<T>, smem_b, sizeof(T) == 4 ? g_bwd_k_f32 : g_bwd_k_bf16);
+    if (r != AA_OK) return r;
+    bwd_key_kernel<T><<<grid_b, kBwdThreads, smem_b, st>>>(g);
+    AA_CUDA(cudaGetLastError());
+    // 5. dQ (+ pooling adjoint) in the run dtype; the agents' own gradient
+    const dim3 grid_f((unsigned)(((long long)nd + 255) / 256), (unsigned)BH);
+    bwd_finish_kernel<T><<<grid_f, 256, 0, st>>>(dqa, da, static_cast<T*>(dq), p.N, p.d, p.grid_h,
+                                                 p.grid_w, p.pool_h, p.pool_w,
+                                                 agents == nullptr ? 1 : 0);
+    AA_CUDA(cudaGetLastError());
+    if (dagents) AA_CUDA(cudaMemcpyAsync(dagents, da, BH * kd * 4, cudaMemcpyDeviceToDevice, st));
+    return AA_OK;
+  };
+  rc = run();
+  cudaError_t e = cudaFreeAsync(ws, st);
+  if (rc == AA_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
+  return rc;
 }
 
 // Fixed scratch of agent_attn_stage_aggregate_static: a file-scope device
@@ -785,6 +928,32 @@ int agent_attn_forward_bias(const void* q, const void* k, const void* v, const v
   AgentsRef learn{agents_or_null, 0, (long long)kk * d};
   return forward_impl(p, q, k, v, agents_or_null ? &learn : nullptr, out, nullptr, 0, false,
                       static_cast<cudaStream_t>(stream));
+}
+
+int agent_attn_backward(const void* q, const void* k, const void* v, const void* agents_or_null,
+                        const void* dout, void* dq, void* dk, void* dv, float* dagents_or_null,
+                        int B, int H, int N, int d, int grid_h, int grid_w, int pool_h, int pool_w,
+                        float scale, int dtype, void* stream) {
+  int rc = validate_grid(N, grid_h, grid_w, pool_h, pool_w);
+  if (rc != AA_OK) return rc;
+  const int kk = pool_h * pool_w;
+  rc = validate_common(B, H, N, d, kk, scale, dtype);
+  if (rc != AA_OK) return rc;
+  rc = check_tensor_ptrs(q, k, v, dout);
+  if (rc != AA_OK) return rc;
+  if (!dq || !dk || !dv) return AA_ERR_NULL;
+  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return AA_ERR_ALIGN;
+  if (agents_or_null && !aligned16(agents_or_null)) return AA_ERR_ALIGN;
+  if (dagents_or_null && (reinterpret_cast<uintptr_t>(dagents_or_null) & 3u)) return AA_ERR_ALIGN;
+  if ((long long)B * H > 65535) return AA_ERR_SHAPE;
+  Problem p{B, H, N, d, kk, grid_h, grid_w, pool_h, pool_w, scale, dtype};
+  p.force_simt = true;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dtype == AA_FP32
+             ? backward_impl<float>(p, q, k, v, agents_or_null, dout, dq, dk, dv, dagents_or_null,
+                                    st)
+             : backward_impl<__nv_bfloat16>(p, q, k, v, agents_or_null, dout, dq, dk, dv,
+                                            dagents_or_null, st);
 }
 
 int agent_attn_check_device_error(void) {

@@ -1,0 +1,333 @@
+// Backward pass of the Agent Attention forward pass (SIMT, fp32 arithmetic),
+// for finetuning through both softmax stages.  With
+//   P1 = softmax_rows(s A K^T) (k x N), V_A = P1 V,
+//   P2 = softmax_rows(s Q A^T) (N x k), O = P2 V_A
+// and an output gradient dO:
+//   bwd_query_kernel  per query row i: P2_i (two passes over agent chunks for
+//                     its max and sum), dP2_ij = dO_i . V_A_j, D_i = sum_j
+//                     P2_ij dP2_ij, dS2 = P2 (dP2 - D_i); writes dQ_i = s sum_j
+//                     dS2_ij A_j (fp32) and adds the CTA's sums of
+//                     P2_ij dO_i (-> dV_A_j) and s dS2_ij Q_i (-> dA_j) into
+//                     global fp32 accumulators.
+//   bwd_key_kernel    per key row n: P1_jn from the aggregation's stored row
+//                     max and sum, dP1_jn = dV_A_j . V_n, dS1 = P1 (dP1 - E_j)
+//                     with E_j = dV_A_j . V_A_j; writes dK_n = s sum_j dS1_jn
+//                     A_j and dV_n = sum_j P1_jn dV_A_j and adds s dS1_jn K_n
+//                     into dA_j.
+//   bwd_finish_kernel dQ += the pooling adjoint of dA (each token gets dA of
+//                     every bin holding it divided by the bin's size), in the
+//                     output dtype.
+// Scores are in log2 units (scale * log2 e), like the forward kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace aa {
+
+constexpr int kBwdRows = 64;     // query or key rows per CTA
+constexpr int kBwdCols = 32;     // agents per chunk
+constexpr int kBwdThreads = 256;
+
+struct BwdArgs {
+  const void* x;        // q (query kernel) or k (key kernel): [BH][N][d] of T
+  const void* y;        // dO (query kernel) or v (key kernel): [BH][N][d] of T
+  const float* a;       // agents [BH][n_agents][d] fp32
+  const float* va;      // V_A [BH][n_agents][d] fp32
+  const float* dva;     // key kernel: dV_A [BH][n_agents][d]
+  const float* ml;      // key kernel: aggregation row max (log2 units) and sum [BH][n_agents][2]
+  float* dq;            // query kernel: dQ [BH][N][d] fp32
+  float* dva_acc;       // query kernel: += dV_A
+  float* da_acc;        // both: += dA
+  void* dk;             // key kernel: dK [BH][N][d] of T
+  void* dv;             // key kernel: dV [BH][N][d] of T
+  int N, n_agents, d;
+  float scale;          // s
+  float scale_log2;     // s * log2 e
+};
+
+__host__ __forceinline__ size_t bwd_smem_bytes(int d) {
+  const size_t dp = d + 1;
+  return sizeof(float) * (2 * kBwdRows * dp + 2 * kBwdCols * dp + 2 * kBwdRows * (kBwdCols + 1) +
+                          (size_t)kBwdRows * d * 2 + 4 * kBwdRows + 2 * kBwdCols);
+}
+
+template <typename T>
+__device__ __forceinline__ void bwd_load_rows(float* dst, const T* src, int r0, int n_rows, int d,
+                                              int dp) {
+  for (int e = threadIdx.x; e < kBwdRows * d; e += kBwdThreads) {
+    const int r = e / d, c = e - r * d;
+    dst[r * dp + c] = (r0 + r < n_rows) ? to_f32(src[(long long)(r0 + r) * d + c]) : 0.f;
+  }
+}
+
+__device__ __forceinline__ void bwd_load_agents(float* dst, const float* src, int j0, int n_agents,
+                                                int d, int dp) {
+  for (int e = threadIdx.x; e < kBwdCols * d; e += kBwdThreads) {
+    const int j = e / d, c = e - j * d;
+    dst[j * dp + c] = (j0 + j < n_agents) ? src[(long long)(j0 + j) * d + c] : 0.f;
+  }
+}
+
+// dot products of the CTA's rows with a chunk's agents: out[r][j] = X_r . Y_j * mul
+__device__ __forceinline__ void bwd_dots(float* out, const float* X, const float* Y, int d, int dp,
+                                         float mul) {
+  for (int e = threadIdx.x; e < kBwdRows * kBwdCols; e += kBwdThreads) {
+    const int r = e / kBwdCols, j = e - r * kBwdCols;
+    const float* x = X + r * dp;
+    const float* y = Y + j * dp;
+    float acc = 0.f;
+    for (int c = 0; c < d; ++c) acc = fmaf(x[c], y[c], acc);
+    out[r * (kBwdCols + 1) + j] = acc * mul;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
+  extern __shared__ float sm[];
+  const int d = p.d, dp = d + 1;
+  float* s_x = sm;                                   // Q rows [64][d+1]
+  float* s_y = s_x + kBwdRows * dp;                  // dO rows
+  float* s_a = s_y + kBwdRows * dp;                  // agent chunk [32][d+1]
+  float* s_va = s_a + kBwdCols * dp;
+  float* s_t = s_va + kBwdCols * dp;                 // scores / P2 [64][33]
+  float* s_g = s_t + kBwdRows * (kBwdCols + 1);      // dP2 / dS2 [64][33]
+  float* s_acc = s_g + kBwdRows * (kBwdCols + 1);    // dQ accumulator [64][d]
+  float* s_red = s_acc + kBwdRows * d;               // chunk reductions [64][d] (2 x 32 x d)
+  float* s_m = s_red + kBwdRows * d;
+  float* s_l = s_m + kBwdRows;
+  float* s_D = s_l + kBwdRows;
+  const long long bh = blockIdx.y;
+  const int r0 = blockIdx.x * kBwdRows;
+  const int n_rows = p.N, K = p.n_agents;
+  const T* X = static_cast<const T*>(p.x) + bh * (long long)p.N * d;
+  const T* Y = static_cast<const T*>(p.y) + bh * (long long)p.N * d;
+  const float* A = p.a + bh * (long long)K * d;
+  const float* VA = p.va + bh * (long long)K * d;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  bwd_load_rows(s_x, X, r0, n_rows, d, dp);
+  bwd_load_rows(s_y, Y, r0, n_rows, d, dp);
+  for (int e = tid; e < kBwdRows * d; e += kBwdThreads) s_acc[e] = 0.f;
+  for (int r = tid; r < kBwdRows; r += kBwdThreads) {
+    s_m[r] = -INFINITY;
+    s_l[r] = 0.f;
+    s_D[r] = 0.f;
+  }
+  __syncthreads();
+  // pass 1: row max and sum of the scores over all agents (online, per chunk)
+  for (int j0 = 0; j0 < K; j0 += kBwdCols) {
+    const int valid = min(kBwdCols, K - j0);
+    bwd_load_agents(s_a, A, j0, K, d, dp);
+    __syncthreads();
+    bwd_dots(s_t, s_x, s_a, d, dp, p.scale_log2);
+    __syncthreads();
+    for (int r = warp; r < kBwdRows; r += kBwdThreads / 32) {
+      const float t = lane < valid ? s_t[r * (kBwdCols + 1) + lane] : -INFINITY;
+      float mx = t;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float m_new = fmaxf(s_m[r], mx);
+      float e = lane < valid ? exp2f(t - m_new) : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+      if (lane == 0) {
+        s_l[r] = s_l[r] * exp2f(s_m[r] - m_new) + e;
+        s_m[r] = m_new;
+      }
+    }
+    __syncthreads();
+  }
+  // pass 2: D_i = sum_j P2_ij (dO_i . V_A_j)
+  for (int j0 = 0; j0 < K; j0 += kBwdCols) {
+    const int valid = min(kBwdCols, K - j0);
+    bwd_load_agents(s_a, A, j0, K, d, dp);
+    bwd_load_agents(s_va, VA, j0, K, d, dp);
+    __syncthreads();
+    bwd_dots(s_t, s_x, s_a, d, dp, p.scale_log2);
+    bwd_dots(s_g, s_y, s_va, d, dp, 1.f);
+    __syncthreads();
+    for (int r = warp; r < kBwdRows; r += kBwdThreads / 32) {
+      float v = 0.f;
+      if (lane < valid)
+        v = exp2f(s_t[r * (kBwdCols + 1) + lane] - s_m[r]) / s_l[r] * s_g[r * (kBwdCols + 1) + lane];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) s_D[r] += v;
+    }
+    __syncthreads();
+  }
+  // pass 3: dS2, dQ, and the chunk's contributions to dV_A and dA
+  float* dva = p.dva_acc + bh * (long long)K * d;
+  float* da = p.da_acc + bh * (long long)K * d;
+  for (int j0 = 0; j0 < K; j0 += kBwdCols) {
+    const int valid = min(kBwdCols, K - j0);
+    bwd_load_agents(s_a, A, j0, K, d, dp);
+    bwd_load_agents(s_va, VA, j0, K, d, dp);
+    __syncthreads();
+    bwd_dots(s_t, s_x, s_a, d, dp, p.scale_log2);
+    bwd_dots(s_g, s_y, s_va, d, dp, 1.f);
+    __syncthreads();
+    for (int e = tid; e < kBwdRows * kBwdCols; e += kBwdThreads) {
+      const int r = e / kBwdCols, j = e - r * kBwdCols;
+      float pr = 0.f, ds = 0.f;
+      if (j < valid && r0 + r < n_rows) {
+        pr = exp2f(s_t[r * (kBwdCols + 1) + j] - s_m[r]) / s_l[r];
+        ds = pr * (s_g[r * (kBwdCols + 1) + j] - s_D[r]);
+      }
+      s_t[r * (kBwdCols + 1) + j] = pr;
+      s_g[r * (kBwdCols + 1) + j] = ds;
+    }
+    __syncthreads();
+    for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {      // dQ_r += s sum_j ds A_j
+      const int r = e / d, c = e - r * d;
+      float acc = 0.f;
+      for (int j = 0; j < valid; ++j) acc = fmaf(s_g[r * (kBwdCols + 1) + j], s_a[j * dp + c], acc);
+      s_acc[e] += p.scale * acc;
+    }
+    for (int e = tid; e < kBwdCols * d; e += kBwdThreads) {      // per agent: sums over rows
+      const int j = e / d, c = e - j * d;
+      if (j >= valid) continue;
+      float sv = 0.f, sa = 0.f;
+      for (int r = 0; r < kBwdRows; ++r) {
+        sv = fmaf(s_t[r * (kBwdCols + 1) + j], s_y[r * dp + c], sv);
+        sa = fmaf(s_g[r * (kBwdCols + 1) + j], s_x[r * dp + c], sa);
+      }
+      atomicAdd(dva + (long long)(j0 + j) * d + c, sv);
+      atomicAdd(da + (long long)(j0 + j) * d + c, p.scale * sa);
+    }
+    __syncthreads();
+  }
+  float* dq = p.dq + bh * (long long)p.N * d;
+  for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {
+    const int r = e / d, c = e - r * d;
+    if (r0 + r < n_rows) dq[(long long)(r0 + r) * d + c] = s_acc[e];
+  }
+  (void)s_red;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
+  extern __shared__ float sm[];
+  const int d = p.d, dp = d + 1;
+  float* s_x = sm;                                   // K rows
+  float* s_y = s_x + kBwdRows * dp;                  // V rows
+  float* s_a = s_y + kBwdRows * dp;                  // agent chunk
+  float* s_dva = s_a + kBwdCols * dp;                // dV_A chunk
+  float* s_t = s_dva + kBwdCols * dp;                // P1 [64][33]
+  float* s_g = s_t + kBwdRows * (kBwdCols + 1);      // dS1 [64][33]
+  float* s_dk = s_g + kBwdRows * (kBwdCols + 1);     // [64][d]
+  float* s_dv = s_dk + kBwdRows * d;                 // [64][d]
+  float* s_jm = s_dv + kBwdRows * d;                 // chunk: row max, sum, E (3 x 32)
+  float* s_jl = s_jm + kBwdCols;
+  float* s_je = s_jl + kBwdCols;
+  const long long bh = blockIdx.y;
+  const int r0 = blockIdx.x * kBwdRows;
+  const int n_rows = p.N, K = p.n_agents;
+  const T* X = static_cast<const T*>(p.x) + bh * (long long)p.N * d;
+  const T* Y = static_cast<const T*>(p.y) + bh * (long long)p.N * d;
+  const float* A = p.a + bh * (long long)K * d;
+  const float* VA = p.va + bh * (long long)K * d;
+  const float* DVA = p.dva + bh * (long long)K * d;
+  const float* ML = p.ml + bh * (long long)K * 2;
+  float* da = p.da_acc + bh * (long long)K * d;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  bwd_load_rows(s_x, X, r0, n_rows, d, dp);
+  bwd_load_rows(s_y, Y, r0, n_rows, d, dp);
+  for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {
+    s_dk[e] = 0.f;
+    s_dv[e] = 0.f;
+  }
+  for (int j0 = 0; j0 < K; j0 += kBwdCols) {
+    const int valid = min(kBwdCols, K - j0);
+    __syncthreads();
+    bwd_load_agents(s_a, A, j0, K, d, dp);
+    bwd_load_agents(s_dva, DVA, j0, K, d, dp);
+    // E_j = dV_A_j . V_A_j, one warp per agent of the chunk
+    for (int j = warp; j < kBwdCols; j += kBwdThreads / 32) {
+      float e = 0.f;
+      if (j < valid)
+        for (int c = lane; c < d; c += 32)
+          e = fmaf(DVA[(long long)(j0 + j) * d + c], VA[(long long)(j0 + j) * d + c], e);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+      if (lane == 0) {
+        s_je[j] = e;
+        s_jm[j] = j < valid ? ML[(long long)(j0 + j) * 2] : 0.f;
+        s_jl[j] = j < valid ? ML[(long long)(j0 + j) * 2 + 1] : 1.f;
+      }
+    }
+    __syncthreads();
+    bwd_dots(s_t, s_x, s_a, d, dp, p.scale_log2);
+    bwd_dots(s_g, s_y, s_dva, d, dp, 1.f);
+    __syncthreads();
+    for (int e = tid; e < kBwdRows * kBwdCols; e += kBwdThreads) {
+      const int r = e / kBwdCols, j = e - r * kBwdCols;
+      float pr = 0.f, ds = 0.f;
+      if (j < valid && r0 + r < n_rows) {
+        pr = exp2f(s_t[r * (kBwdCols + 1) + j] - s_jm[j]) / s_jl[j];
+        ds = pr * (s_g[r * (kBwdCols + 1) + j] - s_je[j]);
+      }
+      s_t[r * (kBwdCols + 1) + j] = pr;
+      s_g[r * (kBwdCols + 1) + j] = ds;
+    }
+    __syncthreads();
+    for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {
+      const int r = e / d, c = e - r * d;
+      float ak = 0.f, av = 0.f;
+      for (int j = 0; j < valid; ++j) {
+        ak = fmaf(s_g[r * (kBwdCols + 1) + j], s_a[j * dp + c], ak);
+        av = fmaf(s_t[r * (kBwdCols + 1) + j], s_dva[j * dp + c], av);
+      }
+      s_dk[e] += p.scale * ak;
+      s_dv[e] += av;
+    }
+    for (int e = tid; e < kBwdCols * d; e += kBwdThreads) {
+      const int j = e / d, c = e - j * d;
+      if (j >= valid) continue;
+      float sa = 0.f;
+      for (int r = 0; r < kBwdRows; ++r) sa = fmaf(s_g[r * (kBwdCols + 1) + j], s_x[r * dp + c], sa);
+      atomicAdd(da + (long long)(j0 + j) * d + c, p.scale * sa);
+    }
+  }
+  __syncthreads();
+  T* dk = static_cast<T*>(p.dk) + bh * (long long)p.N * d;
+  T* dv = static_cast<T*>(p.dv) + bh * (long long)p.N * d;
+  for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {
+    const int r = e / d, c = e - r * d;
+    if (r0 + r < n_rows) {
+      dk[(long long)(r0 + r) * d + c] = from_f32<T>(s_dk[e]);
+      dv[(long long)(r0 + r) * d + c] = from_f32<T>(s_dv[e]);
+    }
+  }
+}
+
+// dQ = dq_acc (+ the pooling adjoint of dA when the agents were pooled), in T.
+// Thread per (token, channel); grid (ceil(N*d / 256), BH).
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_finish_kernel(const float* __restrict__ dq_acc,
+                                                         const float* __restrict__ da, T* dq,
+                                                         int N, int d, int grid_h, int grid_w,
+                                                         int pool_h, int pool_w, int pooled) {
+  const long long bh = blockIdx.y;
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (long long)N * d) return;
+  const int n = (int)(e / d), c = (int)(e - (long long)n * d);
+  float g = dq_acc[bh * (long long)N * d + e];
+  if (pooled) {
+    const int y = n / grid_w, x = n - y * grid_w;
+    const long long n_agents = (long long)pool_h * pool_w;
+    const float* D = da + bh * n_agents * d;
+    const int cy = (int)(((long long)y * pool_h) / grid_h), cx = (int)(((long long)x * pool_w) / grid_w);
+    for (int py = max(0, cy - 1); py <= min(pool_h - 1, cy + 1); ++py) {
+      const int y0 = bin_start(py, grid_h, pool_h), y1 = bin_end(py, grid_h, pool_h);
+      if (y < y0 || y >= y1) continue;
+      for (int px = max(0, cx - 1); px <= min(pool_w - 1, cx + 1); ++px) {
+        const int x0 = bin_start(px, grid_w, pool_w), x1 = bin_end(px, grid_w, pool_w);
+        if (x < x0 || x >= x1) continue;
+        g += D[((long long)py * pool_w + px) * d + c] / (float)((y1 - y0) * (x1 - x0));
+      }
+    }
+  }
+  dq[bh * (long long)N * d + e] = from_f32<T>(g);
+}
+
+}  // namespace aa

@@ -166,7 +166,9 @@ __host__ __forceinline__ size_t simt_attend_smem_bytes(int d) {
                           (size_t)kSimtRows * d + 3 * kSimtRows);
 }
 
-template <typename T>
+// T: element type of the column vectors, values and output; TR: element type
+// of the row vectors (T, or float for fp32 rows next to bf16 columns).
+template <typename T, typename TR = T>
 __global__ void __launch_bounds__(kSimtThreads) simt_attend_kernel(SimtAttendArgs p) {
   extern __shared__ float smem[];
   const int d = p.d, dp = d + 1;
@@ -189,7 +191,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_attend_kernel(SimtAttendArg
   int c_end = c_begin + p.cols_per_split;
   if (c_end > p.n_cols) c_end = p.n_cols;
 
-  const T* rows = static_cast<const T*>(p.rows) +
+  const TR* rows = static_cast<const TR*>(p.rows) +
                   agent_set_offset(bh, p.H, p.rows_bstride, p.rows_hstride);
   const T* cols = static_cast<const T*>(p.cols) +
                   agent_set_offset(bh, p.H, p.cols_bstride, p.cols_hstride);
@@ -309,7 +311,8 @@ constexpr int kMergeThreads = 256;
 template <typename T>
 __global__ void __launch_bounds__(kMergeThreads) agent_merge_kernel(
     const float* __restrict__ part_u, const float* __restrict__ part_ml, SplitPlan plan,
-    long long BH, int n_agents, int d, float* __restrict__ va_f32, T* __restrict__ va_lowp) {
+    long long BH, int n_agents, int d, float* __restrict__ va_f32, T* __restrict__ va_lowp,
+    float* __restrict__ ml_out = nullptr) {
   const int quads = d >> 2;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   pdl_wait();
@@ -361,6 +364,10 @@ __global__ void __launch_bounds__(kMergeThreads) agent_merge_kernel(
     }
   }
   const float inv = 1.f / den;
+  if (ml_out != nullptr && cq == 0) {     // the row's softmax max (log2 units) and sum
+    ml_out[row * 2] = mx;
+    ml_out[row * 2 + 1] = den;
+  }
   const float v[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
   const long long o = row * d + cq * 4;
   if (va_f32) *reinterpret_cast<float4*>(va_f32 + o) = make_float4(v[0], v[1], v[2], v[3]);

@@ -196,6 +196,33 @@ AA_API int agent_attn_forward_bias(const void* q, const void* k, const void* v,
                                    int grid_h, int grid_w, int pool_h, int pool_w, float scale,
                                    int dtype, void* stream);
 
+/* ---- backward pass ----
+ *
+ * Gradients of agent_attn_forward (pooled agents, agents_or_null == NULL) or
+ * of the forward pass with given agents [H, k, d] (agents_or_null), for
+ * finetuning through both softmax stages (arXiv:2312.08874v3 summary, C.4
+ * "AgentSD for finetuning": agent attention is used during finetuning).  The
+ * pages give no formulas; the gradients are the derivatives of the forward
+ * definition:
+ *   dV_A = P2^T dO, dS2 = P2 .* (dO V_A^T - rowsum(P2 .* dO V_A^T)),
+ *   dQ = s dS2 A (+ the pooling adjoint of dA for pooled agents),
+ *   dS1 = P1 .* (dV_A V^T - rowsum(P1 .* dV_A V^T)), dK = s dS1^T A,
+ *   dV = P1^T dV_A, dA = s dS2^T Q + s dS1 K,
+ * with P1 = softmax_rows(s A K^T), P2 = softmax_rows(s Q A^T).
+ *   dout            : [B, H, N, d] gradient of the output, `dtype`.
+ *   dq, dk, dv      : [B, H, N, d] outputs, `dtype` (16-byte aligned).
+ *   dagents_or_null : [B, H, k, d] fp32 output (gradient of each slice's
+ *                     agents; sum over B for agents shared over the batch),
+ *                     or NULL.
+ * Runs on SIMT kernels with fp32 arithmetic (the forward statistics are
+ * recomputed); the per-agent sums use fp32 atomic additions, so results may
+ * differ from run to run at rounding level.  B*H <= 65535. */
+AA_API int agent_attn_backward(const void* q, const void* k, const void* v,
+                               const void* agents_or_null, const void* dout, void* dq, void* dk,
+                               void* dv, float* dagents_or_null, int B, int H, int N, int d,
+                               int grid_h, int grid_w, int pool_h, int pool_w, float scale,
+                               int dtype, void* stream);
+
 /* ---- the depth-wise convolution term of the full module ----
  *
  * The full Agent Attention module adds a depth-wise convolution term to the

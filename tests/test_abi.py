@@ -162,3 +162,16 @@ def test_bias_validation():
     assert f(**{**base, "N": 65}) == 2
     assert f(**{**base, "q": None}) == 1
     assert f(**{**base, "scale": -1.0}) == 7
+
+
+def test_backward_validation():
+    base = dict(q=A16, k=A16, v=A16, agents_or_null=None, dout=A16, dq=A16, dk=A16, dv=A16,
+                dagents_or_null=None, B=1, H=1, N=64, d=32, grid_h=8, grid_w=8, pool_h=2,
+                pool_w=2, scale=0.1, dtype=eva.AA_BF16, stream=0, check=False)
+    f = eva.agent_attn_backward
+    assert f(**{**base, "dout": None}) == 1
+    assert f(**{**base, "dk": None}) == 1
+    assert f(**{**base, "dv": ODD}) == 4
+    assert f(**{**base, "dagents_or_null": A16 + 2}) == 4
+    assert f(**{**base, "N": 60}) == 2
+    assert f(**{**base, "B": 70000, "H": 1}) == 2
