@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "kernels_bwd.cuh"
 #include "kernels_dwc.cuh"
+#include "kernels_merge.cuh"
 #include "kernels_pool.cuh"
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
@@ -149,9 +150,21 @@ int validate_grid(int N, int grid_h, int grid_w, int pool_h, int pool_w) {
 }
 
 bool has_bias(const Problem& p) { return (p.b1 && p.b1->any()) || (p.b2 && p.b2->any()); }
-// The agent bias runs on the SIMT kernels only (no tensor-core variant yet).
+// The tensor-core kernels take the agent bias while its cell tables fit in
+// shared memory; larger grids run the biased problem on the SIMT kernels.
 bool use_tensor_cores(const Problem& p) {
-  return p.dtype == AA_BF16 && tc_supported(p.d, p.k) && !has_bias(p) && !p.force_simt;
+  if (p.force_simt || p.dtype != AA_BF16 || !tc_supported(p.d, p.k)) return false;
+  return !has_bias(p) || (long long)p.grid_h + p.grid_w <= tc::kBiasGridMax;
+}
+
+tc::BiasParams tc_bias(const Problem& p, const AgentBiasRef* b) {
+  tc::BiasParams r{nullptr, nullptr, nullptr, p.grid_h, p.grid_w, p.pool_h, p.pool_w};
+  if (b) {
+    r.row = b->row;
+    r.col = b->col;
+    r.block = b->block;
+  }
+  return r;
 }
 
 void set_bias(SimtAttendArgs& a, const Problem& p, const AgentBiasRef* b, bool tok_is_col) {
@@ -314,10 +327,11 @@ int run_aggregate(const Problem& p, const Scratch& s, const AgentsRef& ag, const
                   bool pdl = false) {
   const long long qstride_h = (long long)p.N * p.d, qstride_b = qstride_h * p.H;
   if (use_tensor_cores(p)) {
+    const tc::BiasParams b1 = tc_bias(p, p.b1);
     cudaError_t e = tc_launch_aggregate(ag.ptr, ag.bstride, ag.hstride, k, v, p.B, p.H, p.N, p.d,
                                         p.k, p.scale * kLog2e, s.plan,
                                         reinterpret_cast<float*>(ws + s.pu_off),
-                                        reinterpret_cast<float*>(ws + s.pml_off), st, pdl);
+                                        reinterpret_cast<float*>(ws + s.pml_off), st, pdl, &b1);
     if (e != cudaSuccess) return cuda_fail(e, "agent_aggregate (tensor cores) launch");
   } else {
     SimtAttendArgs a;
@@ -358,8 +372,9 @@ int run_broadcast(const Problem& p, const void* q, const AgentsRef& ag, const vo
     int sms = 0;
     int rc = device_sm_count(&sms);
     if (rc != AA_OK) return rc;
+    const tc::BiasParams b2 = tc_bias(p, p.b2);
     cudaError_t e = tc_launch_broadcast(q, ag.ptr, ag.bstride, va, out, p.B, p.H, p.N, p.d, p.k,
-                                        p.scale * kLog2e, sms, st, pdl);
+                                        p.scale * kLog2e, sms, st, pdl, &b2);
     if (e != cudaSuccess) return cuda_fail(e, "agent_broadcast (tensor cores) launch");
     return AA_OK;
   }

@@ -62,6 +62,19 @@ constexpr int kBcStages = 4;
 constexpr int kMaxAgents = 256;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale only when the max grows by > 2^8
 
+// Agent bias in the score tiles: for agent a and grid token (y, x) of head h,
+// row[h][a][y] + col[h][a][x] + block[h][a][cell(y, x)] (fp32 components, any
+// may be null), cell = cell_y[y] * pool_w + cell_x[x] from tables the kernel
+// builds in shared memory (grid_h + grid_w <= kBiasGridMax).
+constexpr int kBiasGridMax = 4096;
+struct BiasParams {
+  const float* row;
+  const float* col;
+  const float* block;
+  int grid_h, grid_w, pool_h, pool_w;
+  __host__ __device__ bool any() const { return row || col || block; }
+};
+
 struct AggParams {
   int H, N, d, k;
   float c;                   // scale * log2(e)
@@ -71,6 +84,7 @@ struct AggParams {
   int slots;                 // partial slots per slice
   float* part_u;             // [BH][slots][k][d]
   float* part_ml;            // [BH][slots][k][2]
+  BiasParams bias;           // B1 (agents x keys), all null when absent
 };
 
 struct BcParams {
@@ -79,6 +93,7 @@ struct BcParams {
   int tiles_per_slice;
   long long total_tiles;
   int ctas;
+  BiasParams bias;           // B2 (queries x agents), all null when absent
 };
 
 struct AggBars {
@@ -124,9 +139,33 @@ __device__ __forceinline__ void drain_commits(uint64_t* bar) {
 }
 
 // ============================================================== aggregation
-constexpr size_t kAggSmemBytes = 1024 + (size_t)kMaxAgents * kRowBytes +
-                                 2 * (size_t)kAggStages * kKTileBytes + sizeof(AggBars);
+// Cell tables of the agent bias: cell_y[grid_h], cell_x[grid_w] as int16.
+__device__ __forceinline__ void build_cell_tables(int16_t* cy, int16_t* cx, const BiasParams& b,
+                                                  int tid, int nthreads) {
+  for (int i = tid; i < b.grid_h; i += nthreads)
+    cy[i] = (int16_t)(((long long)i * b.pool_h) / b.grid_h);
+  for (int i = tid; i < b.grid_w; i += nthreads)
+    cx[i] = (int16_t)(((long long)i * b.pool_w) / b.grid_w);
+}
 
+// Bias of agent a (row offset ra = (h*k + a)) for grid token n.
+__device__ __forceinline__ float agent_bias_at(const BiasParams& b, const int16_t* cy,
+                                               const int16_t* cx, long long ra, int y, int x) {
+  float v = 0.f;
+  if (b.row) v += __ldg(b.row + ra * b.grid_h + y);
+  if (b.col) v += __ldg(b.col + ra * b.grid_w + x);
+  if (b.block)
+    v += __ldg(b.block + ra * ((long long)b.pool_h * b.pool_w) + (int)cy[y] * b.pool_w + cx[x]);
+  return v;
+}
+
+constexpr size_t kAggSmemBytes = 1024 + (size_t)kMaxAgents * kRowBytes +
+                                 2 * (size_t)kAggStages * kKTileBytes + sizeof(AggBars) +
+                                 2 * (size_t)kBiasGridMax;
+
+// kBias: the agent bias B1 is added to the score tiles (a separate
+// instantiation, so the unbiased kernel carries none of its code).
+template <bool kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     agent_aggregate_tc_kernel(const __grid_constant__ CUtensorMap map_k,
                               const __grid_constant__ CUtensorMap map_v,
@@ -138,6 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK = sA + kMaxAgents * kRowBytes;
   uint8_t* sV = sK + kAggStages * kKTileBytes;
   AggBars* bars = reinterpret_cast<AggBars*>(sV + kAggStages * kKTileBytes);
+  int16_t* cell_y = reinterpret_cast<int16_t*>(reinterpret_cast<uint8_t*>(bars) + sizeof(AggBars));
+  int16_t* cell_x = cell_y + p.bias.grid_h;
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -176,6 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
+  constexpr bool biased = kBias;
+  if (biased) build_cell_tables(cell_y, cell_x, p.bias, threadIdx.x, blockDim.x);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -347,10 +390,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v[32];
           slab_ld64(s_col, v);
           if (valid < kKeyTile) slab_mask<8>(v, 0, j4, valid);   // ragged last tile
+          if (biased) {
+            // scores become log2-unit logits: S*c + bias*log2(e), then ce = 1
+            const int n0 = (int)(t + i - bh * tps) * kKeyTile;
+            const int h = (int)(bh % p.H);
+            const long long ra0 = (long long)h * p.k + row_base + r0;
+            const long long ra1 = ra0 + 8;
+            const bool in0 = row_base + r0 < p.k, in1 = row_base + r1 < p.k;
+#pragma unroll
+            for (int g8 = 0; g8 < 8; ++g8) {
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int col = 8 * g8 + 2 * j4 + e;
+                float& va = v[4 * g8 + e];
+                float& vb = v[4 * g8 + 2 + e];
+                if (col < valid) {
+                  const int n = n0 + col;
+                  const int y = n / p.bias.grid_w, x = n - y * p.bias.grid_w;
+                  va = fmaf(va, p.c,
+                            in0 ? agent_bias_at(p.bias, cell_y, cell_x, ra0, y, x) * kLog2e : 0.f);
+                  vb = fmaf(vb, p.c,
+                            in1 ? agent_bias_at(p.bias, cell_y, cell_x, ra1, y, x) * kLog2e : 0.f);
+                }
+              }
+            }
+          }
+          const float ce = biased ? 1.f : p.c;
           float t0 = -INFINITY, t1 = -INFINITY;
           slab_max<8>(v, t0, t1);
-          t0 = row4_max(t0) * p.c;
-          t1 = row4_max(t1) * p.c;
+          t0 = row4_max(t0) * ce;
+          t1 = row4_max(t1) * ce;
           if (first) {
             m0 = t0;
             m1 = t1;
@@ -381,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (ok) {
             uint32_t pk[16];
-            slab_exp<8>(v, p.c, -m0, -m1, pk, l0, l1);
+            slab_exp<8>(v, ce, -m0, -m1, pk, l0, l1);
             slab_st_p32(s_col, pk);
             tmem_wait_st();
           }
@@ -516,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ================================================================ broadcast
 constexpr size_t kBcSmemBytes = 1024 + 2 * (size_t)kMaxAgents * kRowBytes +
                                 (size_t)kBcStages * kQTileBytes + 2 * (size_t)kQTileBytes +
-                                sizeof(BcBars);
+                                sizeof(BcBars) + 2 * (size_t)kBiasGridMax;
 
 // Row maxima of a slab's two rows (this thread's columns) over score columns
 // [0, kpad), columns >= k masked; 64 columns per TMEM load, then 32 and 16.
@@ -543,6 +612,77 @@ __device__ __forceinline__ void bc_slab_max(uint32_t s_col, int k, int kpad, int
     if (c + 16 > k) slab_mask<2>(v, c, j4, k);
     slab_max<2>(v, t0, t1);
   }
+}
+
+// The agent bias of a slab's two query rows: token (y, x) and cell per row.
+struct BcRowBias {
+  int y0, x0, cell0, y1, x1, cell1;
+  bool in0, in1;             // the row is a real token
+  long long hk;              // h * k: agent rows of this head
+};
+
+// Scores of a block (16x256b layout, first column c) become log2-unit logits
+// S*c + B2*log2(e); masked columns stay -inf.
+template <int R>
+__device__ __forceinline__ void bc_bias_block(float (&v)[4 * R], int c, int k, int j4, float cs,
+                                              const BiasParams& b, const BcRowBias& rb) {
+#pragma unroll
+  for (int g = 0; g < R; ++g) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int a = c + 8 * g + 2 * j4 + e;
+      if (a >= k) continue;
+      const long long ra = rb.hk + a;
+      float b0 = 0.f, b1 = 0.f;
+      if (rb.in0) {
+        if (b.row) b0 += __ldg(b.row + ra * b.grid_h + rb.y0);
+        if (b.col) b0 += __ldg(b.col + ra * b.grid_w + rb.x0);
+        if (b.block) b0 += __ldg(b.block + ra * ((long long)b.pool_h * b.pool_w) + rb.cell0);
+      }
+      if (rb.in1) {
+        if (b.row) b1 += __ldg(b.row + ra * b.grid_h + rb.y1);
+        if (b.col) b1 += __ldg(b.col + ra * b.grid_w + rb.x1);
+        if (b.block) b1 += __ldg(b.block + ra * ((long long)b.pool_h * b.pool_w) + rb.cell1);
+      }
+      v[4 * g + e] = fmaf(v[4 * g + e], cs, b0 * kLog2e);
+      v[4 * g + 2 + e] = fmaf(v[4 * g + 2 + e], cs, b1 * kLog2e);
+    }
+  }
+}
+
+// Biased max pass: adds B2 to every score, writes the logits back over the
+// scores (the exponential pass then uses scale 1) and returns the row maxima.
+__device__ __forceinline__ void bc_slab_bias_max(uint32_t s_col, int k, int kpad, int j4,
+                                                 float cs, const BiasParams& b,
+                                                 const BcRowBias& rb, float& t0, float& t1) {
+  int c = 0;
+#pragma unroll 1
+  for (; c + 64 <= kpad; c += 64) {
+    float v[32];
+    slab_ld64(s_col + c, v);
+    if (c + 64 > k) slab_mask<8>(v, c, j4, k);
+    bc_bias_block<8>(v, c, k, j4, cs, b, rb);
+    slab_st64(s_col + c, v);
+    slab_max<8>(v, t0, t1);
+  }
+  if (c + 32 <= kpad) {
+    float v[16];
+    slab_ld32(s_col + c, v);
+    if (c + 32 > k) slab_mask<4>(v, c, j4, k);
+    bc_bias_block<4>(v, c, k, j4, cs, b, rb);
+    slab_st32(s_col + c, v);
+    slab_max<4>(v, t0, t1);
+    c += 32;
+  }
+  if (c < kpad) {
+    float v[8];
+    slab_ld16(s_col + c, v);
+    if (c + 16 > k) slab_mask<2>(v, c, j4, k);
+    bc_bias_block<2>(v, c, k, j4, cs, b, rb);
+    slab_st16(s_col + c, v);
+    slab_max<2>(v, t0, t1);
+  }
+  tmem_wait_st();
 }
 
 // TMEM column (within a 256-column buffer) of the bf16 P of 64-score-column
@@ -604,6 +744,8 @@ __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int
   }
 }
 
+// kBias: the agent bias B2 is added in the max pass (a separate instantiation).
+template <bool kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     agent_broadcast_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                               const __grid_constant__ CUtensorMap map_a,
@@ -617,6 +759,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = sVA + kMaxAgents * kRowBytes;
   uint8_t* sO = sQ + kBcStages * kQTileBytes;
   BcBars* bars = reinterpret_cast<BcBars*>(sO + 2 * kQTileBytes);
+  int16_t* cell_y = reinterpret_cast<int16_t*>(reinterpret_cast<uint8_t*>(bars) + sizeof(BcBars));
+  int16_t* cell_x = cell_y + p.bias.grid_h;
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -657,6 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
+  if (kBias) build_cell_tables(cell_y, cell_x, p.bias, threadIdx.x, blockDim.x);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -799,12 +944,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = warp_wait(&bars->s_full[g], u & 1, abort);
       tc_fence_after();
       float l0 = 0.f, l1 = 0.f, t0 = -INFINITY, t1 = -INFINITY;
+      const float ce = kBias ? 1.f : p.c;     // biased scores are already logits
       if (ok) {
-        bc_slab_max(s_col, p.k, kpad, j4, t0, t1);
-        t0 = row4_max(t0) * p.c;
-        t1 = row4_max(t1) * p.c;
+        if constexpr (kBias) {
+          BcRowBias rb;
+          const int n0 = q0 + r0, n1 = q0 + r1;
+          rb.in0 = n0 < p.N;
+          rb.in1 = n1 < p.N;
+          rb.y0 = rb.in0 ? n0 / p.bias.grid_w : 0;
+          rb.x0 = rb.in0 ? n0 - rb.y0 * p.bias.grid_w : 0;
+          rb.y1 = rb.in1 ? n1 / p.bias.grid_w : 0;
+          rb.x1 = rb.in1 ? n1 - rb.y1 * p.bias.grid_w : 0;
+          rb.cell0 = (int)cell_y[rb.y0] * p.bias.pool_w + cell_x[rb.x0];
+          rb.cell1 = (int)cell_y[rb.y1] * p.bias.pool_w + cell_x[rb.x1];
+          rb.hk = (long long)(bh % p.H) * p.k;
+          bc_slab_bias_max(s_col, p.k, kpad, j4, p.c, p.bias, rb, t0, t1);
+        } else {
+          bc_slab_max(s_col, p.k, kpad, j4, t0, t1);
+        }
+        t0 = row4_max(t0) * ce;
+        t1 = row4_max(t1) * ce;
       }
-      bc_slab_exp(s_col, p.k, kpad, j4, wide, p.c, -t0, -t1, l0, l1, ok, bars->p_chunk[g]);
+      bc_slab_exp(s_col, p.k, kpad, j4, wide, ce, -t0, -t1, l0, l1, ok, bars->p_chunk[g]);
       const float inv0 = 1.f / row4_sum(l0), inv1 = 1.f / row4_sum(l1);
       // epilogue: O = (P V_A) / l -> bf16 -> swizzled staging tile -> TMA store
       if (ok) ok = warp_wait(&bars->o_full[g], u & 1, abort);
@@ -935,6 +1096,14 @@ inline std::atomic<int>* smem_flags_agg() {
   static std::atomic<int> f[64];
   return f;
 }
+inline std::atomic<int>* smem_flags_agg_bias() {
+  static std::atomic<int> f[64];
+  return f;
+}
+inline std::atomic<int>* smem_flags_bc_bias() {
+  static std::atomic<int> f[64];
+  return f;
+}
 inline std::atomic<int>* smem_flags_bc() {
   static std::atomic<int> f[64];
   return f;
@@ -957,7 +1126,7 @@ inline cudaError_t tc_launch_aggregate(const void* agents, long long a_bstride, 
                                        const void* k, const void* v, int B, int H, int N, int d,
                                        int n_agents, float c, const SplitPlan& plan,
                                        float* part_u, float* part_ml, cudaStream_t st,
-                                       bool pdl) {
+                                       bool pdl, const tc::BiasParams* bias = nullptr) {
   (void)a_hstride;
   using namespace tc;
   CUtensorMap mk, mv, ma;
@@ -967,8 +1136,13 @@ inline cudaError_t tc_launch_aggregate(const void* agents, long long a_bstride, 
   if (!make_map_3d(&mk, k, d, N, BH, kKeyTile) || !make_map_3d(&mv, v, d, N, BH, kKeyTile) ||
       !make_map_agents(&ma, agents, d, n_agents, H, B, a_bstride, box_a, &a_sets))
     return cudaErrorInvalidValue;
-  cudaError_t e = ensure_tc_smem(reinterpret_cast<const void*>(agent_aggregate_tc_kernel),
-                                 (int)kAggSmemBytes, smem_flags_agg());
+  const bool biased = bias != nullptr && bias->any();
+  cudaError_t e = biased ? ensure_tc_smem(reinterpret_cast<const void*>(
+                                              agent_aggregate_tc_kernel<true>),
+                                          (int)kAggSmemBytes, smem_flags_agg_bias())
+                         : ensure_tc_smem(reinterpret_cast<const void*>(
+                                              agent_aggregate_tc_kernel<false>),
+                                          (int)kAggSmemBytes, smem_flags_agg());
   if (e != cudaSuccess) return e;
   AggParams p;
   p.H = H;
@@ -982,14 +1156,16 @@ inline cudaError_t tc_launch_aggregate(const void* agents, long long a_bstride, 
   p.slots = plan.slots;
   p.part_u = part_u;
   p.part_ml = part_ml;
-  return launch_kernel(agent_aggregate_tc_kernel, dim3(plan.ctas), dim3(kThreads), kAggSmemBytes,
+  p.bias = bias ? *bias : BiasParams{nullptr, nullptr, nullptr, 1, 1, 1, 1};
+  return launch_kernel(biased ? agent_aggregate_tc_kernel<true> : agent_aggregate_tc_kernel<false>,
+                       dim3(plan.ctas), dim3(kThreads), kAggSmemBytes,
                        st, pdl, mk, mv, ma, a_sets, p);
 }
 
 inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long long a_bstride,
                                        const void* va, void* out, int B, int H, int N, int d,
                                        int n_agents, float c, int sm_count, cudaStream_t st,
-                                       bool pdl) {
+                                       bool pdl, const tc::BiasParams* bias = nullptr) {
   using namespace tc;
   CUtensorMap mq, ma, mva, mo;
   int a_sets = 1;
@@ -999,8 +1175,13 @@ inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long l
       !make_map_3d(&mva, va, d, n_agents, BH, kpad) ||
       !make_map_agents(&ma, agents, d, n_agents, H, B, a_bstride, kpad, &a_sets))
     return cudaErrorInvalidValue;
-  cudaError_t e = ensure_tc_smem(reinterpret_cast<const void*>(agent_broadcast_tc_kernel),
-                                 (int)kBcSmemBytes, smem_flags_bc());
+  const bool biased = bias != nullptr && bias->any();
+  cudaError_t e = biased ? ensure_tc_smem(reinterpret_cast<const void*>(
+                                              agent_broadcast_tc_kernel<true>),
+                                          (int)kBcSmemBytes, smem_flags_bc_bias())
+                         : ensure_tc_smem(reinterpret_cast<const void*>(
+                                              agent_broadcast_tc_kernel<false>),
+                                          (int)kBcSmemBytes, smem_flags_bc());
   if (e != cudaSuccess) return e;
   BcParams p;
   p.H = H;
@@ -1011,8 +1192,10 @@ inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long l
   p.tiles_per_slice = (N + kQTile - 1) / kQTile;
   p.total_tiles = BH * p.tiles_per_slice;
   p.ctas = (int)(p.total_tiles < sm_count ? p.total_tiles : sm_count);
-  return launch_kernel(agent_broadcast_tc_kernel, dim3(p.ctas), dim3(kThreads), kBcSmemBytes, st,
-                       pdl, mq, ma, mva, mo, a_sets, p);
+  p.bias = bias ? *bias : BiasParams{nullptr, nullptr, nullptr, 1, 1, 1, 1};
+  return launch_kernel(biased ? agent_broadcast_tc_kernel<true> : agent_broadcast_tc_kernel<false>,
+                       dim3(p.ctas), dim3(kThreads), kBcSmemBytes, st, pdl, mq, ma, mva, mo,
+                       a_sets, p);
 }
 
 }  // namespace aa
