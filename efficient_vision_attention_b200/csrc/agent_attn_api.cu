@@ -158,7 +158,7 @@ bool use_tensor_cores(const Problem& p) {
 }
 
 tc::BiasParams tc_bias(const Problem& p, const AgentBiasRef* b) {
-  tc::BiasParams r{nullptr, nullptr, nullptr, p.grid_h, p.grid_w, p.pool_h, p.pool_w};
+  tc::BiasParams r{nullptr, nullptr, nullptr, p.grid_h, p.grid_w, p.pool_h, p.pool_w, 0};
   if (b) {
     r.row = b->row;
     r.col = b->col;
@@ -183,6 +183,7 @@ void set_bias(SimtAttendArgs& a, const Problem& p, const AgentBiasRef* b, bool t
 // Scratch layout.  Every region starts on a 256-byte boundary.
 struct Scratch {
   size_t a_off, va_off, pu_off, pml_off, total;
+  size_t b2t_off;            // agent-contiguous copy of B2's components (tensor-core bias)
   SplitPlan plan;
   int simt_row_blocks;
   int simt_cols_per_split;
@@ -219,7 +220,26 @@ void plan_scratch(const Problem& p, int sm_count, Scratch* s) {
   off += round256((size_t)BH * s->plan.slots * p.k * p.d * sizeof(float));
   s->pml_off = off;
   off += round256((size_t)BH * s->plan.slots * p.k * 2 * sizeof(float));
+  s->b2t_off = off;
+  if (use_tensor_cores(p) && p.b2 && p.b2->any()) {
+    const size_t kp = (size_t)((p.k + 15) & ~15);
+    off += round256((size_t)p.H * ((size_t)p.grid_h + p.grid_w + (size_t)p.pool_h * p.pool_w) *
+                    kp * sizeof(float));
+  }
   s->total = off;
+}
+
+// B2's components [H][k][L] -> [H][L][kp] (agents contiguous, kp = k rounded
+// up to 16, zero padding), so a query row of the tensor-core broadcast reads
+// its agents' bias as coalesced float2 runs.  Thread per destination element.
+__global__ void bias_transpose_kernel(const float* __restrict__ src, float* __restrict__ dst,
+                                      int H, int k, int L, int kp) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (long long)H * L * kp) return;
+  const int a = (int)(e % kp);
+  const long long hl = e / kp;
+  const int l = (int)(hl % L), h = (int)(hl / L);
+  dst[e] = a < k ? src[((long long)h * k + a) * L + l] : 0.f;
 }
 
 template <typename KernelT>
@@ -365,14 +385,33 @@ int run_aggregate(const Problem& p, const Scratch& s, const AgentsRef& ag, const
 
 template <typename T>
 int run_broadcast(const Problem& p, const void* q, const AgentsRef& ag, const void* va,
-                  void* out, cudaStream_t st, bool pdl = false) {
+                  void* out, cudaStream_t st, bool pdl = false, float* b2t = nullptr) {
   const long long qstride_h = (long long)p.N * p.d, qstride_b = qstride_h * p.H;
   const long long vstride_h = (long long)p.k * p.d, vstride_b = vstride_h * p.H;
   if (use_tensor_cores(p)) {
     int sms = 0;
     int rc = device_sm_count(&sms);
     if (rc != AA_OK) return rc;
-    const tc::BiasParams b2 = tc_bias(p, p.b2);
+    tc::BiasParams b2 = tc_bias(p, p.b2);
+    if (b2.any()) {
+      if (b2t == nullptr) return AA_ERR_WORKSPACE;
+      const int kp = (p.k + 15) & ~15;
+      const int lens[3] = {p.grid_h, p.grid_w, p.pool_h * p.pool_w};
+      const float* srcs[3] = {b2.row, b2.col, b2.block};
+      float* dst = b2t;
+      const float** outs[3] = {&b2.row, &b2.col, &b2.block};
+      for (int c = 0; c < 3; ++c) {
+        if (srcs[c] == nullptr) continue;
+        const long long n = (long long)p.H * lens[c] * kp;
+        bias_transpose_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(srcs[c], dst, p.H, p.k,
+                                                                         lens[c], kp);
+        AA_CUDA(cudaGetLastError());
+        *outs[c] = dst;
+        dst += n;
+      }
+      b2.agent_minor = kp;
+      pdl = false;    // the broadcast follows the transposes, not the merge
+    }
     cudaError_t e = tc_launch_broadcast(q, ag.ptr, ag.bstride, va, out, p.B, p.H, p.N, p.d, p.k,
                                         p.scale * kLog2e, sms, st, pdl, &b2);
     if (e != cudaSuccess) return cuda_fail(e, "agent_broadcast (tensor cores) launch");
@@ -431,7 +470,8 @@ int run_forward(const Problem& p, const Scratch& s, const void* q, const void* k
                                   st, pdl_agg)
                : run_aggregate<T>(p, s, ag, k, v, ws, nullptr, va_ws, st, pdl_agg);
   if (rc != AA_OK) return rc;
-  return run_broadcast<T>(p, q, ag, va_ws, out, st, true);
+  return run_broadcast<T>(p, q, ag, va_ws, out, st, true,
+                          reinterpret_cast<float*>(ws + s.b2t_off));
 }
 
 int forward_impl(const Problem& p, const void* q, const void* k, const void* v,

@@ -72,6 +72,7 @@ struct BiasParams {
   const float* col;
   const float* block;
   int grid_h, grid_w, pool_h, pool_w;
+  int agent_minor;           // 0: components [H][k][L]; kp > 0: [H][L][kp] (agents contiguous)
   __host__ __device__ bool any() const { return row || col || block; }
 };
 
@@ -622,10 +623,40 @@ struct BcRowBias {
 };
 
 // Scores of a block (16x256b layout, first column c) become log2-unit logits
-// S*c + B2*log2(e); masked columns stay -inf.
+// S*c + B2*log2(e); masked columns stay -inf.  With the agent-contiguous
+// component layout a row's two agents of a column pair come as one float2.
+__device__ __forceinline__ float2 ld_pair(const float* p) {
+  return __ldg(reinterpret_cast<const float2*>(p));
+}
 template <int R>
 __device__ __forceinline__ void bc_bias_block(float (&v)[4 * R], int c, int k, int j4, float cs,
                                               const BiasParams& b, const BcRowBias& rb) {
+  if (b.agent_minor > 0) {
+    const long long kp = b.agent_minor;
+    const long long h = rb.hk / k;
+    const long long nb = (long long)b.pool_h * b.pool_w;
+#pragma unroll
+    for (int g = 0; g < R; ++g) {
+      const int a = c + 8 * g + 2 * j4;       // even; a + 1 < kp (zero padding)
+      float2 b0 = make_float2(0.f, 0.f), b1 = make_float2(0.f, 0.f);
+      if (rb.in0) {
+        if (b.row) { const float2 t = ld_pair(b.row + (h * b.grid_h + rb.y0) * kp + a); b0.x += t.x; b0.y += t.y; }
+        if (b.col) { const float2 t = ld_pair(b.col + (h * b.grid_w + rb.x0) * kp + a); b0.x += t.x; b0.y += t.y; }
+        if (b.block) { const float2 t = ld_pair(b.block + (h * nb + rb.cell0) * kp + a); b0.x += t.x; b0.y += t.y; }
+      }
+      if (rb.in1) {
+        if (b.row) { const float2 t = ld_pair(b.row + (h * b.grid_h + rb.y1) * kp + a); b1.x += t.x; b1.y += t.y; }
+        if (b.col) { const float2 t = ld_pair(b.col + (h * b.grid_w + rb.x1) * kp + a); b1.x += t.x; b1.y += t.y; }
+        if (b.block) { const float2 t = ld_pair(b.block + (h * nb + rb.cell1) * kp + a); b1.x += t.x; b1.y += t.y; }
+      }
+      // columns >= k keep their -inf (their fma stays -inf as cs > 0)
+      v[4 * g] = fmaf(v[4 * g], cs, b0.x * kLog2e);
+      v[4 * g + 1] = fmaf(v[4 * g + 1], cs, b0.y * kLog2e);
+      v[4 * g + 2] = fmaf(v[4 * g + 2], cs, b1.x * kLog2e);
+      v[4 * g + 3] = fmaf(v[4 * g + 3], cs, b1.y * kLog2e);
+    }
+    return;
+  }
 #pragma unroll
   for (int g = 0; g < R; ++g) {
 #pragma unroll
@@ -1156,7 +1187,7 @@ inline cudaError_t tc_launch_aggregate(const void* agents, long long a_bstride, 
   p.slots = plan.slots;
   p.part_u = part_u;
   p.part_ml = part_ml;
-  p.bias = bias ? *bias : BiasParams{nullptr, nullptr, nullptr, 1, 1, 1, 1};
+  p.bias = bias ? *bias : BiasParams{nullptr, nullptr, nullptr, 1, 1, 1, 1, 0};
   return launch_kernel(biased ? agent_aggregate_tc_kernel<true> : agent_aggregate_tc_kernel<false>,
                        dim3(plan.ctas), dim3(kThreads), kAggSmemBytes,
                        st, pdl, mk, mv, ma, a_sets, p);
@@ -1192,7 +1223,7 @@ inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long l
   p.tiles_per_slice = (N + kQTile - 1) / kQTile;
   p.total_tiles = BH * p.tiles_per_slice;
   p.ctas = (int)(p.total_tiles < sm_count ? p.total_tiles : sm_count);
-  p.bias = bias ? *bias : BiasParams{nullptr, nullptr, nullptr, 1, 1, 1, 1};
+  p.bias = bias ? *bias : BiasParams{nullptr, nullptr, nullptr, 1, 1, 1, 1, 0};
   return launch_kernel(biased ? agent_broadcast_tc_kernel<true> : agent_broadcast_tc_kernel<false>,
                        dim3(p.ctas), dim3(kThreads), kBcSmemBytes, st, pdl, mq, ma, mva, mo,
                        a_sets, p);
