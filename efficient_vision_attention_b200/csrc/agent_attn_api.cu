@@ -102,6 +102,31 @@ int device_pool(cudaMemPool_t* out) {
   return AA_OK;
 }
 
+// A library-owned non-blocking stream per device (the second stream of the
+// host-buffer pipeline), created on first use.
+std::atomic<cudaStream_t> g_side_stream[kMaxDevices];
+
+int side_stream(cudaStream_t* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return AA_ERR_UNSUPPORTED;
+  cudaStream_t s = g_side_stream[dev].load(std::memory_order_acquire);
+  if (s != nullptr) {
+    *out = s;
+    return AA_OK;
+  }
+  e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreateWithFlags");
+  cudaStream_t expected = nullptr;
+  if (!g_side_stream[dev].compare_exchange_strong(expected, s)) {
+    cudaStreamDestroy(s);      // another thread won the race
+    s = expected;
+  }
+  *out = s;
+  return AA_OK;
+}
+
 int scratch_alloc(void** ptr, size_t bytes, cudaStream_t st) {
   cudaMemPool_t pool = nullptr;
   int rc = device_pool(&pool);
@@ -784,6 +809,9 @@ int agent_attn_forward_host(const void* q_host, const void* k_host, const void* 
   if (rc != AA_OK) return rc;
   if (!q_host || !k_host || !v_host || !out_host) return AA_ERR_NULL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t st2 = nullptr;
+  rc = side_stream(&st2);
+  if (rc != AA_OK) return rc;
   const size_t eb = dtype == AA_FP32 ? 4 : 2;
   const size_t tbytes = round256((size_t)B * H * N * d * eb);
   const size_t abytes = agents_host_or_null ? round256((size_t)H * kk * d * eb) : 0;
@@ -792,27 +820,59 @@ int agent_attn_forward_host(const void* q_host, const void* k_host, const void* 
   if (rc != AA_OK) return rc;
   char *dq = dev, *dk = dev + tbytes, *dv = dev + 2 * tbytes, *dout = dev + 3 * tbytes;
   char* da = agents_host_or_null ? dev + 4 * tbytes : nullptr;
-  const size_t raw = (size_t)B * H * N * d * eb;
-  cudaError_t e = cudaMemcpyAsync(dq, q_host, raw, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k_host, raw, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v_host, raw, cudaMemcpyHostToDevice, st);
+  // The slices are independent: cut them into chunks (whole batches when the
+  // agents are per head) and pipeline chunk c's upload, forward pass and
+  // download on one of two streams, so uploads overlap the previous chunk's
+  // compute and download (the link is full duplex).
+  const long long units = agents_host_or_null ? B : (long long)B * H;
+  const long long per_unit = agents_host_or_null ? (long long)H : 1;   // slices per unit
+  const long long n_chunks = units < 8 ? units : 8;
+  const size_t slice_bytes = (size_t)N * d * eb;
+  cudaEvent_t ev_alloc = nullptr, ev_done = nullptr;
+  cudaError_t e = cudaEventCreateWithFlags(&ev_alloc, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming);
   if (e == cudaSuccess && da)
     e = cudaMemcpyAsync(da, agents_host_or_null, (size_t)H * kk * d * eb, cudaMemcpyHostToDevice,
                         st);
-  if (e != cudaSuccess) {
-    cudaFreeAsync(dev, st);
-    return cuda_fail(e, "cudaMemcpyAsync(host to device)");
-  }
-  rc = pooled_forward(dq, dk, dv, da, dout, B, H, N, d, grid_h, grid_w, pool_h, pool_w, scale,
-                      dtype, nullptr, 0, false, stream);
-  if (rc == AA_OK) {
-    e = cudaMemcpyAsync(out_host, dout, raw, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaEventRecord(ev_alloc, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st2, ev_alloc, 0);
+  if (e != cudaSuccess) rc = cuda_fail(e, "host pipeline setup");
+  for (long long c = 0; c < n_chunks && rc == AA_OK; ++c) {
+    const long long u0 = c * units / n_chunks, u1 = (c + 1) * units / n_chunks;
+    const size_t off = (size_t)(u0 * per_unit) * slice_bytes;
+    const size_t len = (size_t)((u1 - u0) * per_unit) * slice_bytes;
+    cudaStream_t cs = (c & 1) ? st2 : st;
+    e = cudaMemcpyAsync(dq + off, static_cast<const char*>(q_host) + off, len,
+                        cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(dk + off, static_cast<const char*>(k_host) + off, len,
+                          cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(dv + off, static_cast<const char*>(v_host) + off, len,
+                          cudaMemcpyHostToDevice, cs);
+    if (e != cudaSuccess) {
+      rc = cuda_fail(e, "cudaMemcpyAsync(host to device)");
+      break;
+    }
+    const int cb = agents_host_or_null ? (int)(u1 - u0) : (int)(u1 - u0);
+    const int ch = agents_host_or_null ? H : 1;
+    rc = pooled_forward(dq + off, dk + off, dv + off, da, dout + off, cb, ch, N, d, grid_h,
+                        grid_w, pool_h, pool_w, scale, dtype, nullptr, 0, false, cs);
+    if (rc != AA_OK) break;
+    e = cudaMemcpyAsync(static_cast<char*>(out_host) + off, dout + off, len,
+                        cudaMemcpyDeviceToHost, cs);
     if (e != cudaSuccess) rc = cuda_fail(e, "cudaMemcpyAsync(device to host)");
   }
+  // the side stream's work ends before the buffers go back to the pool
+  cudaError_t e1 = cudaEventRecord(ev_done, st2);
+  if (e1 == cudaSuccess) e1 = cudaStreamWaitEvent(st, ev_done, 0);
+  if (rc == AA_OK && e1 != cudaSuccess) rc = cuda_fail(e1, "host pipeline join");
   cudaError_t e2 = cudaFreeAsync(dev, st);
   if (rc == AA_OK && e2 != cudaSuccess) rc = cuda_fail(e2, "cudaFreeAsync");
   cudaError_t e3 = cudaStreamSynchronize(st);
   if (rc == AA_OK && e3 != cudaSuccess) rc = cuda_fail(e3, "cudaStreamSynchronize");
+  if (ev_alloc) cudaEventDestroy(ev_alloc);
+  if (ev_done) cudaEventDestroy(ev_done);
   return rc;
 }
 

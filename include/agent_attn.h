@@ -110,10 +110,13 @@ AA_API size_t agent_attn_workspace_bytes(int B, int H, int N, int d, int n_agent
 
 /* Synchronous convenience call on HOST buffers: copies q, k, v (and agents,
  * if non-NULL: [H, pool_h*pool_w, d]) to the device, runs the forward pass
- * and copies the result back into out_host, all on `stream`, then
- * synchronizes `stream`.  Device buffers come from the library's
- * stream-ordered pool.  Host buffers should be page-locked for the copies to overlap
- * nothing else but run at full link speed; pageable memory also works. */
+ * and copies the result back into out_host, then synchronizes `stream`.
+ * The slices are cut into up to 8 chunks (whole batches when agents are
+ * given) whose upload, forward pass and download alternate between `stream`
+ * and a second, library-owned stream, so one chunk's upload overlaps the
+ * previous chunk's compute and download.  Device buffers come from the
+ * library's stream-ordered pool.  Host buffers should be page-locked for the
+ * copies to run asynchronously at full link speed; pageable memory also works. */
 AA_API int agent_attn_forward_host(const void* q_host, const void* k_host, const void* v_host,
                             const void* agents_host_or_null, void* out_host, int B, int H, int N,
                             int d, int grid_h, int grid_w, int pool_h, int pool_w, float scale,

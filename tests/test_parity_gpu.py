@@ -246,14 +246,29 @@ def test_workspace_variant_and_determinism():
     assert status == 4
 
 
-def test_host_buffer_entry_point():
-    w = WORKLOADS["deit_tiny_224"]
+@pytest.mark.parametrize("name", ["deit_tiny_224", "sd_latent_1024", "highres_256_learnable256"])
+def test_host_buffer_entry_point(name):
+    """The host-buffer call pipelines chunks of slices over two streams; each
+    chunk is its own forward pass, so the split-over-keys schedule (and with
+    it the rounding order) differs from one call over all slices: compare with
+    the device call at rounding level and with the oracle on sampled slices."""
+    w = WORKLOADS[name]
     inp = make_inputs(w)
     q, k, v = (inp[n].pin_memory() for n in "qkv")
+    ag = inp["agents"].pin_memory() if inp["agents"] is not None else None
     out = torch.empty_like(q).pin_memory()
     B, H, N, d = q.shape
-    eva.agent_attn_forward_host(q, k, v, None, out, B, H, N, d, w.grid_h, w.grid_w, w.pool_h,
+    eva.agent_attn_forward_host(q, k, v, ag, out, B, H, N, d, w.grid_h, w.grid_w, w.pool_h,
                                 w.pool_w, w.scale, eva.AA_BF16)
-    dev = run_forward(inp["q"], inp["k"], inp["v"], w.grid_h, w.grid_w, w.pool_h, w.pool_w,
-                      w.scale)
-    assert torch.equal(out, dev)
+    if ag is None:
+        dev = run_forward(inp["q"], inp["k"], inp["v"], w.grid_h, w.grid_w, w.pool_h, w.pool_w,
+                          w.scale)
+    else:
+        dev = run_forward_agents(inp["q"], inp["k"], inp["v"], inp["agents"], w.scale)
+    assert_close(f64(out), f64(dev), torch.bfloat16, "host vs device", max_abs=4e-3,
+                 rel_l2=2e-3)
+    slices = sample_slices(B, H, 2)
+    ref = oracle_slices(inp["q"], inp["k"], inp["v"], w.grid_h, w.grid_w, w.pool_h, w.pool_w,
+                        w.scale, slices, agents=inp["agents"])
+    got = np.stack([f64(out[b, h]) for (b, h) in slices])
+    assert_close(got, ref, torch.bfloat16, "host vs oracle")
