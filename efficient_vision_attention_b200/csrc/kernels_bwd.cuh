@@ -68,16 +68,31 @@ __device__ __forceinline__ void bwd_load_agents(float* dst, const float* src, in
   }
 }
 
-// dot products of the CTA's rows with a chunk's agents: out[r][j] = X_r . Y_j * mul
+// dot products of the CTA's rows with a chunk's agents: out[r][j] = X_r . Y_j * mul.
+// Register-tiled: thread t owns rows 2(t/8), 2(t/8)+1 and columns 4(t%8) .. +3
+// (256 threads x 8 dots = 64 x 32), reading 6 shared values per 8 FMAs.
 __device__ __forceinline__ void bwd_dots(float* out, const float* X, const float* Y, int d, int dp,
                                          float mul) {
-  for (int e = threadIdx.x; e < kBwdRows * kBwdCols; e += kBwdThreads) {
-    const int r = e / kBwdCols, j = e - r * kBwdCols;
-    const float* x = X + r * dp;
-    const float* y = Y + j * dp;
-    float acc = 0.f;
-    for (int c = 0; c < d; ++c) acc = fmaf(x[c], y[c], acc);
-    out[r * (kBwdCols + 1) + j] = acc * mul;
+  static_assert(kBwdRows * kBwdCols == kBwdThreads * 8, "2 x 4 dots per thread");
+  const int t = threadIdx.x;
+  const int r = 2 * (t >> 3), j = 4 * (t & 7);
+  const float* x0 = X + r * dp;
+  const float* x1 = x0 + dp;
+  const float* y0 = Y + j * dp;
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  for (int c = 0; c < d; ++c) {
+    const float a0 = x0[c], a1 = x1[c];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float bq = y0[q * dp + c];
+      acc[0][q] = fmaf(a0, bq, acc[0][q]);
+      acc[1][q] = fmaf(a1, bq, acc[1][q]);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    out[r * (kBwdCols + 1) + j + q] = acc[0][q] * mul;
+    out[(r + 1) * (kBwdCols + 1) + j + q] = acc[1][q] * mul;
   }
 }
 

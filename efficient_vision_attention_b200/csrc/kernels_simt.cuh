@@ -221,12 +221,27 @@ __global__ void __launch_bounds__(kSimtThreads) simt_attend_kernel(SimtAttendArg
     }
     __syncthreads();
     const bool biased = p.bias_row || p.bias_col || p.bias_block;
-    for (int e = tid; e < kSimtRows * kSimtCols; e += kSimtThreads) {
-      const int r = e / kSimtCols, j = e % kSimtCols;
-      const float* a = s_rows + r * dp;
-      const float* b = s_cols + j * dp;
-      float acc = 0.f;
-      for (int c = 0; c < d; ++c) acc = fmaf(a[c], b[c], acc);
+    // scores, register-tiled: thread t owns rows 2(t/8), +1 and columns 4(t%8) .. +3
+    static_assert(kSimtRows * kSimtCols == kSimtThreads * 8, "2 x 4 scores per thread");
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    {
+      const int rr = 2 * (tid >> 3), jj = 4 * (tid & 7);
+      const float* x0 = s_rows + rr * dp;
+      const float* x1 = x0 + dp;
+      const float* y0 = s_cols + jj * dp;
+      for (int c = 0; c < d; ++c) {
+        const float a0 = x0[c], a1 = x1[c];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float bq = y0[q * dp + c];
+          sc[0][q] = fmaf(a0, bq, sc[0][q]);
+          sc[1][q] = fmaf(a1, bq, sc[1][q]);
+        }
+      }
+    }
+    for (int u = 0; u < 8; ++u) {
+      const int r = 2 * (tid >> 3) + (u >> 2), j = 4 * (tid & 7) + (u & 3);
+      const float acc = sc[u >> 2][u & 3];
       float logit = acc * p.scale_log2;
       if (biased && r0 + r < p.n_rows && j < valid) {
         const int tok = p.bias_tok_is_col ? c0 + j : r0 + r;
