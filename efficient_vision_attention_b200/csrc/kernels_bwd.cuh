@@ -96,6 +96,63 @@ __device__ __forceinline__ void bwd_dots(float* out, const float* X, const float
   }
 }
 
+// out[r][c] += mul * sum_{j < valid} W[r][j] M[j][c] for the CTA's 64 rows:
+// thread items = (row pair, 4 channels), 6 shared reads per 8 FMAs.
+__device__ __forceinline__ void bwd_rows_acc(float* out, const float* W, const float* M, int d,
+                                             int dp, int valid, float mul) {
+  const int nq = (d + 3) >> 2;
+  for (int e = threadIdx.x; e < (kBwdRows / 2) * nq; e += kBwdThreads) {
+    const int rp = e / nq, c = 4 * (e - rp * nq);
+    const int r = 2 * rp;
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < valid; ++j) {
+      const float w0 = W[r * (kBwdCols + 1) + j], w1 = W[(r + 1) * (kBwdCols + 1) + j];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float m = (c + q < d) ? M[j * dp + c + q] : 0.f;
+        a0[q] = fmaf(w0, m, a0[q]);
+        a1[q] = fmaf(w1, m, a1[q]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (c + q < d) {
+        out[r * d + c + q] += mul * a0[q];
+        out[(r + 1) * d + c + q] += mul * a1[q];
+      }
+    }
+  }
+}
+
+// acc[j][c] = mul * sum_r W[r][j] X[r][c] for the chunk's agents j < valid,
+// added atomically into dst[(j0 + j) * d + c]: items = (agent pair, 4 channels).
+__device__ __forceinline__ void bwd_agents_acc(float* dst, int j0, const float* W, const float* X,
+                                               int d, int dp, int valid, float mul) {
+  const int nq = (d + 3) >> 2;
+  for (int e = threadIdx.x; e < (kBwdCols / 2) * nq; e += kBwdThreads) {
+    const int jp = e / nq, c = 4 * (e - jp * nq);
+    const int j = 2 * jp;
+    if (j >= valid) continue;
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int r = 0; r < kBwdRows; ++r) {
+      const float w0 = W[r * (kBwdCols + 1) + j], w1 = W[r * (kBwdCols + 1) + j + 1];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float x = (c + q < d) ? X[r * dp + c + q] : 0.f;
+        a0[q] = fmaf(w0, x, a0[q]);
+        a1[q] = fmaf(w1, x, a1[q]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (c + q < d) {
+        atomicAdd(dst + (long long)(j0 + j) * d + c + q, mul * a0[q]);
+        if (j + 1 < valid) atomicAdd(dst + (long long)(j0 + j + 1) * d + c + q, mul * a1[q]);
+      }
+    }
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
   extern __shared__ float sm[];
@@ -192,23 +249,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
       s_g[r * (kBwdCols + 1) + j] = ds;
     }
     __syncthreads();
-    for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {      // dQ_r += s sum_j ds A_j
-      const int r = e / d, c = e - r * d;
-      float acc = 0.f;
-      for (int j = 0; j < valid; ++j) acc = fmaf(s_g[r * (kBwdCols + 1) + j], s_a[j * dp + c], acc);
-      s_acc[e] += p.scale * acc;
-    }
-    for (int e = tid; e < kBwdCols * d; e += kBwdThreads) {      // per agent: sums over rows
-      const int j = e / d, c = e - j * d;
-      if (j >= valid) continue;
-      float sv = 0.f, sa = 0.f;
-      for (int r = 0; r < kBwdRows; ++r) {
-        sv = fmaf(s_t[r * (kBwdCols + 1) + j], s_y[r * dp + c], sv);
-        sa = fmaf(s_g[r * (kBwdCols + 1) + j], s_x[r * dp + c], sa);
-      }
-      atomicAdd(dva + (long long)(j0 + j) * d + c, sv);
-      atomicAdd(da + (long long)(j0 + j) * d + c, p.scale * sa);
-    }
+    bwd_rows_acc(s_acc, s_g, s_a, d, dp, valid, p.scale);       // dQ_r += s sum_j ds A_j
+    bwd_agents_acc(dva, j0, s_t, s_y, d, dp, valid, 1.f);       // dV_A_j += sum_r P2 dO_r
+    bwd_agents_acc(da, j0, s_g, s_x, d, dp, valid, p.scale);    // dA_j += s sum_r dS2 Q_r
     __syncthreads();
   }
   float* dq = p.dq + bh * (long long)p.N * d;
@@ -285,23 +328,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
       s_g[r * (kBwdCols + 1) + j] = ds;
     }
     __syncthreads();
-    for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {
-      const int r = e / d, c = e - r * d;
-      float ak = 0.f, av = 0.f;
-      for (int j = 0; j < valid; ++j) {
-        ak = fmaf(s_g[r * (kBwdCols + 1) + j], s_a[j * dp + c], ak);
-        av = fmaf(s_t[r * (kBwdCols + 1) + j], s_dva[j * dp + c], av);
-      }
-      s_dk[e] += p.scale * ak;
-      s_dv[e] += av;
-    }
-    for (int e = tid; e < kBwdCols * d; e += kBwdThreads) {
-      const int j = e / d, c = e - j * d;
-      if (j >= valid) continue;
-      float sa = 0.f;
-      for (int r = 0; r < kBwdRows; ++r) sa = fmaf(s_g[r * (kBwdCols + 1) + j], s_x[r * dp + c], sa);
-      atomicAdd(da + (long long)(j0 + j) * d + c, p.scale * sa);
-    }
+    bwd_rows_acc(s_dk, s_g, s_a, d, dp, valid, p.scale);        // dK_r += s sum_j dS1 A_j
+    bwd_rows_acc(s_dv, s_t, s_dva, d, dp, valid, 1.f);          // dV_r += sum_j P1 dV_A_j
+    bwd_agents_acc(da, j0, s_g, s_x, d, dp, valid, p.scale);    // dA_j += s sum_r dS1 K_r
   }
   __syncthreads();
   T* dk = static_cast<T*>(p.dk) + bh * (long long)p.N * d;
