@@ -283,12 +283,37 @@ __global__ void __launch_bounds__(kSimtThreads) simt_attend_kernel(SimtAttendArg
       }
     }
     __syncthreads();
-    for (int e = tid; e < kSimtRows * d; e += kSimtThreads) {
-      const int r = e / d, c = e % d;
-      const float* pr = s_p + r * (kSimtCols + 1);
-      float acc = s_u[e] * s_alpha[r];
-      for (int j = 0; j < valid; ++j) acc = fmaf(pr[j], s_vals[j * d + c], acc);
-      s_u[e] = acc;
+    // U = alpha U + P V, register-tiled: items (row pair, 4 channels)
+    {
+      const int nq = (d + 3) >> 2;
+      for (int e = tid; e < (kSimtRows / 2) * nq; e += kSimtThreads) {
+        const int rp = e / nq, c = 4 * (e - rp * nq);
+        const int r = 2 * rp;
+        const float* p0 = s_p + r * (kSimtCols + 1);
+        const float* p1 = p0 + (kSimtCols + 1);
+        float a0[4], a1[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          a0[q] = (c + q < d) ? s_u[r * d + c + q] * s_alpha[r] : 0.f;
+          a1[q] = (c + q < d) ? s_u[(r + 1) * d + c + q] * s_alpha[r + 1] : 0.f;
+        }
+        for (int j = 0; j < valid; ++j) {
+          const float w0 = p0[j], w1 = p1[j];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float m = (c + q < d) ? s_vals[j * d + c + q] : 0.f;
+            a0[q] = fmaf(w0, m, a0[q]);
+            a1[q] = fmaf(w1, m, a1[q]);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (c + q < d) {
+            s_u[r * d + c + q] = a0[q];
+            s_u[(r + 1) * d + c + q] = a1[q];
+          }
+        }
+      }
     }
     __syncthreads();
   }
