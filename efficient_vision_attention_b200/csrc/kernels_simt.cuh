@@ -5,8 +5,11 @@
 //                         (rows = agents, columns = keys, split over keys,
 //                         partial output) and the broadcast (rows = queries,
 //                         columns = agents, normalised output)
-// These carry the fp32 path end to end (exact enough for a 1e-5 tolerance) and
-// the bf16 path for head dims the tensor-core kernels do not take.
+// These carry the fp32 path end to end (exact enough for a 1e-5 tolerance), the
+// bf16 path for head dims the tensor-core kernels do not take, the agent bias
+// of grids too large for the tensor-core tables, and the forward statistics of
+// the backward pass.  Score blocks and P V updates are register-tiled (2 rows x
+// 4 columns per thread).
 #pragma once
 
 #include "common.cuh"
