@@ -554,9 +554,44 @@ int pooled_forward(const void* q, const void* k, const void* v, const void* agen
 }
 
 // Depth-wise 3x3 term: out (+)= DWConv3x3(v) over the grid, per (head, channel).
+std::atomic<int> g_dwc_stream_f32[kMaxDevices], g_dwc_stream_bf16[kMaxDevices];
+
+template <typename T>
+int dwc_stream_launch(const void* v, const float* w, const float* bias, void* out, int H,
+                      int grid_h, int grid_w, int d, int accumulate, long long BH,
+                      const DwcStreamPlan& pl, int sms, cudaStream_t st, bool pdl) {
+  int rc = ensure_smem(dwc_stream_kernel<T>, pl.smem,
+                       sizeof(T) == 4 ? g_dwc_stream_f32 : g_dwc_stream_bf16);
+  if (rc != AA_OK) return rc;
+  int per_sm = 0;
+  AA_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dwc_stream_kernel<T>,
+                                                        pl.threads, pl.smem));
+  if (per_sm < 1) return AA_ERR_SHAPE;
+  const int band = dwc_stream_band(grid_h, BH * pl.n_xc, (long long)sms * per_sm);
+  const long long grid_x = (long long)((grid_h + band - 1) / band) * pl.n_xc;
+  if (grid_x > 0x7fffffffLL || BH > 65535) return AA_ERR_SHAPE;
+  AA_CUDA(launch_kernel(dwc_stream_kernel<T>, dim3((unsigned)grid_x, (unsigned)BH),
+                        dim3(pl.threads), pl.smem, st, pdl, static_cast<const T*>(v), w, bias,
+                        static_cast<T*>(out), H, grid_h, grid_w, d, pl.cols, band, pl.vslot,
+                        accumulate));
+  return AA_OK;
+}
+
 int dwc_impl(const void* v, const float* w, const float* bias, void* out, int B, int H,
              int grid_h, int grid_w, int d, int dtype, int accumulate, cudaStream_t st, bool pdl) {
   const long long BH = (long long)B * H;
+  if (BH <= 65535) {
+    int sms = 0;
+    int rc = device_sm_count(&sms);
+    if (rc != AA_OK) return rc;
+    const DwcStreamPlan pl = dwc_stream_plan(grid_w, d, dtype == AA_FP32 ? 4 : 2);
+    if (pl.ok)
+      return dtype == AA_FP32
+                 ? dwc_stream_launch<float>(v, w, bias, out, H, grid_h, grid_w, d, accumulate,
+                                            BH, pl, sms, st, pdl)
+                 : dwc_stream_launch<__nv_bfloat16>(v, w, bias, out, H, grid_h, grid_w, d,
+                                                    accumulate, BH, pl, sms, st, pdl);
+  }
   const long long N = (long long)grid_h * grid_w;
   const long long items = (long long)grid_h * ((grid_w + kDwcSpan - 1) / kDwcSpan) * (d / 8);
   if (N * (d / 8) >= (1LL << 31)) return AA_ERR_SHAPE;   // per-slice index math is 32-bit

@@ -24,7 +24,8 @@ def dwc_params(H, d, seed, with_bias=True):
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("B,H,gh,gw,d", [(2, 3, 7, 9, 8), (1, 2, 1, 17, 16), (1, 1, 13, 1, 32),
                                          (2, 2, 56, 56, 32), (1, 8, 128, 128, 40),
-                                         (1, 2, 5, 5, 128), (1, 1, 1, 1, 8)])
+                                         (1, 2, 5, 5, 128), (1, 1, 1, 1, 8),
+                                         (1, 2, 9, 50, 128), (2100, 32, 2, 3, 8)])
 @pytest.mark.parametrize("with_bias,accumulate", [(True, False), (False, True), (True, True)])
 def test_dwc_matches_oracle(dtype, B, H, gh, gw, d, with_bias, accumulate):
     N = gh * gw
