@@ -196,19 +196,6 @@ inline int dwc_stream_band(int grid_h, long long units, long long resident) {
   return band < grid_h ? band : grid_h;
 }
 
-// (a0, a1) += (w0, w1) * (v0, v1) on the paired FP32 datapath (sm_100 f32x2).
-__device__ __forceinline__ void dwc_fma2(float& a0, float& a1, float w0, float w1, float v0,
-                                         float v1) {
-  asm("{\n\t.reg .b64 x, y, z;\n\t"
-      "mov.b64 x, {%0, %1};\n\t"
-      "mov.b64 y, {%2, %3};\n\t"
-      "mov.b64 z, {%4, %5};\n\t"
-      "fma.rn.f32x2 x, y, z, x;\n\t"
-      "mov.b64 {%0, %1}, x;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "f"(w0), "f"(w1), "f"(v0), "f"(v1));
-}
-
 // Raw 8-channel group of one token (16 bytes for bf16, 32 for fp32).
 template <typename T> struct DwcRaw;
 template <> struct DwcRaw<__nv_bfloat16> {
@@ -217,13 +204,11 @@ template <> struct DwcRaw<__nv_bfloat16> {
     a = *reinterpret_cast<const uint4*>(p);
   }
   __device__ __forceinline__ void zero() { a = make_uint4(0u, 0u, 0u, 0u); }
-  __device__ __forceinline__ void widen(float (&f)[8]) const {
+  __device__ __forceinline__ void widen(float2 (&f)[4]) const {
     const uint32_t u[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[2 * i] = __uint_as_float(u[i] << 16);
-      f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
-    }
+    for (int i = 0; i < 4; ++i)
+      f[i] = make_float2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
   }
 };
 template <> struct DwcRaw<float> {
@@ -233,11 +218,11 @@ template <> struct DwcRaw<float> {
     b = *reinterpret_cast<const uint4*>(p + 4);
   }
   __device__ __forceinline__ void zero() { a = b = make_uint4(0u, 0u, 0u, 0u); }
-  __device__ __forceinline__ void widen(float (&f)[8]) const {
-    f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y);
-    f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
-    f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y);
-    f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+  __device__ __forceinline__ void widen(float2 (&f)[4]) const {
+    f[0] = make_float2(__uint_as_float(a.x), __uint_as_float(a.y));
+    f[1] = make_float2(__uint_as_float(a.z), __uint_as_float(a.w));
+    f[2] = make_float2(__uint_as_float(b.x), __uint_as_float(b.y));
+    f[3] = make_float2(__uint_as_float(b.z), __uint_as_float(b.w));
   }
 };
 
@@ -327,26 +312,44 @@ __global__ void __launch_bounds__(kDwcMaxThreads)
   if (mine && accumulate) load_prev(ya);
   __syncthreads();   // barriers initialised, weights staged
 
+  // slot columns x0 .. x0+kDwcTok+1 = grid columns xs+x0-1 .. xs+x0+kDwcTok;
+  // bit c of cmask: column x0+c is inside the grid and staged (else it adds 0)
+  unsigned cmask = 0;
+#pragma unroll
+  for (int c = 0; c < kDwcTok + 2; ++c) {
+    const int j = x0 + c, gx = xs - 1 + j;
+    if (gx >= 0 && gx < grid_w && j <= xw + 1) cmask |= 1u << c;
+  }
+  const T* vcol = vring + (size_t)x0 * d + ch * 8;               // + slot * vslot + c * d
+  const float4* w4 = reinterpret_cast<const float4*>(s_w + ch * 8);  // + tap * d/4
+  const int dq = d >> 2;
+
   bool ok = true;
   int y = ya;
-  for (; y < yb; ++y) {
+  int s0 = 0;   // ring slot of V row y-1 (slots of rows y, y+1 follow cyclically)
+  for (; y < yb; ++y, s0 = (s0 + 1 == kDwcRing) ? 0 : s0 + 1) {
     for (int r = max(y - 1, 0); r <= min(y + 1, grid_h - 1); ++r) ok = ok && wait_row(r);
     // one vote per row: every thread has finished row y-1 (the slot of V
     // row y-2 is free) and sees row y's loads complete
     if (__syncthreads_or(!ok)) break;
     if (threadIdx.x == 0 && y > ya) issue_v(y - 2 + kDwcRing);
     if (!mine) continue;
-    float acc[kDwcTok][8];
+    float2 acc[kDwcTok][4];
     {
-      float b8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) b8[e] = s_w[9 * d + ch * 8 + e];
+      const float4 b0 = w4[9 * dq], b1 = w4[9 * dq + 1];
+      const float2 b2[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w),
+                            make_float2(b1.x, b1.y), make_float2(b1.z, b1.w)};
 #pragma unroll
       for (int t = 0; t < kDwcTok; ++t) {
-        float p8[8];
-        if (accumulate) pre[t].widen(p8);
+        if (accumulate) {
+          float2 p[4];
+          pre[t].widen(p);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[t][e] = accumulate ? b8[e] + p8[e] : b8[e];
+          for (int i = 0; i < 4; ++i) acc[t][i] = __fadd2_rn(b2[i], p[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[t][i] = b2[i];
+        }
       }
     }
     if (accumulate && y + 1 < yb) load_prev(y + 1);   // consumed at the next row
@@ -354,35 +357,41 @@ __global__ void __launch_bounds__(kDwcMaxThreads)
     for (int ty = 0; ty < 3; ++ty) {
       const int r = y + ty - 1;
       if (r < 0 || r >= grid_h) continue;
-      float wv[3][8];
+      float2 wv[3][4];
 #pragma unroll
-      for (int tx = 0; tx < 3; ++tx)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) wv[tx][e] = s_w[(ty * 3 + tx) * d + ch * 8 + e];
-      const T* srow = vring + (size_t)vslot_of(r) * vslot + ch * 8;
-      // slot columns x0 .. x0+kDwcTok+1 = grid columns xs+x0-1 .. xs+x0+kDwcTok;
-      // a column outside the grid, or past the staged halo, reads as zero
+      for (int tx = 0; tx < 3; ++tx) {
+        const float4 a0 = w4[(ty * 3 + tx) * dq], a1 = w4[(ty * 3 + tx) * dq + 1];
+        wv[tx][0] = make_float2(a0.x, a0.y);
+        wv[tx][1] = make_float2(a0.z, a0.w);
+        wv[tx][2] = make_float2(a1.x, a1.y);
+        wv[tx][3] = make_float2(a1.z, a1.w);
+      }
+      int sl = s0 + ty;
+      if (sl >= kDwcRing) sl -= kDwcRing;
+      const T* src = vcol + (size_t)sl * vslot;
 #pragma unroll
       for (int c = 0; c < kDwcTok + 2; ++c) {
-        const int j = x0 + c, gx = xs - 1 + j;
-        if (gx < 0 || gx >= grid_w || j > xw + 1) continue;
+        if (!((cmask >> c) & 1u)) continue;
         DwcRaw<T> raw;
-        raw.load(srow + (size_t)j * d);
-        float cv[8];
+        raw.load(src + c * d);
+        float2 cv[4];
         raw.widen(cv);
 #pragma unroll
         for (int tx = 0; tx < 3; ++tx) {
           const int t = c - tx;
           if (t < 0 || t >= kDwcTok) continue;
 #pragma unroll
-          for (int e = 0; e < 8; e += 2)
-            dwc_fma2(acc[t][e], acc[t][e + 1], wv[tx][e], wv[tx][e + 1], cv[e], cv[e + 1]);
+          for (int i = 0; i < 4; ++i) acc[t][i] = __ffma2_rn(wv[tx][i], cv[i], acc[t][i]);
         }
       }
     }
 #pragma unroll
-    for (int t = 0; t < kDwcTok; ++t)
-      if (x0 + t < xw) store8(orow + ((long long)y * grid_w + t) * d, acc[t]);
+    for (int t = 0; t < kDwcTok; ++t) {
+      if (x0 + t >= xw) continue;
+      const float o8[8] = {acc[t][0].x, acc[t][0].y, acc[t][1].x, acc[t][1].y,
+                           acc[t][2].x, acc[t][2].y, acc[t][3].x, acc[t][3].y};
+      store8(orow + ((long long)y * grid_w + t) * d, o8);
+    }
   }
   if (y < yb && threadIdx.x == 0) {
     // a load outlived the limit: wait (bounded) for every copy still in
