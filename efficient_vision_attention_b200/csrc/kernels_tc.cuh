@@ -149,14 +149,49 @@ __device__ __forceinline__ void build_cell_tables(int16_t* cy, int16_t* cx, cons
     cx[i] = (int16_t)(((long long)i * b.pool_w) / b.grid_w);
 }
 
-// Bias of agent a (row offset ra = (h*k + a)) for grid token n.
-__device__ __forceinline__ float agent_bias_at(const BiasParams& b, const int16_t* cy,
-                                               const int16_t* cx, long long ra, int y, int x) {
+// Per-agent-row bases of the three components (null where a component is absent).
+struct BiasRowPtrs {
+  const float* row;
+  const float* col;
+  const float* block;
+};
+__device__ __forceinline__ BiasRowPtrs bias_row_ptrs(const BiasParams& b, long long ra) {
+  BiasRowPtrs r;
+  r.row = b.row ? b.row + ra * b.grid_h : nullptr;
+  r.col = b.col ? b.col + ra * b.grid_w : nullptr;
+  r.block = b.block ? b.block + ra * ((long long)b.pool_h * b.pool_w) : nullptr;
+  return r;
+}
+// Bias of one agent row for the token pair (y, x), (y, x+1) of one grid row:
+// one row term, the two column terms as one float2 (8-byte aligned), two cells.
+__device__ __forceinline__ float2 agent_bias_pair(const BiasRowPtrs& r, const BiasParams& b,
+                                                  const int16_t* cy, const int16_t* cx, int y,
+                                                  int x) {
+  float2 v = make_float2(0.f, 0.f);
+  if (r.row) {
+    const float t = __ldg(r.row + y);
+    v.x = t;
+    v.y = t;
+  }
+  if (r.col) {
+    const float2 t = __ldg(reinterpret_cast<const float2*>(r.col + x));
+    v.x += t.x;
+    v.y += t.y;
+  }
+  if (r.block) {
+    const float* br = r.block + (int)cy[y] * b.pool_w;
+    v.x += __ldg(br + cx[x]);
+    v.y += __ldg(br + cx[x + 1]);
+  }
+  return v;
+}
+__device__ __forceinline__ float agent_bias_one(const BiasRowPtrs& r, const BiasParams& b,
+                                                const int16_t* cy, const int16_t* cx, int y,
+                                                int x) {
   float v = 0.f;
-  if (b.row) v += __ldg(b.row + ra * b.grid_h + y);
-  if (b.col) v += __ldg(b.col + ra * b.grid_w + x);
-  if (b.block)
-    v += __ldg(b.block + ra * ((long long)b.pool_h * b.pool_w) + (int)cy[y] * b.pool_w + cx[x]);
+  if (r.row) v += __ldg(r.row + y);
+  if (r.col) v += __ldg(r.col + x);
+  if (r.block) v += __ldg(r.block + (int)cy[y] * b.pool_w + cx[x]);
   return v;
 }
 
@@ -392,26 +427,55 @@ __global__ void __launch_bounds__(kThreads, 1)
           slab_ld64(s_col, v);
           if (valid < kKeyTile) slab_mask<8>(v, 0, j4, valid);   // ragged last tile
           if (biased) {
-            // scores become log2-unit logits: S*c + bias*log2(e), then ce = 1
+            // scores become log2-unit logits: S*c + bias*log2(e), then ce = 1.
+            // The tile's first key is split into (y, x) once.  A thread's
+            // columns come in pairs (x, x+1); on an even-width grid a pair
+            // starts at an even x, so it never straddles two grid rows and
+            // shares the row term and the cell row (the column terms as one
+            // float2 when the column component is 8-byte aligned).
             const int n0 = (int)(t + i - bh * tps) * kKeyTile;
             const int h = (int)(bh % p.H);
             const long long ra0 = (long long)h * p.k + row_base + r0;
-            const long long ra1 = ra0 + 8;
             const bool in0 = row_base + r0 < p.k, in1 = row_base + r1 < p.k;
+            const BiasRowPtrs br0 = bias_row_ptrs(p.bias, ra0);
+            const BiasRowPtrs br1 = bias_row_ptrs(p.bias, ra0 + 8);
+            const int gw = p.bias.grid_w;
+            const int ty0 = n0 / gw, tx0 = n0 - ty0 * gw;
+            const bool pairs = (gw & 1) == 0 && (reinterpret_cast<uintptr_t>(p.bias.col) & 7u) == 0;
 #pragma unroll
             for (int g8 = 0; g8 < 8; ++g8) {
+              const int col = 8 * g8 + 2 * j4;
+              if (col >= valid) continue;
+              int x = tx0 + col, y = ty0;
+              if (x >= gw) {
+                const int q = x / gw;
+                y += q;
+                x -= q * gw;
+              }
+              if (pairs) {   // valid is even here (N = grid_h * gw is even)
+                const float2 b0 = in0 ? agent_bias_pair(br0, p.bias, cell_y, cell_x, y, x)
+                                      : make_float2(0.f, 0.f);
+                const float2 b1 = in1 ? agent_bias_pair(br1, p.bias, cell_y, cell_x, y, x)
+                                      : make_float2(0.f, 0.f);
+                v[4 * g8] = fmaf(v[4 * g8], p.c, b0.x * kLog2e);
+                v[4 * g8 + 1] = fmaf(v[4 * g8 + 1], p.c, b0.y * kLog2e);
+                v[4 * g8 + 2] = fmaf(v[4 * g8 + 2], p.c, b1.x * kLog2e);
+                v[4 * g8 + 3] = fmaf(v[4 * g8 + 3], p.c, b1.y * kLog2e);
+              } else {
 #pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int col = 8 * g8 + 2 * j4 + e;
-                float& va = v[4 * g8 + e];
-                float& vb = v[4 * g8 + 2 + e];
-                if (col < valid) {
-                  const int n = n0 + col;
-                  const int y = n / p.bias.grid_w, x = n - y * p.bias.grid_w;
+                for (int e = 0; e < 2; ++e) {
+                  if (col + e >= valid) continue;
+                  int xe = x + e, ye = y;
+                  if (xe >= gw) {   // x < gw, so x + 1 wraps at most once
+                    xe -= gw;
+                    ++ye;
+                  }
+                  float& va = v[4 * g8 + e];
+                  float& vb = v[4 * g8 + 2 + e];
                   va = fmaf(va, p.c,
-                            in0 ? agent_bias_at(p.bias, cell_y, cell_x, ra0, y, x) * kLog2e : 0.f);
+                            in0 ? agent_bias_one(br0, p.bias, cell_y, cell_x, ye, xe) * kLog2e : 0.f);
                   vb = fmaf(vb, p.c,
-                            in1 ? agent_bias_at(p.bias, cell_y, cell_x, ra1, y, x) * kLog2e : 0.f);
+                            in1 ? agent_bias_one(br1, p.bias, cell_y, cell_x, ye, xe) * kLog2e : 0.f);
                 }
               }
             }
@@ -619,6 +683,7 @@ __device__ __forceinline__ void bc_slab_max(uint32_t s_col, int k, int kpad, int
 struct BcRowBias {
   int y0, x0, cell0, y1, x1, cell1;
   bool in0, in1;             // the row is a real token
+  long long h;               // head
   long long hk;              // h * k: agent rows of this head
 };
 
@@ -633,7 +698,7 @@ __device__ __forceinline__ void bc_bias_block(float (&v)[4 * R], int c, int k, i
                                               const BiasParams& b, const BcRowBias& rb) {
   if (b.agent_minor > 0) {
     const long long kp = b.agent_minor;
-    const long long h = rb.hk / k;
+    const long long h = rb.h;
     const long long nb = (long long)b.pool_h * b.pool_w;
 #pragma unroll
     for (int g = 0; g < R; ++g) {
@@ -988,7 +1053,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           rb.x1 = rb.in1 ? n1 - rb.y1 * p.bias.grid_w : 0;
           rb.cell0 = (int)cell_y[rb.y0] * p.bias.pool_w + cell_x[rb.x0];
           rb.cell1 = (int)cell_y[rb.y1] * p.bias.pool_w + cell_x[rb.x1];
-          rb.hk = (long long)(bh % p.H) * p.k;
+          rb.h = (long long)(bh % p.H);
+          rb.hk = rb.h * p.k;
           bc_slab_bias_max(s_col, p.k, kpad, j4, p.c, p.bias, rb, t0, t1);
         } else {
           bc_slab_max(s_col, p.k, kpad, j4, t0, t1);

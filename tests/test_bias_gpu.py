@@ -89,3 +89,28 @@ def test_bias_at_the_sd_latent_size_on_sampled_slices():
                                      full(hb(b1), w.grid_h, w.grid_w, w.pool_h, w.pool_w),
                                      full(hb(b2), w.grid_h, w.grid_w, w.pool_h, w.pool_w))
         assert_close(f64(out[b, h]), ref[0, 0], w.torch_dtype, f"biased O slice {(b, h)}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16])
+def test_bias_with_a_column_component_on_a_4_byte_boundary(dtype):
+    """An even-width grid whose column component starts 4 bytes past an
+    8-byte boundary takes the per-element path of the biased aggregation."""
+    B, H, gh, gw, ph, pw, d = 1, 2, 16, 16, 4, 4, 32
+    N, k = gh * gw, ph * pw
+    q, kk, v = random_qkv((B, H, N, d), seed=5, dtype=dtype)
+    b1 = parts(H, k, gh, gw, 31)
+    b2 = parts(H, k, gh, gw, 32)
+    col = b1[1]
+    buf = torch.zeros(col.numel() + 1, device="cuda")
+    shifted = buf[1:].view(col.shape)
+    shifted.copy_(col.cuda())
+    assert shifted.data_ptr() % 8 == 4
+    out = torch.empty((B, H, N, d), dtype=dtype, device="cuda")
+    eva.agent_attn_forward_bias(q.cuda(), kk.cuda(), v.cuda(), None,
+                                [b1[0].cuda(), shifted, b1[2].cuda()],
+                                [t.cuda() for t in b2], out, B, H, N, d, gh, gw, ph, pw,
+                                1 / math.sqrt(d), dtype_code(dtype))
+    torch.cuda.synchronize()
+    ref = oracle.agent_attn_bias(f64(q), f64(kk), f64(v), gh, gw, ph, pw, 1 / math.sqrt(d),
+                                 full(b1, gh, gw, ph, pw), full(b2, gh, gw, ph, pw))
+    assert_close(f64(out), ref, dtype, "biased O")
