@@ -235,8 +235,9 @@ __global__ void __launch_bounds__(kDwcMaxThreads)
                       int grid_w, int d, int cols, int band, int vslot, int accumulate) {
   extern __shared__ uint8_t dwc_smem[];
   pdl_trigger();
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dwc_smem) + 127) &
-                                             ~uintptr_t(127));
+  // 128-byte aligned by pointer arithmetic on the shared array, so the
+  // compiler keeps the shared address space for every access through it
+  uint8_t* base = dwc_smem + ((128u - (tc::smem_u32(dwc_smem) & 127u)) & 127u);
   T* vring = reinterpret_cast<T*>(base);                                   // [kDwcRing][vslot]
   float* s_w = reinterpret_cast<float*>(vring + (size_t)kDwcRing * vslot);  // [9][d], [d]
   uint64_t* vbar = reinterpret_cast<uint64_t*>(s_w + 10 * d);

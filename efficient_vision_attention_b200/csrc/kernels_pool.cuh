@@ -76,8 +76,9 @@ __global__ void __launch_bounds__(kPoolTmaThreads) agent_pool_tma_kernel(
     int tile_region) {
   extern __shared__ uint8_t pool_smem[];
   pdl_trigger();
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pool_smem) + 127) &
-                                             ~uintptr_t(127));
+  // 128-byte aligned by pointer arithmetic on the shared array, so the
+  // compiler keeps the shared address space for every access through it
+  uint8_t* base = pool_smem + ((128u - (tc::smem_u32(pool_smem) & 127u)) & 127u);
   T* tile = reinterpret_cast<T*>(base);
   float* colsum = reinterpret_cast<float*>(base + tile_region);
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + tile_region + (size_t)cols_max * d * 4);
