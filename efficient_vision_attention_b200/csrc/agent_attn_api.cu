@@ -594,7 +594,7 @@ int dwc_impl(const void* v, const float* w, const float* bias, void* out, int B,
   }
   const long long N = (long long)grid_h * grid_w;
   const long long items = (long long)grid_h * ((grid_w + kDwcSpan - 1) / kDwcSpan) * (d / 8);
-  if (N * (d / 8) >= (1LL << 31)) return AA_ERR_SHAPE;   // per-slice index math is 32-bit
+  if (N * (d / 8) >= (1LL << 31)) return AA_ERR_SHAPE;   // checked by validate_dwc too
   const long long blocks = (items + kDwcThreads - 1) / kDwcThreads;
   const dim3 grid((unsigned)blocks, (unsigned)(BH < 65535 ? BH : 65535));
   const size_t smem = (size_t)10 * d * sizeof(float);
@@ -617,6 +617,7 @@ int validate_dwc(const void* v, const float* w, const void* out, int B, int H, i
   if (B < 1 || H < 1 || grid_h < 1 || grid_w < 1) return AA_ERR_SHAPE;
   if (d < 8 || d > 128 || (d % 8) != 0) return AA_ERR_UNSUPPORTED;
   if ((long long)B * H * grid_h * (long long)grid_w > (1LL << 40)) return AA_ERR_SHAPE;
+  if ((long long)grid_h * grid_w * (d / 8) >= (1LL << 31)) return AA_ERR_SHAPE;
   if (!v || !w || !out) return AA_ERR_NULL;
   if (!aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(w) & 3u)) return AA_ERR_ALIGN;
   return AA_OK;

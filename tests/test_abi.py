@@ -143,6 +143,8 @@ def test_dwc_validation():
     assert f(**{**base, "d": 136}) == 3
     assert f(**{**base, "dtype": 5}) == 3
     assert f(**{**base, "grid_w": 0}) == 2
+    # a slice of 2^31 8-channel groups or more is refused before any launch
+    assert f(**{**base, "grid_h": 1 << 16, "grid_w": 1 << 13, "d": 32}) == 2
     g = eva.agent_attn_forward_dwc
     full = dict(q=A16, k=A16, v=A16, agents_or_null=None, dwc_w=A16, dwc_bias_or_null=None,
                 out=A16, B=1, H=1, N=64, d=32, grid_h=8, grid_w=8, pool_h=2, pool_w=2, scale=0.1,
