@@ -145,6 +145,21 @@ def recorded_traffic(kernel: str, workload: str):
     return None
 
 
+# ex2.approx.f32 results per clock per SM (measured on B200 with a
+# micro-benchmark; the packed bf16x2 / f16x2 forms give no more per clock).
+SFU_EXP_PER_CLK_PER_SM = 16
+
+
+def sfu_roofline(n_exp: int, ms: float, sms: int, mhz: float) -> dict:
+    """The exponential roofline of a softmax kernel: n_exp exponentials per
+    launch in `ms` milliseconds against SFU_EXP_PER_CLK_PER_SM results per
+    clock on each of `sms` SMs at `mhz`."""
+    peak = SFU_EXP_PER_CLK_PER_SM * sms * mhz * 1e6
+    achieved = n_exp / (ms * 1e-3)
+    return {"bound": "sfu", "achieved": achieved, "peak": peak, "unit": "exp/s",
+            "frac": achieved / peak, "exps_per_launch": n_exp, "sm_mhz": mhz}
+
+
 def cpu_baseline(w, target_s=12.0):
     """The fp64 oracle, as it stands, on a bounded sample of the workload:
     whole (b, h) slices, as many as fit in about target_s seconds."""
@@ -338,6 +353,13 @@ def run_native(args, w):
                 "kernel": kernel_name,
                 "algorithmic_bytes_per_launch": half_bytes,
                 "traffic": recorded_traffic(kernel_name, w.name)}
+    # The same kernel against its exponential bound (one exp per score: B*H*N*k
+    # in either stage), at the SM clock the sampler saw as the maximum.
+    clk_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
+    sfu = sfu_roofline(B * H * N * nk, stage_ms[dom],
+                       torch.cuda.get_device_properties(dev).multi_processor_count,
+                       float(clk_mhz))
+    sfu["kernel"] = kernel_name
 
     # The DWC term of the full module (depth-wise 3x3 convolution of V added to
     # O) on the same workload: its own kernel, HBM-bound (V read, O read and
@@ -472,6 +494,7 @@ def run_native(args, w):
         "hbm_frac_aggregate_plus_broadcast": both / peak,
         "stage_ms": stage_ms,
         "roofline": roofline,
+        "sfu_roofline": sfu,
         "dwc_term": dwc,
         "agent_bias_forward": bias_fwd,
         "backward": bwd,
