@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "agent_attn.h"
 #include "common.cuh"
@@ -267,14 +268,21 @@ __global__ void bias_transpose_kernel(const float* __restrict__ src, float* __re
   dst[e] = a < k ? src[((long long)h * k + a) * L + l] : 0.f;
 }
 
+std::mutex g_smem_attr_mutex;   // serialises raising a kernel's shared-memory limit
+
 template <typename KernelT>
 int ensure_smem(KernelT kernel, size_t bytes, std::atomic<int>* flags) {
   int dev = 0;
   AA_CUDA(cudaGetDevice(&dev));
+  if (dev < kMaxDevices && flags[dev].load(std::memory_order_acquire) >= (int)bytes)
+    return AA_OK;
+  // Check, raise and record under one lock, so that a smaller request of
+  // another thread can never lower the limit after a larger one was recorded.
+  std::lock_guard<std::mutex> lock(g_smem_attr_mutex);
   if (dev < kMaxDevices && flags[dev].load(std::memory_order_relaxed) >= (int)bytes)
     return AA_OK;
   AA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
-  if (dev < kMaxDevices) flags[dev].store((int)bytes, std::memory_order_relaxed);
+  if (dev < kMaxDevices) flags[dev].store((int)bytes, std::memory_order_release);
   return AA_OK;
 }
 
