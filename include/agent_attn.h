@@ -30,11 +30,15 @@
  * and > 0; `out` must not alias an input.
  *
  * Ownership: the caller owns every buffer.  The library keeps no pointer to
- * them after a call returns.  Its only global state is per device: a cache of
- * the SM count and a library-owned stream-ordered memory pool (created on
- * first use, release threshold = unlimited) from which the entry points
- * without a caller workspace take their scratch; calls on different streams
- * are independent.
+ * them after a call returns.  Its global state is per device and created on
+ * first use: a cache of the SM count and of each kernel's raised
+ * shared-memory limit; a library-owned stream-ordered memory pool (release
+ * threshold = unlimited) from which the entry points without a caller
+ * workspace take their scratch; one non-blocking side stream (used only by
+ * agent_attn_forward_host); the in-kernel watchdog word read by
+ * agent_attn_check_device_error; and the fixed scratch array of
+ * agent_attn_stage_aggregate_static.  Calls on different streams are
+ * independent.
  *
  * Errors: every call validates all arguments before it launches anything and
  * returns an aa_status.  AA_ERR_CUDA means a CUDA call or launch failed; the
