@@ -200,6 +200,13 @@ def bench_config(w, world, set_bytes=None, n_sets=None):
     return cfg
 
 
+def input_sets(w):
+    """Bytes of one input set and the number of sets the native arm rotates
+    through so that consecutive steps' inputs together exceed L2."""
+    set_bytes = workload_bytes(w, w.B)
+    return set_bytes, max(2, math.ceil(3 * L2_BYTES / set_bytes))
+
+
 def run_reference(args, w):
     from efficient_vision_attention_b200.replicas import dist_env
     world, rank, _ = dist_env()
@@ -220,7 +227,7 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": steps, "warmup": warm, "ms_per_step": 1e3 * el / max(1, steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": bench_config(w, world),
+        "data": "synthetic", "config": bench_config(w, world, *input_sets(w)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": base["cores"], "kind": "oracle",
                          "sample": vals[-1]["sample"] + " per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -246,8 +253,7 @@ def run_native(args, w):
     B, H, N, d, nk = w.B, w.H, w.N, w.d, w.n_agents
 
     # Rotate input sets so that the inputs of consecutive steps together exceed L2.
-    set_bytes = workload_bytes(w, B)
-    n_sets = max(2, math.ceil(3 * L2_BYTES / set_bytes))
+    set_bytes, n_sets = input_sets(w)
     sets = []
     for i in range(n_sets):
         inp = make_inputs(w, seed=replicas.rank_seed(w.seed, rank) + i)

@@ -990,18 +990,25 @@ int agent_attn_stage_aggregate_static(const void* agents, long long agents_batch
   Scratch s;
   plan_scratch(p, sms, &s);
   // The aggregation touches only the partial-state regions [pu_off, total) of
-  // the scratch layout; they are placed at the start of the fixed array.
+  // the scratch layout: a copy of the plan with those regions moved to offset
+  // 0 addresses the fixed array from its start (the agent and V_A regions,
+  // which the aggregation does not use, are left empty).
   const size_t need = s.total - s.pu_off;
   if (need > (size_t)AA_STATIC_SCRATCH_BYTES) return AA_ERR_WORKSPACE;
+  Scratch r = s;
+  r.a_off = r.va_off = r.b2t_off = 0;
+  r.pml_off = s.pml_off - s.pu_off;
+  r.pu_off = 0;
+  r.total = need;
   void* base = nullptr;
   rc = static_scratch_address(&base);
   if (rc != AA_OK) return rc;
-  char* ws = static_cast<char*>(base) - s.pu_off;   // only ws + pu_off onwards is addressed
+  char* ws = static_cast<char*>(base);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   AgentsRef ag{agents, agents_batch_stride, (long long)n_agents * d};
   return (dtype == AA_FP32)
-             ? run_aggregate<float>(p, s, ag, k, v, ws, va_f32, nullptr, st)
-             : run_aggregate<__nv_bfloat16>(p, s, ag, k, v, ws, va_f32,
+             ? run_aggregate<float>(p, r, ag, k, v, ws, va_f32, nullptr, st)
+             : run_aggregate<__nv_bfloat16>(p, r, ag, k, v, ws, va_f32,
                                             static_cast<__nv_bfloat16*>(va_lowp), st);
 }
 

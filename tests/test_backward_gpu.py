@@ -67,3 +67,23 @@ def test_backward_with_given_agents(dtype):
                                                 scale, agents=f64(agents))
     for got, want, name in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV"), (da, ra, "dA")):
         close(f64(got), want, dtype, name)
+
+
+def test_backward_at_the_sd_latent_size():
+    """The bench's backward configuration (2 x 8 slices, N = 16384 on a
+    128 x 128 grid, k = 256 pooled agents, d = 40, bf16): the gradient sums over
+    16384 keys and the per-agent accumulation over 128 query tiles differ most
+    from the small cases; three whole slices are compared with the oracle."""
+    from efficient_vision_attention_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS["sd_latent_1024"]
+    inp = make_inputs(w)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(5)).to(q.dtype)
+    dq, dk, dv, da = run_backward(q, k, v, dout, w.grid_h, w.grid_w, w.pool_h, w.pool_w,
+                                  w.scale)
+    for (b, h) in ((0, 0), (0, 7), (1, 3)):
+        sl = lambda t: f64(t[b:b + 1, h:h + 1])
+        rq, rk, rv, ra = oracle.agent_attn_backward(sl(q), sl(k), sl(v), sl(dout), w.grid_h,
+                                                    w.grid_w, w.pool_h, w.pool_w, w.scale)
+        for got, want, name in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV"), (da, ra, "dA")):
+            close(sl(got), want, q.dtype, f"{name} slice ({b}, {h})")

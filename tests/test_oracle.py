@@ -335,6 +335,44 @@ def test_bias_components_build_the_full_matrix_by_grid_cell():
     assert set(ys * ph // gh) == {4 // pw} and set(xs * pw // gw) == {4 % pw}
 
 
+@pytest.mark.parametrize("gh,gw,ph,pw", [
+    (13, 11, 4, 3), (256, 256, 12, 12), (7, 5, 3, 2), (128, 128, 16, 16), (5, 9, 5, 2),
+    (31, 17, 6, 4)])
+def test_bias_matches_library_nearest_upsampling(gh, gw, ph, pw):
+    """The bias matrix against library routines: the block component is the
+    pool_h x pool_w grid of block values upsampled to the token grid by torch's
+    nearest-neighbour interpolation (source cell floor(y * pool_h / grid_h),
+    floor(x * pool_w / grid_w)), the row and column components are torch
+    broadcasts along the other grid axis.  Non-square pools and non-dividing
+    grids make a swapped pool_h / pool_w, a ceil instead of a floor, or a token
+    assigned to the later of two overlapping adaptive-pool bins fail."""
+    # torch computes the source index in single precision; for these sizes it
+    # agrees with the exact integer floor, which is asserted first
+    for g, p in ((gh, ph), (gw, pw)):
+        idx = F.interpolate(torch.arange(p, dtype=torch.float64).reshape(1, 1, p), size=g,
+                            mode="nearest")[0, 0].numpy().astype(int)
+        assert (idx == (np.arange(g) * p) // g).all()
+    H, k = 2, 3
+    row, col, block = bias_parts(H, k, gh, gw, ph * pw, 61)
+    t_row = torch.from_numpy(row)[:, :, :, None].expand(H, k, gh, gw)
+    t_col = torch.from_numpy(col)[:, :, None, :].expand(H, k, gh, gw)
+    t_blk = F.interpolate(torch.from_numpy(block).reshape(H * k, 1, ph, pw), size=(gh, gw),
+                          mode="nearest").reshape(H, k, gh, gw)
+    want = (torch.zeros(H, k, gh, gw, dtype=torch.float64) + t_row + t_col + t_blk).numpy()
+    got = oracle.agent_bias(row, col, block, gh, gw, ph, pw).reshape(H, k, gh, gw)
+    np.testing.assert_array_equal(got, want)
+    # each component alone, through the same library routines
+    np.testing.assert_array_equal(
+        oracle.agent_bias(None, None, block, gh, gw, ph, pw).reshape(H, k, gh, gw),
+        t_blk.numpy())
+    np.testing.assert_array_equal(
+        oracle.agent_bias(row, None, None, gh, gw, ph, pw).reshape(H, k, gh, gw),
+        t_row.numpy())
+    np.testing.assert_array_equal(
+        oracle.agent_bias(None, col, None, gh, gw, ph, pw).reshape(H, k, gh, gw),
+        t_col.numpy())
+
+
 def test_zero_bias_is_the_plain_forward_pass():
     q, k, v = (rnd((2, 2, 30, 4), s) for s in (51, 52, 53))
     z = np.zeros((2, 4, 30))

@@ -13,6 +13,7 @@ import pytest
 import torch
 
 import efficient_vision_attention_b200 as eva
+import oracle
 from efficient_vision_attention_b200.workloads import random_qkv
 from gpu_helpers import assert_close, dtype_code, f64
 
@@ -39,11 +40,18 @@ def test_static_scratch_matches_regular_entry_point(dtype, B, H, N, n_agents, d)
     g = torch.Generator().manual_seed(21)
     agents = (torch.randn((B, H, n_agents, d), generator=g) * 0.5).to(dtype).cuda()
     k, v = k.cuda(), v.cuda()
-    ref32, _ = aggregate(eva.agent_attn_stage_aggregate, agents, k, v, n_agents, dtype)
+    ref32, reflow = aggregate(eva.agent_attn_stage_aggregate, agents, k, v, n_agents, dtype)
+    want = oracle.agent_aggregate(f64(agents), f64(k), f64(v), 1 / math.sqrt(d))
     for _ in range(2):                     # two calls in a row share the fixed array
-        got32, _ = aggregate(eva.agent_attn_stage_aggregate_static, agents, k, v, n_agents,
-                             dtype)
-        assert_close(f64(got32), f64(ref32), dtype, "static-scratch V_A")
+        got32, gotlow = aggregate(eva.agent_attn_stage_aggregate_static, agents, k, v,
+                                  n_agents, dtype)
+        assert_close(f64(got32), f64(ref32), dtype, "static-scratch V_A vs regular call")
+        assert_close(f64(got32), want, dtype, "static-scratch V_A vs oracle")
+        if dtype != torch.float32:
+            # the run-dtype copy feeds the broadcast: the same bits as the
+            # regular call's, and the fp32 result rounded once
+            assert torch.equal(gotlow, reflow), "static-scratch bf16 V_A differs"
+            assert_close(f64(gotlow), want, dtype, "static-scratch bf16 V_A vs oracle")
     assert eva.agent_attn_check_device_error(check=False) == 0
 
 
