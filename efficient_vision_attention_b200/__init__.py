@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     agent_attn_dwc,
     agent_attn_forward_dwc,
     agent_attn_forward_ws,
+    agent_attn_selftest_exp2,
     agent_attn_stage_pool,
     agent_attn_stage_aggregate,
     agent_attn_stage_aggregate_static,

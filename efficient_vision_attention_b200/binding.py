@@ -56,6 +56,7 @@ _SIGNATURES = {
     "agent_attn_dwc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "agent_attn_forward_dwc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                     _i, _f, _i, _vp]),
+    "agent_attn_selftest_exp2": (_i, [_vp, _vp, _vp, _i, _vp]),
 }
 
 # Size of the library's fixed scratch array (AA_STATIC_SCRATCH_BYTES in the header).
@@ -248,3 +249,8 @@ def agent_attn_backward(q, k, v, agents_or_null, dout, dq, dk, dv, dagents_or_nu
         _ptr(dagents_or_null), B, H, N, d, grid_h, grid_w, pool_h, pool_w, scale, dtype,
         _stream(stream))
     return _finish(st, check)
+
+
+def agent_attn_selftest_exp2(x, y_fma, y_ref, n, stream=None, check=True):
+    return _finish(load_library().agent_attn_selftest_exp2(_ptr(x), _ptr(y_fma), _ptr(y_ref),
+                                                           int(n), _stream(stream)), check)

@@ -794,6 +794,17 @@ int static_scratch_address(void** out) {
   return AA_OK;
 }
 
+// One FMA-pipe exponential and one exp2f per element (agent_attn_selftest_exp2).
+__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y_fma,
+                                     float* __restrict__ y_ref, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float a = x[i], b = x[i];
+  tc::exp2_fma2(a, b);
+  y_fma[i] = a;
+  y_ref[i] = exp2f(x[i]);
+}
+
 }  // namespace
 }  // namespace aa
 
@@ -1045,6 +1056,19 @@ const char* agent_attn_status_string(int status) {
 }
 
 const char* agent_attn_version(void) { return "0.1.0"; }
+
+int agent_attn_selftest_exp2(const float* x, float* y_fma, float* y_ref, int n, void* stream) {
+  if (n < 0) return AA_ERR_SHAPE;
+  if (n == 0) return AA_OK;
+  if (!x || !y_fma || !y_ref) return AA_ERR_NULL;
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y_fma) |
+                        reinterpret_cast<uintptr_t>(y_ref);
+  if (mis & 3u) return AA_ERR_ALIGN;
+  selftest_exp2_kernel<<<(unsigned)((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, y_fma, y_ref, n);
+  AA_CUDA(cudaGetLastError());
+  return AA_OK;
+}
 
 int agent_attn_dwc(const void* v, const float* w, const float* bias_or_null, void* out, int B,
                    int H, int grid_h, int grid_w, int d, int dtype, int accumulate, void* stream) {

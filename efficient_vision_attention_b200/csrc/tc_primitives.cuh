@@ -324,6 +324,68 @@ __device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
       : "+f"(a0), "+f"(a1)
       : "f"(b0), "f"(b1));
 }
+// (a0, a1) = (a0, a1) * (b0, b1) + (c0, c1) on the paired FP32 datapath.
+__device__ __forceinline__ void fma2v(float& a0, float& a1, float b0, float b1, float c0,
+                                      float c1) {
+  asm("{\n\t.reg .b64 x, y, z;\n\t"
+      "mov.b64 x, {%0, %1};\n\t"
+      "mov.b64 y, {%2, %3};\n\t"
+      "mov.b64 z, {%4, %5};\n\t"
+      "fma.rn.f32x2 x, x, y, z;\n\t"
+      "mov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// ------------------------------------------- exponential on the FMA pipe
+// 2^x for a pair of arguments without the SFU, for x <= 2^22 (the softmax
+// arguments here are <= 8).  Cody-Waite split x = j + f with j = rint(x)
+// taken by adding 1.5 * 2^23 (round to nearest in fp32 leaves j in the low
+// mantissa bits of the sum), f = x - j in [-1/2, 1/2] exactly; 2^f from a
+// degree-3 polynomial with coefficients fitted to the smallest maximum
+// relative error on [-1/2, 1/2] (Remez exchange, fit_exp2_poly.py in this
+// directory: 7.5e-5 for the fp32 Horner form); 2^j enters by adding j to the
+// exponent field: the sum's bit pattern shifted left by 23 equals j << 23
+// modulo 2^32.  Arguments are clamped at -125 first, so the exponent field
+// stays >= 1 (results below 2^-125, including x = -inf, come out as about
+// 2^-125, negligible against the row maximum's 1).
+constexpr float kExp2Round = 12582912.0f;            // 1.5 * 2^23
+constexpr float kExp2C0 = 0.999928057f;
+constexpr float kExp2C1 = 0.693260968f;
+constexpr float kExp2C2 = 0.242611125f;
+constexpr float kExp2C3 = 0.0551716685f;
+__device__ __forceinline__ void exp2_fma2(float& x0, float& x1) {
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  float t0 = x0, t1 = x1;
+  add2(t0, t1, kExp2Round, kExp2Round);              // j in the low bits
+  float r0 = t0, r1 = t1;
+  add2(r0, r1, -kExp2Round, -kExp2Round);            // rint(x), exact
+  float f0 = x0, f1 = x1;
+  add2(f0, f1, -r0, -r1);                            // f = x - j, exact
+  float p0 = kExp2C3, p1 = kExp2C3;
+  fma2v(p0, p1, f0, f1, kExp2C2, kExp2C2);
+  fma2v(p0, p1, f0, f1, kExp2C1, kExp2C1);
+  fma2v(p0, p1, f0, f1, kExp2C0, kExp2C0);
+  x0 = __uint_as_float((__float_as_uint(t0) << 23) + __float_as_uint(p0));
+  x1 = __uint_as_float((__float_as_uint(t1) << 23) + __float_as_uint(p1));
+}
+
+// Share of a score row's exponentials taken on the FMA pipe instead of the
+// SFU: this many column pairs out of every 8 (the others use ex2.approx).
+#ifndef AA_EXP_FMA_EIGHTHS
+#define AA_EXP_FMA_EIGHTHS 0
+#endif
+// 2^x of the pair with index i within a row (i = column / 2).
+__device__ __forceinline__ void exp2_pair(float& x0, float& x1, int i) {
+  if ((i & 7) < AA_EXP_FMA_EIGHTHS) {
+    exp2_fma2(x0, x1);
+  } else {
+    x0 = ex2(x0);
+    x1 = ex2(x1);
+  }
+}
+
 // 8 consecutive 32-bit TMEM columns of this thread's lane -> registers.
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
   uint32_t r[8];
@@ -357,7 +419,7 @@ __device__ __forceinline__ float exp_pack32(float (&v)[32], float c, float neg_m
 #pragma unroll
   for (int e = 0; e < 32; e += 2) fma2(v[e], v[e + 1], c, neg_m);
 #pragma unroll
-  for (int e = 0; e < 32; ++e) v[e] = ex2(v[e]);
+  for (int e = 0; e < 32; e += 2) exp2_pair(v[e], v[e + 1], e >> 1);
 #pragma unroll
   for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
   float s0 = v[0], s1 = v[1], s2 = v[2], s3 = v[3];
@@ -525,7 +587,7 @@ __device__ __forceinline__ void slab_exp(float (&v)[4 * R], float c, float neg_m
     fma2(v[4 * g + 2], v[4 * g + 3], c, neg_m1);
   }
 #pragma unroll
-  for (int e = 0; e < 4 * R; ++e) v[e] = ex2(v[e]);
+  for (int e = 0; e < 4 * R; e += 2) exp2_pair(v[e], v[e + 1], e >> 1);
   float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
   for (int g = 0; g < R; ++g) {

@@ -278,6 +278,20 @@ AA_API const char* agent_attn_status_string(int status);
  * check, AA_OK otherwise.  Synchronous with respect to the device. */
 AA_API int agent_attn_check_device_error(void);
 
+/* Test hook for the exponential that the tensor-core softmax kernels take on
+ * the FMA pipe for part of each score row instead of the SFU.  No counterpart
+ * in the pages: it exists so that this function can be checked against
+ * CUDA's exp2f.  It computes 2^x by the Cody-Waite split x = j + f
+ * (j = rint(x), f in [-1/2, 1/2]), a degree-3 polynomial for 2^f fitted to
+ * the smallest maximum relative error on [-1/2, 1/2] (7.5e-5) and the
+ * exponent-field insertion of j; arguments below -125 give about 2^-125.
+ *   x     : [n] device floats (4-byte aligned), the arguments;
+ *   y_fma : [n] device floats, the FMA-pipe exponential of x;
+ *   y_ref : [n] device floats, exp2f(x).
+ * n >= 0 (0 launches nothing); asynchronous on `stream`. */
+AA_API int agent_attn_selftest_exp2(const float* x, float* y_fma, float* y_ref, int n,
+                                    void* stream);
+
 /* Library version, "major.minor.patch". */
 AA_API const char* agent_attn_version(void);
 

@@ -481,3 +481,32 @@ def test_backward_sums_follow_the_forward_invariances():
     _, dk, dv, _ = oracle.agent_attn_backward(q, k, v, do, 4, 6, 2, 3, 0.5)
     np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
     np.testing.assert_allclose(dv.sum(axis=2), do.sum(axis=2), rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------- the kernels' FMA-pipe exponential
+def test_fma_exp2_polynomial_constants_meet_their_bound():
+    """The degree-3 coefficients compiled into the tensor-core kernels,
+    evaluated in fp32 Horner form as the kernels do, approximate 2^f on
+    [-1/2, 1/2] to a relative error below 1e-4 (the fit reports 7.5e-5); a
+    dropped or mistyped coefficient fails."""
+    import re
+    src = open(os.path.join(os.path.dirname(os.path.dirname(__file__)),
+                            "efficient_vision_attention_b200", "csrc",
+                            "tc_primitives.cuh")).read()
+    coef = [np.float32(re.search(rf"kExp2C{i} = ([0-9.e+-]+)f;", src).group(1))
+            for i in range(4)]
+    f = np.linspace(-0.5, 0.5, 1_000_001).astype(np.float32)
+    p = np.full_like(f, coef[3])
+    for c in coef[2::-1]:
+        p = (p * f + c).astype(np.float32)
+    rel = np.abs(p.astype(np.float64) / np.exp2(f.astype(np.float64)) - 1.0)
+    assert rel.max() < 1e-4
+    # whole arguments: rint split, exponent insertion (2^j exactly) times p(f)
+    x = np.linspace(-125.0, 8.0, 200_001).astype(np.float32)
+    j = np.rint(x)
+    fx = (x - j).astype(np.float32)
+    px = np.full_like(fx, coef[3])
+    for c in coef[2::-1]:
+        px = (px * fx + c).astype(np.float32)
+    y = px.astype(np.float64) * np.exp2(j)
+    assert np.abs(y / np.exp2(x.astype(np.float64)) - 1.0).max() < 1e-4
