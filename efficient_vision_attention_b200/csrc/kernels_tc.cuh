@@ -51,6 +51,7 @@ namespace tc {
 constexpr int kSoftmaxThreads = 256;           // per softmax group: 8 warps, two per lane quadrant
 constexpr int kFirstSoftmaxWarp = 3;
 constexpr int kThreads = kFirstSoftmaxWarp * 32 + 2 * kSoftmaxThreads;
+constexpr int kSoftmaxWarps = kSoftmaxThreads / 32;  // arrivals per group on its barriers
 constexpr int kRowBytes = 128;               // one swizzled 128-byte row per token (d <= 64 bf16)
 constexpr int kKeyTile = 64;                 // keys per aggregation tile
 constexpr int kQTile = 128;                  // queries per broadcast tile (MMA M)
@@ -123,6 +124,16 @@ __host__ __device__ constexpr int round16(int x) { return (x + 15) & ~15; }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// One arrival per warp on a barrier that counts warps: every lane's earlier
+// tcgen05 and shared-memory accesses are ordered before the warp-wide sync,
+// after which lane 0 arrives (a warp-collective call; the warp must be
+// converged).  One shared-memory atomic per warp instead of 32.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  tc_fence_before();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // Agent set coordinates (h, b) of slice bh for the 4-D agents tensor map.
@@ -236,13 +247,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = 0; g < 2; ++g) {
       for (int b = 0; b < kSBuf; ++b) {
         mbar_init(&bars->s_full[g][b], 1);
-        mbar_init(&bars->p_full[g][b], kSoftmaxThreads);
+        mbar_init(&bars->p_full[g][b], kSoftmaxWarps);
         mbar_init(&bars->pv_done[g][b], 1);
       }
       mbar_init(&bars->drain[g], 1);
     }
-    mbar_init(&bars->x_pub, kSoftmaxThreads);
-    mbar_init(&bars->x_done, kSoftmaxThreads);
+    mbar_init(&bars->x_pub, kSoftmaxWarps);
+    mbar_init(&bars->x_done, kSoftmaxWarps);
     bars->abort = 0;
     mbar_fence_init();
     prefetch_tensormap(&map_k);
@@ -520,8 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_st();
           }
         }
-        tc_fence_before();
-        mbar_arrive(&bars->p_full[g][b]);
+        warp_arrive(&bars->p_full[g][b]);
         ++J;
       }
       // ---- segment epilogue: write this CTA's partial for slice bh
@@ -570,8 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bars->l_x[r0] = l0;
           bars->l_x[r1] = l1;
         }
-        tc_fence_before();
-        mbar_arrive(&bars->x_pub);
+        warp_arrive(&bars->x_pub);
         if (ok) ok = warp_wait(&bars->x_done, (uint32_t)seg & 1, abort);
         tc_fence_after();
       } else {
@@ -627,8 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               *reinterpret_cast<float2*>(p.part_ml + (slot_row + r1) * 2) = make_float2(mm1, lt1);
           }
         }
-        tc_fence_before();
-        mbar_arrive(&bars->x_done);
+        warp_arrive(&bars->x_done);
       }
       // group 1 writes m_x / l_x again only after the next segment's x_done
       // phase, which follows group 0's reads of this one
@@ -793,7 +801,7 @@ __device__ __forceinline__ int bc_p_col(int ch, bool wide) { return (wide && ch 
 
 // P = 2^(S*c - m_row) as bf16 for score columns [0, kpad) (columns >= k give
 // 0), placed by bc_p_col.  Adds the exponentials to the partial row sums l0,
-// l1.  After each 64-column chunk the thread arrives on that chunk's barrier
+// l1.  After each 64-column chunk the warp arrives on that chunk's barrier
 // (whether or not it did the work).
 __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int j4, bool wide,
                                             float c_scale, float neg_m0, float neg_m1, float& l0,
@@ -810,8 +818,7 @@ __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int
       slab_st_p32(s_col + bc_p_col(ch, wide), pk);
       tmem_wait_st();
     }
-    tc_fence_before();
-    mbar_arrive(&chunk_bar[ch]);
+    warp_arrive(&chunk_bar[ch]);
   }
   if (c < kpad) {
     if (run) {
@@ -835,8 +842,7 @@ __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int
       }
       tmem_wait_st();
     }
-    tc_fence_before();
-    mbar_arrive(&chunk_bar[ch]);
+    warp_arrive(&chunk_bar[ch]);
   }
 }
 
@@ -881,9 +887,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->ag_empty, 2);          // both issuers are done with the slice
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      for (int c = 0; c < 4; ++c) mbar_init(&bars->p_chunk[i][c], kSoftmaxThreads);
+      for (int c = 0; c < 4; ++c) mbar_init(&bars->p_chunk[i][c], kSoftmaxWarps);
       mbar_init(&bars->o_full[i], 1);
-      mbar_init(&bars->o_free[i], kSoftmaxThreads);
+      mbar_init(&bars->o_free[i], kSoftmaxWarps);
       mbar_init(&bars->drain[i], 1);
     }
     bars->abort = 0;
@@ -1077,8 +1083,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 8; ++e) o[q][e] = 0.f;
         }
       }
-      tc_fence_before();
-      mbar_arrive(&bars->o_free[g]);           // the buffer may take the next S now
+      warp_arrive(&bars->o_free[g]);           // the buffer may take the next S now
       if (leader) tma_store_wait_read();
       named_barrier(3 + g, kSoftmaxThreads);
 #pragma unroll
