@@ -10,7 +10,8 @@
 // divides by its token count.  fp32 sums.  Bins follow the adaptive-pool
 // convention [floor(iG/P), ceil((i+1)G/P)) (they may overlap by one token).
 // The host uses this kernel when the tile of one agent column fits the
-// shared-memory budget and falls back to agent_pool_kernel otherwise.
+// shared-memory budget and falls back to agent_pool_kernel otherwise; bf16 Q
+// on a grid that the bins divide exactly goes to agent_pool_band_kernel.
 #pragma once
 
 #include "common.cuh"
@@ -162,6 +163,120 @@ __global__ void __launch_bounds__(kPoolTmaThreads) agent_pool_tma_kernel(
       const float m = acc[i] * inv;
       if (a_f32) a_f32[off + i] = m;
       if (a_lowp) a_lowp[off + i] = from_f32<T>(m);
+    }
+  }
+}
+
+
+// ------------------------------------------------ uniform bins, bf16 Q
+// When the bins tile the grid exactly (grid_h = R pool_h, grid_w = W pool_w)
+// every agent averages an R x W block, and a CTA takes one band of R grid
+// rows and a chunk of token columns of one slice: a thread per (token column,
+// 8-channel group) issues the R 16-byte loads of its column at once (all in
+// flight, straight into registers, no staging), sums them in fp32 into a
+// shared column sum, and a thread per (agent, 8-channel group) then adds the
+// W columns of its bin and divides by R W.
+constexpr int kPoolBandMaxRows = 16;
+
+struct PoolBandPlan {
+  int rows, bin_w, chunk_cols, threads;
+  size_t smem;
+  bool ok;
+};
+
+inline PoolBandPlan pool_band_plan(int grid_h, int grid_w, int pool_h, int pool_w, int d) {
+  PoolBandPlan pl{0, 0, 0, 0, 0, false};
+  if (grid_h % pool_h != 0 || grid_w % pool_w != 0 || d % 8 != 0) return pl;
+  pl.rows = grid_h / pool_h;
+  pl.bin_w = grid_w / pool_w;
+  if (pl.rows > kPoolBandMaxRows) return pl;
+  const int groups = d / 8;
+  // whole bins per chunk: the fewest that divide pool_w and span at least
+  // 32 token columns (all of them when no smaller divisor does)
+  const int want = (32 + pl.bin_w - 1) / pl.bin_w;
+  int bins = pool_w;
+  for (int b = 1; b < pool_w; ++b)
+    if (pool_w % b == 0 && b >= want) {
+      bins = b;
+      break;
+    }
+  pl.chunk_cols = bins * pl.bin_w;
+  const int items = pl.chunk_cols * groups;
+  pl.threads = ((items + 31) / 32) * 32;
+  if (pl.threads > 1024) return pl;
+  pl.smem = (size_t)items * 8 * sizeof(float);
+  pl.ok = pl.smem <= 48 * 1024;
+  return pl;
+}
+
+template <typename T>
+__global__ void agent_pool_band_kernel(const __nv_bfloat16* __restrict__ q,
+                                       float* __restrict__ a_f32, T* __restrict__ a_lowp, int N,
+                                       int d, int grid_w, int pool_h, int pool_w, int rows,
+                                       int bin_w, int chunk_cols) {
+  extern __shared__ float band_colsum[];
+  pdl_trigger();
+  const int n_chunks = grid_w / chunk_cols;
+  const int py = blockIdx.x / n_chunks, ch = blockIdx.x - py * n_chunks;
+  const long long bh = blockIdx.y;
+  const int groups = d >> 3;
+  const int xs = ch * chunk_cols;
+  const int items = chunk_cols * groups;
+  const int it = threadIdx.x;
+  if (it < items) {
+    const int x = it / groups, g = it - x * groups;
+    const __nv_bfloat16* src =
+        q + (bh * (long long)N + (long long)py * rows * grid_w + xs + x) * d + g * 8;
+    const long long row_step = (long long)grid_w * d;
+    uint4 raw[kPoolBandMaxRows];
+#pragma unroll
+    for (int r = 0; r < kPoolBandMaxRows; ++r)
+      if (r < rows) raw[r] = __ldcs(reinterpret_cast<const uint4*>(src + r * row_step));
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int r = 0; r < kPoolBandMaxRows; ++r) {
+      if (r < rows) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[r]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(h[i]);
+          acc[2 * i] += f.x;
+          acc[2 * i + 1] += f.y;
+        }
+      }
+    }
+    float4* cs = reinterpret_cast<float4*>(band_colsum + (size_t)it * 8);
+    cs[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    cs[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+  __syncthreads();
+  const int per = chunk_cols / bin_w;            // agents of this chunk
+  if (it < per * groups) {
+    const int pxl = it / groups, g = it - pxl * groups;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int x = pxl * bin_w; x < (pxl + 1) * bin_w; ++x) {
+      const float4* cs = reinterpret_cast<const float4*>(band_colsum + ((size_t)x * groups + g) * 8);
+      const float4 a = cs[0], b = cs[1];
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+    const float inv = 1.f / (float)(rows * bin_w);
+    const int px = ch * per + pxl;
+    const long long off = (bh * pool_h * (long long)pool_w + (long long)py * pool_w + px) * d + g * 8;
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = acc[i] * inv;
+    if (a_f32) {
+      *reinterpret_cast<float4*>(a_f32 + off) = make_float4(m[0], m[1], m[2], m[3]);
+      *reinterpret_cast<float4*>(a_f32 + off + 4) = make_float4(m[4], m[5], m[6], m[7]);
+    }
+    if (a_lowp) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a_lowp[off + i] = from_f32<T>(m[i]);
     }
   }
 }

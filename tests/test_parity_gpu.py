@@ -71,7 +71,9 @@ def test_shapes_and_edges(dtype, B, H, gh, gw, ph, pw, d):
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_stage_pool(dtype):
     B, H, gh, gw, d = 2, 3, 56, 56, 32
-    for ph, pw in [(7, 7), (12, 5), (16, 16), (1, 1), (3, 56)]:
+    # uniform bins (8x8, 4x4, 14x1, 7x8 tokens) take the band kernel for bf16;
+    # the others the staged kernel
+    for ph, pw in [(7, 7), (12, 5), (16, 16), (1, 1), (3, 56), (14, 14), (4, 56), (8, 7)]:
         q, _, _ = random_qkv((B, H, gh * gw, d), seed=ph * 31 + pw, dtype=dtype)
         qd = q.cuda()
         a32 = torch.empty((B, H, ph * pw, d), dtype=torch.float32, device="cuda")
@@ -86,6 +88,23 @@ def test_stage_pool(dtype):
             # bf16 can land one bf16 ulp (2^-7 relative at most) away
             np.testing.assert_allclose(f64(alow), f64(torch.from_numpy(ref).to(dtype)),
                                        rtol=2 ** -7, atol=1e-6)
+
+
+@pytest.mark.parametrize("gh,gw,ph,pw,d", [(128, 128, 16, 16, 40), (256, 256, 16, 16, 64),
+                                         (14, 14, 7, 7, 64), (48, 96, 3, 32, 8)])
+def test_stage_pool_uniform_bins(gh, gw, ph, pw, d):
+    """Grids that the bins divide exactly (the band kernel for bf16): the SD
+    latent, high-res, DeiT shapes and one with 16x3-token bins and d = 8."""
+    B, H = 2, 3
+    q, _, _ = random_qkv((B, H, gh * gw, d), seed=gh + pw + d, dtype=torch.bfloat16)
+    a32 = torch.empty((B, H, ph * pw, d), dtype=torch.float32, device="cuda")
+    alow = torch.empty((B, H, ph * pw, d), dtype=torch.bfloat16, device="cuda")
+    eva.agent_attn_stage_pool(q.cuda(), a32, alow, B, H, gh * gw, d, gh, gw, ph, pw, eva.AA_BF16)
+    torch.cuda.synchronize()
+    ref = oracle.agent_pool(f64(q), gh, gw, ph, pw)
+    np.testing.assert_allclose(f64(a32), ref, rtol=0, atol=2e-6)
+    np.testing.assert_allclose(f64(alow), f64(torch.from_numpy(ref).to(torch.bfloat16)),
+                               rtol=2 ** -7, atol=1e-6)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
