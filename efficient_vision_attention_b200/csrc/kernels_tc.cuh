@@ -61,6 +61,7 @@ constexpr int kAggStages = 8;
 constexpr int kSBuf = 3;                     // score buffers per aggregation group
 constexpr int kBcStages = 4;
 constexpr int kMaxAgents = 256;
+constexpr int kAgentBufBytes = kMaxAgents * kRowBytes;   // one agent tile (all agents of a slice)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale only when the max grows by > 2^8
 
 // Agent bias in the score tiles: for agent a and grid token (y, x) of head h,
@@ -100,7 +101,7 @@ struct BcParams {
 
 struct AggBars {
   uint64_t full[kAggStages], empty[kAggStages];
-  uint64_t a_full, a_empty;
+  uint64_t a_full[2], a_empty[2];   // agent tile buffers, alternating per segment
   uint64_t s_full[2][kSBuf], p_full[2][kSBuf], pv_done[2][kSBuf];   // [group][score buffer]
   uint64_t x_pub, x_done;    // group 1 -> group 0 hand-over per segment (k <= 128)
   uint64_t drain[2];
@@ -206,7 +207,7 @@ __device__ __forceinline__ float agent_bias_one(const BiasRowPtrs& r, const Bias
   return v;
 }
 
-constexpr size_t kAggSmemBytes = 1024 + (size_t)kMaxAgents * kRowBytes +
+constexpr size_t kAggSmemBytes = 1024 + 2 * (size_t)kAgentBufBytes +
                                  2 * (size_t)kAggStages * kKTileBytes + sizeof(AggBars) +
                                  2 * (size_t)kBiasGridMax;
 
@@ -220,8 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                               AggParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sA = smem;
-  uint8_t* sK = sA + kMaxAgents * kRowBytes;
+  uint8_t* sA = smem;                                  // 2 agent tile buffers
+  uint8_t* sK = sA + 2 * kAgentBufBytes;
   uint8_t* sV = sK + kAggStages * kKTileBytes;
   AggBars* bars = reinterpret_cast<AggBars*>(sV + kAggStages * kKTileBytes);
   int16_t* cell_y = reinterpret_cast<int16_t*>(reinterpret_cast<uint8_t*>(bars) + sizeof(AggBars));
@@ -242,8 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], two ? 2 : 1);   // released by every group that used the tile
     }
-    mbar_init(&bars->a_full, 1);
-    mbar_init(&bars->a_empty, 2);                 // both issuers finish the segment
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->a_full[b], 1);
+      mbar_init(&bars->a_empty[b], 2);            // both issuers finish the segment
+    }
     for (int g = 0; g < 2; ++g) {
       for (int b = 0; b < kSBuf; ++b) {
         mbar_init(&bars->s_full[g][b], 1);
@@ -280,17 +283,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------------ TMA producer
       long long it = 0;
-      int seg = 0;
+      int seg = 0, a_loads = 0;
       const uint32_t a_bytes = (two ? 256 : 128) * kRowBytes;
       pdl_wait();             // the agents may come from the previous kernel
       for (long long t = t_begin; t < t_end; ++seg) {
         const long long bh = t / tps;
         const long long seg_end = min(t_end, (bh + 1) * tps);
-        if (seg > 0 && !mbar_wait(&bars->a_empty, (seg - 1) & 1, abort)) break;
+        // the segment's agents go to buffer seg % 2 once segment seg - 2 is
+        // done with it, so they load while segment seg - 1 still computes
+        const int ab = seg & 1;
+        if (seg >= 2 && !mbar_wait(&bars->a_empty[ab], (uint32_t)((seg - 2) >> 1) & 1, abort))
+          break;
         int h, b;
         agent_coords(bh, p.H, a_sets, &h, &b);
-        mbar_expect_tx(&bars->a_full, a_bytes);
-        tma_load_4d(sA, &map_a, &bars->a_full, 0, 0, h, b);
+        mbar_expect_tx(&bars->a_full[ab], a_bytes);
+        tma_load_4d(sA + ab * kAgentBufBytes, &map_a, &bars->a_full[ab], 0, 0, h, b);
+        ++a_loads;
         bool ok = true;
         for (; t < seg_end; ++t, ++it) {
           const int s = (int)(it % kAggStages);
@@ -306,11 +314,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
       }
-      // On abort, wait (bounded) for the loads already issued before leaving.
+      // On abort, wait (bounded) for the loads already issued before leaving:
+      // the key tiles still in the ring and the last two agent tiles.
       if (*abort) {
         for (long long j = (it > kAggStages ? it - kAggStages : 0); j < it; ++j) {
           const uint64_t t0 = globaltimer();
           while (!mbar_try_wait(&bars->full[j % kAggStages], (uint32_t)(j / kAggStages) & 1) &&
+                 globaltimer() - t0 < kWaitLimitNs) {
+          }
+        }
+        for (int sg = (a_loads > 2 ? a_loads - 2 : 0); sg < a_loads; ++sg) {
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(&bars->a_full[sg & 1], (uint32_t)(sg >> 1) & 1) &&
                  globaltimer() - t0 < kWaitLimitNs) {
           }
         }
@@ -322,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int g = warp - 1;
       const uint32_t idesc_s = idesc_bf16(128, kKeyTile, 0, 0);
       const uint32_t idesc_pv = idesc_bf16(128, dn, 0, 1);
-      const uint32_t sA_addr = smem_u32(sA) + (two ? g : 0) * 128 * kRowBytes;
+      const uint32_t sA_half = smem_u32(sA) + (two ? g : 0) * 128 * kRowBytes;
       const uint32_t sK_addr = smem_u32(sK), sV_addr = smem_u32(sV);
       const uint32_t u_tm = tmem + g * 256 + 192;
       long long it0 = 0;
@@ -333,7 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long bh = t / tps;
         const long long seg_end = min(t_end, (bh + 1) * tps);
         const int n = (int)(seg_end - t);
-        if (!mbar_wait(&bars->a_full, seg & 1, abort)) break;
+        const int ab = seg & 1;
+        const uint32_t sA_addr = sA_half + ab * kAgentBufBytes;
+        if (!mbar_wait(&bars->a_full[ab], (uint32_t)(seg >> 1) & 1, abort)) break;
         tc_fence_after();
         bool first = true;
         auto issue_s = [&](int i) -> bool {
@@ -388,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (i + kAhead * step < n) ok = issue_s(i + kAhead * step);
           if (ok) ok = issue_pv(i);
         }
-        mma_commit(&bars->a_empty);
+        mma_commit(&bars->a_empty[ab]);
         it0 += n;
         t = seg_end;
       }
