@@ -147,6 +147,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);   // .x (low 16 bits) = lo
   return *reinterpret_cast<uint32_t*>(&h);
 }
+// The two bf16 values of a packed word, widened exactly to fp32.
+__device__ __forceinline__ float bf16x2_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16x2_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// 1: a softmax row sum adds the bf16-rounded P values, i.e. exactly the
+// weights the P.V MMA uses, so the normalised weights of a row sum to one up
+// to fp32 rounding; 0 (default): it adds the fp32 exponentials before
+// rounding, whose sum differs from the rounded one by the bf16 rounding
+// errors of the row (each below 2^-9 relative, of either sign).  The rounded
+// sum costs two integer operations per column pair, measured at about 4% of
+// the broadcast kernel on the SD-latent workload.
+#ifndef AA_ROUNDED_SUM
+#define AA_ROUNDED_SUM 0
+#endif
 
 // ------------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
@@ -399,37 +413,6 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
-// Row max of 32 values, seeded with m.
-__device__ __forceinline__ float max32(const float (&v)[32], float m) {
-  float a = fmax3(m, v[0], v[1]), b = fmax3(v[2], v[3], v[4]), c = fmax3(v[5], v[6], v[7]);
-  float e = fmax3(v[8], v[9], v[10]), f = fmax3(v[11], v[12], v[13]);
-  float g = fmax3(v[14], v[15], v[16]), h = fmax3(v[17], v[18], v[19]);
-  float i = fmax3(v[20], v[21], v[22]), j = fmax3(v[23], v[24], v[25]);
-  float k = fmax3(v[26], v[27], v[28]), l = fmax3(v[29], v[30], v[31]);
-  a = fmax3(a, b, c);
-  e = fmax3(e, f, g);
-  h = fmax3(h, i, j);
-  k = fmaxf(k, l);
-  return fmax3(fmax3(a, e, h), k, k);
-}
-// P = 2^(S*c - m) for 32 scores, packed to 16 bf16x2 words.
-// Returns the fp32 sum of the 32 exponentials (paired adds on the FMA pipe).
-__device__ __forceinline__ float exp_pack32(float (&v)[32], float c, float neg_m,
-                                            uint32_t (&pk)[16]) {
-#pragma unroll
-  for (int e = 0; e < 32; e += 2) fma2(v[e], v[e + 1], c, neg_m);
-#pragma unroll
-  for (int e = 0; e < 32; e += 2) exp2_pair(v[e], v[e + 1], e >> 1);
-#pragma unroll
-  for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-  float s0 = v[0], s1 = v[1], s2 = v[2], s3 = v[3];
-#pragma unroll
-  for (int e = 4; e < 32; e += 4) {
-    add2(s0, s1, v[e], v[e + 1]);
-    add2(s2, s3, v[e + 2], v[e + 3]);
-  }
-  return (s0 + s1) + (s2 + s3);
-}
 
 // ------------------------------------------------- 16-lane slab access
 // The 16x256b / 16x128b shapes move 16 TMEM lanes (a 16-aligned base lane
@@ -576,8 +559,8 @@ __device__ __forceinline__ float row4_sum(float x) {
   return x + __shfl_xor_sync(0xffffffffu, x, 2);
 }
 // P = 2^(S*c - m_row) for a 16x256b register block of both rows, packed to
-// bf16x2 words in the 16x128b order; the fp32 exponentials are added to the
-// rows' partial sums l0, l1.
+// bf16x2 words in the 16x128b order; the rows' partial sums l0, l1 add the
+// rounded P (or the fp32 exponentials, AA_ROUNDED_SUM = 0).
 template <int R>
 __device__ __forceinline__ void slab_exp(float (&v)[4 * R], float c, float neg_m0, float neg_m1,
                                          uint32_t (&pk)[2 * R], float& l0, float& l1) {
@@ -593,8 +576,13 @@ __device__ __forceinline__ void slab_exp(float (&v)[4 * R], float c, float neg_m
   for (int g = 0; g < R; ++g) {
     pk[2 * g] = pack_bf16x2(v[4 * g], v[4 * g + 1]);
     pk[2 * g + 1] = pack_bf16x2(v[4 * g + 2], v[4 * g + 3]);
+#if AA_ROUNDED_SUM
+    add2(a0, a1, bf16x2_lo(pk[2 * g]), bf16x2_hi(pk[2 * g]));
+    add2(b0, b1, bf16x2_lo(pk[2 * g + 1]), bf16x2_hi(pk[2 * g + 1]));
+#else
     add2(a0, a1, v[4 * g], v[4 * g + 1]);
     add2(b0, b1, v[4 * g + 2], v[4 * g + 3]);
+#endif
   }
   l0 += a0 + a1;
   l1 += b0 + b1;

@@ -47,6 +47,29 @@ def test_workload_matches_oracle(name):
     assert_close(got, ref, w.torch_dtype, name)
 
 
+@pytest.mark.parametrize("B,H,gh,gw,ph,pw,d", [
+    (4, 3, 14, 14, 7, 7, 64),      # DeiT-shaped slices: N = 196, k = 49
+    (2, 2, 13, 11, 4, 3, 40),      # N = 143, overlapping bins, d = 40
+    (1, 3, 9, 20, 1, 1, 8),        # one agent, d = 8
+    (2, 1, 16, 16, 16, 8, 64),     # k = 128 (the tile), N = 256 (the limit)
+    (3, 2, 10, 10, 10, 10, 32),    # k = N = 100: every token an agent
+    (1, 2, 7, 7, 3, 3, 16),        # N = 49, bins 3x3 over 7 tokens
+    (5, 1, 12, 15, 5, 4, 24),      # N = 180, k = 20, non-dividing bins
+])
+def test_fused_small_slices_match_oracle(B, H, gh, gw, ph, pw, d):
+    """bf16 slices of at most 256 tokens with at most 128 pooled agents and
+    d <= 64 run the whole pass in one CTA per slice (agent_fused_small_tc):
+    every output against the oracle, and twice in a row bit-identical."""
+    N = gh * gw
+    q, k, v = random_qkv((B, H, N, d), seed=3 * N + d, dtype=torch.bfloat16)
+    scale = 1 / math.sqrt(d)
+    out = run_forward(q, k, v, gh, gw, ph, pw, scale, guard=1024)
+    again = run_forward(q, k, v, gh, gw, ph, pw, scale, guard=1024)
+    assert torch.equal(out, again)
+    ref = oracle.agent_attn(f64(q), f64(k), f64(v), gh, gw, ph, pw, scale)
+    assert_close(f64(out), ref, torch.bfloat16, f"{B}x{H} {gh}x{gw}->{ph}x{pw} d={d}")
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("B,H,gh,gw,ph,pw,d", [
     (1, 1, 8, 8, 2, 2, 32),        # tiny
