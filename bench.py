@@ -274,7 +274,8 @@ def run_native(args, w):
                                       w.grid_h, w.grid_w, w.pool_h, w.pool_w, w.scale, dt, ws,
                                       ws_bytes, stream)
 
-    launches_per_step = 3 if w.learnable_agents else 4
+    fused = takes_fused_small_path(w)
+    launches_per_step = 1 if fused else (3 if w.learnable_agents else 4)
     for i in range(max(3, args.warmup)):
         step(i)
     torch.cuda.synchronize()
@@ -359,10 +360,20 @@ def run_native(args, w):
                 "kernel": kernel_name,
                 "algorithmic_bytes_per_launch": half_bytes,
                 "traffic": recorded_traffic(kernel_name, w.name)}
+    if fused:
+        # the whole pass is one kernel: Q, K, V read once, O written once per
+        # launch, timed as the step itself (one launch per step)
+        fused_bytes = 2 * half_bytes
+        achieved = fused_bytes / (ms_max * 1e-3) / 1e9
+        dom, kernel_name = None, "agent_fused_small"
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "peak_kind": f"of {peak_kind}",
+                    "kernel": kernel_name, "algorithmic_bytes_per_launch": fused_bytes,
+                    "traffic": recorded_traffic(kernel_name, w.name)}
     # The same kernel against its exponential bound (one exp per score: B*H*N*k
     # in either stage), at the SM clock the sampler saw as the maximum.
     clk_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
-    sfu = sfu_roofline(B * H * N * nk, stage_ms[dom],
+    sfu = sfu_roofline((2 if fused else 1) * B * H * N * nk, ms_max if fused else stage_ms[dom],
                        torch.cuda.get_device_properties(dev).multi_processor_count,
                        float(clk_mhz))
     sfu["kernel"] = kernel_name
@@ -499,6 +510,8 @@ def run_native(args, w):
         "hbm_gbs_aggregate_plus_broadcast": both,
         "hbm_frac_aggregate_plus_broadcast": both / peak,
         "stage_ms": stage_ms,
+        "forward_path": "fused_small (one kernel)" if fused else
+                        "pool + aggregate + merge + broadcast",
         "roofline": roofline,
         "sfu_roofline": sfu,
         "dwc_term": dwc,
@@ -510,6 +523,20 @@ def run_native(args, w):
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)
+
+
+def takes_fused_small_path(w) -> bool:
+    """Whether the library runs this workload's forward pass as the single
+    fused small-slice kernel: bf16, pooled agents, N <= 256, k <= 128,
+    8 <= d <= 64 with d % 8 == 0, and the O staging tiles fitting the K and V
+    buffers (the rule of fused_small_fits in kernels_fused.cuh)."""
+    N, d, k = w.grid_h * w.grid_w, w.d, w.pool_h * w.pool_w
+    if w.dtype != "bf16" or w.learnable_agents or not (1 <= N <= 256 and 1 <= k <= 128):
+        return False
+    if not (8 <= d <= 64 and d % 8 == 0):
+        return False
+    rows = (N + 15) // 16 * 16
+    return 2 * rows * 128 >= ((N + 127) // 128) * 128 * 128
 
 
 def main():
