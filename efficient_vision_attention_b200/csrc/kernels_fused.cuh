@@ -42,7 +42,8 @@ constexpr int kFusedMaxAgents = 128;
 constexpr int kFusedTmemCols = 256;
 
 struct FusedBars {
-  uint64_t tma;              // Q, K, V staged
+  uint64_t tma_q;            // Q staged
+  uint64_t tma_kv;           // K and V staged
   uint64_t mma;              // one phase per MMA batch (S1, P1 V, S2, P2 V_A)
   uint64_t chunk[4];         // arrivals of the slab softmax routines (never waited on)
   uint64_t drain;            // completion of every MMA before TMEM is released
@@ -129,7 +130,8 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
   const int n_qt = (N + kQTile - 1) / kQTile;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->tma, 1);
+    mbar_init(&bars->tma_q, 1);
+    mbar_init(&bars->tma_kv, 1);
     mbar_init(&bars->mma, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&bars->chunk[i], kFusedThreads / 32);
     mbar_init(&bars->drain, 1);
@@ -151,16 +153,20 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
 
   if (threadIdx.x == 0) {
     pdl_wait();
-    mbar_expect_tx(&bars->tma, 3u * (uint32_t)L.n_box * (uint32_t)L.box_rows * kRowBytes);
+    // Q on its own barrier, so the pooling starts while K and V still load
+    mbar_expect_tx(&bars->tma_q, (uint32_t)L.n_box * (uint32_t)L.box_rows * kRowBytes);
+    mbar_expect_tx(&bars->tma_kv, 2u * (uint32_t)L.n_box * (uint32_t)L.box_rows * kRowBytes);
+    for (int b = 0; b < L.n_box; ++b)
+      tma_load_3d(sQ + (uint32_t)b * L.box_rows * kRowBytes, &map_q, &bars->tma_q, 0,
+                  b * L.box_rows, bh);
     for (int b = 0; b < L.n_box; ++b) {
       const uint32_t off = (uint32_t)b * L.box_rows * kRowBytes;
-      tma_load_3d(sQ + off, &map_q, &bars->tma, 0, b * L.box_rows, bh);
-      tma_load_3d(sK + off, &map_k, &bars->tma, 0, b * L.box_rows, bh);
-      tma_load_3d(sV + off, &map_v, &bars->tma, 0, b * L.box_rows, bh);
+      tma_load_3d(sK + off, &map_k, &bars->tma_kv, 0, b * L.box_rows, bh);
+      tma_load_3d(sV + off, &map_v, &bars->tma_kv, 0, b * L.box_rows, bh);
     }
   }
   pdl_trigger();
-  bool ok = fused_wait(&bars->tma, 0, abort, true);
+  bool ok = fused_wait(&bars->tma_q, 0, abort, true);
 
   // ---- 1. pool: thread per (agent row of the 128-row tile, 8-channel group)
   for (int it = threadIdx.x; it < kFusedMaxAgents * 8; it += kFusedThreads) {
@@ -196,7 +202,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
     *reinterpret_cast<uint4*>(sA + a * kRowBytes + ((g ^ (a & 7)) << 4)) = o;
   }
   fence_proxy_async_smem();
-  __syncthreads();
+  ok = fused_wait(&bars->tma_kv, 0, abort, ok);
 
   // ---- 2. S1 = A K^T (M = 128 agents, N = npad keys)
   if (threadIdx.x == 0 && ok) {
@@ -286,6 +292,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
   tc_fence_after();
 
   float inv[2][2];
+#pragma unroll
   for (int t = 0; t < 2; ++t) {
     float m0 = 0.f, m1 = 0.f, s0 = 0.f, s1 = 0.f;
     if (t < n_qt) {
@@ -320,7 +327,9 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
   tc_fence_after();
 
   // epilogue: O / l2 -> bf16 -> swizzled staging tiles (over K and V) -> TMA
-  for (int t = 0; t < n_qt; ++t) {
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    if (t >= n_qt) break;
     uint8_t* stage = sO + t * kQTileBytes;
     for (int q = 0; q < 4; ++q) {
       float o[8];
@@ -350,12 +359,13 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
       for (int t = 0; t < n_qt; ++t) tma_store_3d(&map_o, sO + t * kQTileBytes, 0, t * kQTile, bh);
       tma_store_commit();
     }
-    tma_store_wait_all();
+    tma_store_wait_read();                 // the staging may be released once read
     if (!ok) {
       // a wait gave up: let the staged copies and any MMA still running end
       // (bounded) before the CTA releases its TMEM and exits
       atomicOr(&g_watchdog, 1u);
-      fused_drain_wait(&bars->tma, 0);
+      fused_drain_wait(&bars->tma_q, 0);
+      fused_drain_wait(&bars->tma_kv, 0);
     }
     mma_commit(&bars->drain);
     fused_drain_wait(&bars->drain, 0);
