@@ -175,9 +175,11 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     if (ok && a < k && g < groups) {
+      // adaptive bins [floor(i G / P), ceil((i + 1) G / P)) in 32-bit
+      // arithmetic (grid sides <= 256 here)
       const int py = a / pool_w, px = a - py * pool_w;
-      const int y0 = bin_start(py, grid_h, pool_h), y1 = bin_end(py, grid_h, pool_h);
-      const int x0 = bin_start(px, grid_w, pool_w), x1 = bin_end(px, grid_w, pool_w);
+      const int y0 = (py * grid_h) / pool_h, y1 = ((py + 1) * grid_h + pool_h - 1) / pool_h;
+      const int x0 = (px * grid_w) / pool_w, x1 = ((px + 1) * grid_w + pool_w - 1) / pool_w;
       for (int y = y0; y < y1; ++y)
         for (int x = x0; x < x1; ++x) {
           const int r = y * grid_w + x;
@@ -226,13 +228,16 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
   // ---- 3. softmax of the agent rows over the N keys; P1 over S1
   float l0 = 0.f, l1 = 0.f;
   {
+    // slabs whose 16 rows are all padding agents (>= k) skip the work: their
+    // U rows are never read
+    const bool run = ok && slab < k;
     float t0 = -INFINITY, t1 = -INFINITY;
-    if (ok) {
+    if (run) {
       bc_slab_max(lane_col, N, npad, j4, t0, t1);
       t0 = row4_max(t0) * c;
       t1 = row4_max(t1) * c;
     }
-    bc_slab_exp(lane_col, N, npad, j4, false, c, -t0, -t1, l0, l1, ok, bars->chunk);
+    bc_slab_exp(lane_col, N, npad, j4, false, c, -t0, -t1, l0, l1, run, bars->chunk);
     l0 = row4_sum(l0);
     l1 = row4_sum(l1);
   }
@@ -253,25 +258,22 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
 
   // ---- 5. V_A = U / l1 -> bf16 rows of the MN-major operand (over K)
   {
-    const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-    for (int q = 0; q < 4; ++q) {            // 16-column blocks of the 64-column row
-      float u[8];
-      if (ok && q * 16 < dn) {
-        slab_ld16(lane_col + 128 + q * 16, u);
-      } else {
+    const float inv0 = r0 < k ? 1.f / l0 : 0.f, inv1 = r1 < k ? 1.f / l1 : 0.f;
+    float u[32];                             // the 64 columns [128, 192): U and beyond
+    if (ok && slab < k) {
+      slab_ld64(lane_col + 128, u);
+    } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) u[e] = 0.f;
-      }
+      for (int e = 0; e < 32; ++e) u[e] = 0.f;
+    }
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int ch = 2 * q + h;            // 8-column chunk
-        const bool live = ch < groups;
-        const uint32_t w0 = (live && r0 < k) ? pack_bf16x2(u[4 * h] * inv0, u[4 * h + 1] * inv0) : 0u;
-        const uint32_t w1 =
-            (live && r1 < k) ? pack_bf16x2(u[4 * h + 2] * inv1, u[4 * h + 3] * inv1) : 0u;
-        *reinterpret_cast<uint32_t*>(sVA + r0 * kRowBytes + ((ch ^ (r0 & 7)) << 4) + j4 * 4) = w0;
-        *reinterpret_cast<uint32_t*>(sVA + r1 * kRowBytes + ((ch ^ (r1 & 7)) << 4) + j4 * 4) = w1;
-      }
+    for (int ch = 0; ch < 8; ++ch) {         // 8-column chunk
+      const bool live = ch < groups;
+      const uint32_t w0 = (live && r0 < k) ? pack_bf16x2(u[4 * ch] * inv0, u[4 * ch + 1] * inv0) : 0u;
+      const uint32_t w1 =
+          (live && r1 < k) ? pack_bf16x2(u[4 * ch + 2] * inv1, u[4 * ch + 3] * inv1) : 0u;
+      *reinterpret_cast<uint32_t*>(sVA + r0 * kRowBytes + ((ch ^ (r0 & 7)) << 4) + j4 * 4) = w0;
+      *reinterpret_cast<uint32_t*>(sVA + r1 * kRowBytes + ((ch ^ (r1 & 7)) << 4) + j4 * 4) = w1;
     }
   }
   fence_proxy_async_smem();
@@ -296,13 +298,15 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
   for (int t = 0; t < 2; ++t) {
     float m0 = 0.f, m1 = 0.f, s0 = 0.f, s1 = 0.f;
     if (t < n_qt) {
+      // slabs whose rows are all past the slice's last query skip the work
+      const bool run = ok && t * kQTile + slab < N;
       float a0 = -INFINITY, a1 = -INFINITY;
-      if (ok) {
+      if (run) {
         bc_slab_max(lane_col + t * 128, k, kpad, j4, a0, a1);
         m0 = row4_max(a0) * c;
         m1 = row4_max(a1) * c;
       }
-      bc_slab_exp(lane_col + t * 128, k, kpad, j4, false, c, -m0, -m1, s0, s1, ok, bars->chunk);
+      bc_slab_exp(lane_col + t * 128, k, kpad, j4, false, c, -m0, -m1, s0, s1, run, bars->chunk);
       s0 = row4_sum(s0);
       s1 = row4_sum(s1);
     }
@@ -331,23 +335,20 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
   for (int t = 0; t < 2; ++t) {
     if (t >= n_qt) break;
     uint8_t* stage = sO + t * kQTileBytes;
-    for (int q = 0; q < 4; ++q) {
-      float o[8];
-      if (ok && q * 16 < dn) {
-        slab_ld16(lane_col + t * 128 + 64 + q * 16, o);
-      } else {
+    float o[32];                             // the 64 columns [128 t + 64, 128 t + 128): O_t
+    if (ok && t * kQTile + slab < N) {
+      slab_ld64(lane_col + t * 128 + 64, o);
+    } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = 0.f;
-      }
+      for (int e = 0; e < 32; ++e) o[e] = 0.f;
+    }
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int ch = 2 * q + h;
-        if (ch < groups) {
-          *reinterpret_cast<uint32_t*>(stage + r0 * kRowBytes + ((ch ^ (r0 & 7)) << 4) + j4 * 4) =
-              pack_bf16x2(o[4 * h] * inv[t][0], o[4 * h + 1] * inv[t][0]);
-          *reinterpret_cast<uint32_t*>(stage + r1 * kRowBytes + ((ch ^ (r1 & 7)) << 4) + j4 * 4) =
-              pack_bf16x2(o[4 * h + 2] * inv[t][1], o[4 * h + 3] * inv[t][1]);
-        }
+    for (int ch = 0; ch < 8; ++ch) {
+      if (ch < groups) {
+        *reinterpret_cast<uint32_t*>(stage + r0 * kRowBytes + ((ch ^ (r0 & 7)) << 4) + j4 * 4) =
+            pack_bf16x2(o[4 * ch] * inv[t][0], o[4 * ch + 1] * inv[t][0]);
+        *reinterpret_cast<uint32_t*>(stage + r1 * kRowBytes + ((ch ^ (r1 & 7)) << 4) + j4 * 4) =
+            pack_bf16x2(o[4 * ch + 2] * inv[t][1], o[4 * ch + 3] * inv[t][1]);
       }
     }
   }
