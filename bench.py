@@ -115,9 +115,11 @@ class ClockSampler:
                 "samples": len(self.samples), "reasons": sorted(self.reasons)}
 
 
-# Sources of the kernels the roofline reports (aggregation, merge, broadcast);
+# Sources of the kernels the roofline reports (aggregation, merge, broadcast,
+# fused small-slice pass);
 # a recorded DRAM-traffic figure applies only while these hash the same.
-ROOFLINE_SOURCES = ("common.cuh", "tc_primitives.cuh", "kernels_tc.cuh", "kernels_merge.cuh")
+ROOFLINE_SOURCES = ("common.cuh", "tc_primitives.cuh", "kernels_tc.cuh", "kernels_merge.cuh",
+                    "kernels_fused.cuh")
 
 
 def kernel_source_sha():
