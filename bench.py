@@ -115,17 +115,20 @@ class ClockSampler:
                 "samples": len(self.samples), "reasons": sorted(self.reasons)}
 
 
-# Sources of the kernels the roofline reports (aggregation, merge, broadcast,
-# fused small-slice pass);
-# a recorded DRAM-traffic figure applies only while these hash the same.
-ROOFLINE_SOURCES = ("common.cuh", "tc_primitives.cuh", "kernels_tc.cuh", "kernels_merge.cuh",
-                    "kernels_fused.cuh")
+# Sources of each kernel the roofline reports; a recorded DRAM-traffic figure
+# applies only while its kernel's sources hash the same.
+_TC_COMMON = ("common.cuh", "tc_primitives.cuh", "kernels_tc.cuh")
+ROOFLINE_SOURCES = {
+    "agent_aggregate+agent_merge": _TC_COMMON + ("kernels_merge.cuh",),
+    "agent_broadcast": _TC_COMMON,
+    "agent_fused_small": _TC_COMMON + ("kernels_fused.cuh",),
+}
 
 
-def kernel_source_sha():
+def kernel_source_sha(kernel: str):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "efficient_vision_attention_b200", "csrc")
-    for name in ROOFLINE_SOURCES:
+    for name in ROOFLINE_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -133,16 +136,18 @@ def kernel_source_sha():
 
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources."""
+    the kernel's current sources."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except Exception:
         return None
+    if kernel not in ROOFLINE_SOURCES:
+        return None
     for r in rec.get("records", []):
         if (r.get("kernel") == kernel and r.get("workload") == workload
-                and r.get("source_sha") == kernel_source_sha()):
+                and r.get("source_sha") == kernel_source_sha(kernel)):
             return r.get("dram_bytes_per_launch")
     return None
 

@@ -35,8 +35,28 @@ def test_sfu_roofline_of_the_sd_latent_broadcast(bench):
     assert r["exps_per_launch"] == n_exp
 
 
-def test_traffic_record_applies_only_to_the_recorded_sources(bench):
-    sha = bench.kernel_source_sha()
-    assert len(sha) == 16
-    rec = bench.recorded_traffic("agent_broadcast", "no_such_workload")
-    assert rec is None
+def test_traffic_record_applies_only_to_the_recorded_sources(bench, tmp_path, monkeypatch):
+    shas = {k: bench.kernel_source_sha(k) for k in bench.ROOFLINE_SOURCES}
+    assert all(len(v) == 16 for v in shas.values())
+    # the broadcast's sources are a subset of the others': different hashes
+    assert len(set(shas.values())) == len(shas)
+    assert bench.recorded_traffic("agent_broadcast", "no_such_workload") is None
+    assert bench.recorded_traffic("no_such_kernel", "sd_latent_1024") is None
+    # a record applies only while its kernel's sources hash the same
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    import json
+    recs = {"records": [
+        {"kernel": "agent_broadcast", "workload": "w", "source_sha": shas["agent_broadcast"],
+         "dram_bytes_per_launch": 123},
+        {"kernel": "agent_fused_small", "workload": "w", "source_sha": "0" * 16,
+         "dram_bytes_per_launch": 456}]}
+    (prof / "ncu_traffic.json").write_text(json.dumps(recs))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    csrc = tmp_path / "efficient_vision_attention_b200" / "csrc"
+    csrc.parent.mkdir()
+    import shutil, os
+    shutil.copytree(os.path.join(os.path.dirname(os.path.dirname(__file__)),
+                                 "efficient_vision_attention_b200", "csrc"), csrc)
+    assert bench.recorded_traffic("agent_broadcast", "w") == 123
+    assert bench.recorded_traffic("agent_fused_small", "w") is None
