@@ -172,11 +172,12 @@ __global__ void __launch_bounds__(kPoolTmaThreads) agent_pool_tma_kernel(
 // When the bins tile the grid exactly (grid_h = R pool_h, grid_w = W pool_w)
 // every agent averages an R x W block, and a CTA takes one band of R grid
 // rows and a chunk of token columns of one slice: a thread per (token column,
-// 8-channel group) issues the R 16-byte loads of its column at once (all in
-// flight, straight into registers, no staging), sums them in fp32 into a
+// 8-channel group) issues the R 16-byte loads of its column 16 at a time (in
+// flight together, straight into registers, no staging), sums them in fp32 into a
 // shared column sum, and a thread per (agent, 8-channel group) then adds the
 // W columns of its bin and divides by R W.
-constexpr int kPoolBandMaxRows = 16;
+constexpr int kPoolBandBatch = 16;      // rows of a column whose loads are in flight together
+constexpr int kPoolBandMaxRows = 64;
 
 struct PoolBandPlan {
   int rows, bin_w, chunk_cols, threads;
@@ -228,22 +229,46 @@ __global__ void agent_pool_band_kernel(const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* src =
         q + (bh * (long long)N + (long long)py * rows * grid_w + xs + x) * d + g * 8;
     const long long row_step = (long long)grid_w * d;
-    uint4 raw[kPoolBandMaxRows];
-#pragma unroll
-    for (int r = 0; r < kPoolBandMaxRows; ++r)
-      if (r < rows) raw[r] = __ldcs(reinterpret_cast<const uint4*>(src + r * row_step));
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    if (rows <= kPoolBandBatch) {
+      // bins of up to 16 rows: every load of the column in flight at once
+      uint4 raw[kPoolBandBatch];
 #pragma unroll
-    for (int r = 0; r < kPoolBandMaxRows; ++r) {
-      if (r < rows) {
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[r]);
+      for (int r = 0; r < kPoolBandBatch; ++r)
+        if (r < rows) raw[r] = __ldcs(reinterpret_cast<const uint4*>(src + r * row_step));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(h[i]);
-          acc[2 * i] += f.x;
-          acc[2 * i + 1] += f.y;
+      for (int r = 0; r < kPoolBandBatch; ++r) {
+        if (r < rows) {
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[r]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h[i]);
+            acc[2 * i] += f.x;
+            acc[2 * i + 1] += f.y;
+          }
+        }
+      }
+    } else {
+      // taller bins: 16 rows' loads in flight at a time
+      for (int rb = 0; rb < rows; rb += kPoolBandBatch) {
+        uint4 raw[kPoolBandBatch];
+#pragma unroll
+        for (int r = 0; r < kPoolBandBatch; ++r)
+          if (rb + r < rows)
+            raw[r] = __ldcs(reinterpret_cast<const uint4*>(src + (rb + r) * row_step));
+#pragma unroll
+        for (int r = 0; r < kPoolBandBatch; ++r) {
+          if (rb + r < rows) {
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[r]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __bfloat1622float2(h[i]);
+              acc[2 * i] += f.x;
+              acc[2 * i + 1] += f.y;
+            }
+          }
         }
       }
     }

@@ -114,10 +114,12 @@ def test_stage_pool(dtype):
 
 
 @pytest.mark.parametrize("gh,gw,ph,pw,d", [(128, 128, 16, 16, 40), (256, 256, 16, 16, 64),
-                                         (14, 14, 7, 7, 64), (48, 96, 3, 32, 8)])
+                                         (14, 14, 7, 7, 64), (48, 96, 3, 32, 8),
+                                         (256, 256, 8, 8, 64), (120, 40, 2, 5, 16)])
 def test_stage_pool_uniform_bins(gh, gw, ph, pw, d):
     """Grids that the bins divide exactly (the band kernel for bf16): the SD
-    latent, high-res, DeiT shapes and one with 16x3-token bins and d = 8."""
+    latent, high-res (16- and 32-row bins), DeiT shapes, one with 16x3-token
+    bins and d = 8 and one with 60-row bins (four batches of row loads)."""
     B, H = 2, 3
     q, _, _ = random_qkv((B, H, gh * gw, d), seed=gh + pw + d, dtype=torch.bfloat16)
     a32 = torch.empty((B, H, ph * pw, d), dtype=torch.float32, device="cuda")
