@@ -470,6 +470,50 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int gw = p.bias.grid_w;
             const int ty0 = n0 / gw, tx0 = n0 - ty0 * gw;
             const bool pairs = (gw & 1) == 0 && (reinterpret_cast<uintptr_t>(p.bias.col) & 7u) == 0;
+            if (pairs && tx0 + kKeyTile <= gw) {
+              // the whole tile lies in grid row ty0: each agent row's row term
+              // and cell row are loaded once; a pair's block term once when
+              // both of its tokens fall in the same cell
+              const int cyo = (int)cell_y[ty0] * p.bias.pool_w;
+              const float rw0 = (in0 && br0.row) ? __ldg(br0.row + ty0) : 0.f;
+              const float rw1 = (in1 && br1.row) ? __ldg(br1.row + ty0) : 0.f;
+#pragma unroll
+              for (int g8 = 0; g8 < 8; ++g8) {
+                const int col = 8 * g8 + 2 * j4;
+                if (col >= valid) continue;
+                const int x = tx0 + col;
+                float2 b0 = make_float2(rw0, rw0), b1 = make_float2(rw1, rw1);
+                if (p.bias.col) {
+                  if (in0) {
+                    const float2 t0 = __ldg(reinterpret_cast<const float2*>(br0.col + x));
+                    b0.x += t0.x;
+                    b0.y += t0.y;
+                  }
+                  if (in1) {
+                    const float2 t1 = __ldg(reinterpret_cast<const float2*>(br1.col + x));
+                    b1.x += t1.x;
+                    b1.y += t1.y;
+                  }
+                }
+                if (p.bias.block) {
+                  const int c0 = cyo + cell_x[x], c1 = cyo + cell_x[x + 1];
+                  if (in0) {
+                    const float k0 = __ldg(br0.block + c0);
+                    b0.x += k0;
+                    b0.y += (c1 == c0) ? k0 : __ldg(br0.block + c1);
+                  }
+                  if (in1) {
+                    const float k1 = __ldg(br1.block + c0);
+                    b1.x += k1;
+                    b1.y += (c1 == c0) ? k1 : __ldg(br1.block + c1);
+                  }
+                }
+                v[4 * g8] = fmaf(v[4 * g8], p.c, b0.x * kLog2e);
+                v[4 * g8 + 1] = fmaf(v[4 * g8 + 1], p.c, b0.y * kLog2e);
+                v[4 * g8 + 2] = fmaf(v[4 * g8 + 2], p.c, b1.x * kLog2e);
+                v[4 * g8 + 3] = fmaf(v[4 * g8 + 3], p.c, b1.y * kLog2e);
+              }
+            } else
 #pragma unroll
             for (int g8 = 0; g8 < 8; ++g8) {
               const int col = 8 * g8 + 2 * j4;
