@@ -677,6 +677,63 @@ __global__ void expand_agents_f32_kernel(const T* __restrict__ ag, float* __rest
   out[e] = to_f32(ag[(bh % H) * kd + r]);
 }
 
+// Steps 3-5 of the backward pass, given the fp32 agents, V_A and each agent
+// row's softmax max and sum: the broadcast-stage gradients, the
+// aggregation-stage gradients, then dQ with the pooling adjoint and the
+// agents' own gradient.
+template <typename T>
+int backward_gradients(const Problem& p, const void* q, const void* k, const void* v,
+                       const void* agents, const void* dout, void* dq, void* dk, void* dv,
+                       float* dagents, float* a32, float* va32, float* ml, float* dva, float* da,
+                       float* dqa, cudaStream_t st) {
+  const long long BH = p.BH();
+  const size_t kd = (size_t)p.k * p.d;
+  const size_t nd = (size_t)p.N * p.d;
+  int r = AA_OK;
+  // 3. broadcast-stage gradients
+  AA_CUDA(cudaMemsetAsync(dva, 0, BH * kd * 4, st));
+  AA_CUDA(cudaMemsetAsync(da, 0, BH * kd * 4, st));
+  BwdArgs g;
+  memset(&g, 0, sizeof(g));
+  g.x = q;
+  g.y = dout;
+  g.a = a32;
+  g.va = va32;
+  g.dq = dqa;
+  g.dva_acc = dva;
+  g.da_acc = da;
+  g.N = p.N;
+  g.n_agents = p.k;
+  g.d = p.d;
+  g.scale = p.scale;
+  g.scale_log2 = p.scale * kLog2e;
+  const size_t smem_b = bwd_smem_bytes(p.d);
+  const dim3 grid_b((unsigned)((p.N + kBwdRows - 1) / kBwdRows), (unsigned)BH);
+  r = ensure_smem(bwd_query_kernel<T>, smem_b, sizeof(T) == 4 ? g_bwd_q_f32 : g_bwd_q_bf16);
+  if (r != AA_OK) return r;
+  bwd_query_kernel<T><<<grid_b, kBwdThreads, smem_b, st>>>(g);
+  AA_CUDA(cudaGetLastError());
+  // 4. aggregation-stage gradients
+  g.x = k;
+  g.y = v;
+  g.dva = dva;
+  g.ml = ml;
+  g.dk = dk;
+  g.dv = dv;
+  r = ensure_smem(bwd_key_kernel<T>, smem_b, sizeof(T) == 4 ? g_bwd_k_f32 : g_bwd_k_bf16);
+  if (r != AA_OK) return r;
+  bwd_key_kernel<T><<<grid_b, kBwdThreads, smem_b, st>>>(g);
+  AA_CUDA(cudaGetLastError());
+  // 5. dQ (+ pooling adjoint) in the run dtype; the agents' own gradient
+  const dim3 grid_f((unsigned)(((long long)nd + 255) / 256), (unsigned)BH);
+  bwd_finish_kernel<T><<<grid_f, 256, 0, st>>>(dqa, da, static_cast<T*>(dq), p.N, p.d, p.grid_h,
+                                               p.grid_w, p.pool_h, p.pool_w,
+                                               agents == nullptr ? 1 : 0);
+  AA_CUDA(cudaGetLastError());
+  if (dagents) AA_CUDA(cudaMemcpyAsync(dagents, da, BH * kd * 4, cudaMemcpyDeviceToDevice, st));
+  return AA_OK;
+}
+
 template <typename T>
 int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
                   const void* agents, const void* dout, void* dq, void* dk, void* dv,
@@ -684,8 +741,16 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
   int sms = 0;
   int rc = device_sm_count(&sms);
   if (rc != AA_OK) return rc;
+  // bf16 with d <= 64: the forward statistics are recomputed on the tensor
+  // cores from the bf16 agents the forward pass uses, and the gradient
+  // kernels take the same bf16 agents widened to fp32, so the saved maxima
+  // and sums match the scores they recompute; otherwise the SIMT aggregation
+  // with fp32 agents.
+  const bool tc_recompute = sizeof(T) == 2 && tc_supported(p.d, p.k);
+  Problem pp = p;
+  pp.force_simt = !tc_recompute;
   Scratch s;
-  plan_scratch(p, sms, &s);            // p.force_simt: SIMT aggregation plan
+  plan_scratch(pp, sms, &s);
   const long long BH = p.BH();
   const size_t kd = (size_t)p.k * p.d;
   const size_t nd = (size_t)p.N * p.d;
@@ -707,13 +772,42 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
   float* da = reinterpret_cast<float*>(ws + da_off);
   float* dqa = reinterpret_cast<float*>(ws + dq_off);
   auto run = [&]() -> int {
+    const long long n_ag = BH * (long long)kd;
+    if (tc_recompute) {
+      // 1. bf16 agents (pooled, or the given ones) and their fp32 widening
+      const void* ag = agents;
+      long long ag_bstride = 0;
+      if (agents == nullptr) {
+        T* a_low = reinterpret_cast<T*>(ws + s.a_off);
+        int r = launch_pool<T>(p, q, nullptr, a_low, st);
+        if (r != AA_OK) return r;
+        ag = a_low;
+        ag_bstride = (long long)kd * p.H;
+        expand_agents_f32_kernel<T><<<(unsigned)((n_ag + 255) / 256), 256, 0, st>>>(
+            a_low, a32, BH, (int)BH, (long long)kd);
+      } else {
+        expand_agents_f32_kernel<T><<<(unsigned)((n_ag + 255) / 256), 256, 0, st>>>(
+            static_cast<const T*>(agents), a32, BH, p.H, (long long)kd);
+      }
+      AA_CUDA(cudaGetLastError());
+      // 2. forward aggregation on the tensor cores: V_A (fp32) and each agent
+      // row's max and sum from the merge
+      cudaError_t e = tc_launch_aggregate(ag, ag_bstride, (long long)kd, k, v, p.B, p.H, p.N, p.d,
+                                          p.k, p.scale * kLog2e, s.plan,
+                                          reinterpret_cast<float*>(ws + s.pu_off),
+                                          reinterpret_cast<float*>(ws + s.pml_off), st, false);
+      if (e != cudaSuccess) return cuda_fail(e, "agent_aggregate (backward recompute) launch");
+      int r = launch_merge<T>(pp, s, ws, va32, nullptr, st, false, ml);
+      if (r != AA_OK) return r;
+      return backward_gradients<T>(p, q, k, v, agents, dout, dq, dk, dv, dagents, a32, va32, ml,
+                                   dva, da, dqa, st);
+    }
     // 1. fp32 agents
     if (agents == nullptr) {
       int r = launch_pool<T>(p, q, a32, nullptr, st);
       if (r != AA_OK) return r;
     } else {
-      const long long n = BH * (long long)kd;
-      expand_agents_f32_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+      expand_agents_f32_kernel<T><<<(unsigned)((n_ag + 255) / 256), 256, 0, st>>>(
           static_cast<const T*>(agents), a32, BH, p.H, (long long)kd);
       AA_CUDA(cudaGetLastError());
     }
@@ -749,50 +843,10 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
     if (blocks > 0x7fffffffLL) return AA_ERR_SHAPE;
     AA_CUDA(launch_kernel(simt_attend_kernel<T, float>, dim3((unsigned)blocks), dim3(kSimtThreads),
                           smem_a, st, false, a));
-    r = launch_merge<T>(p, s, ws, va32, nullptr, st, false, ml);
+    r = launch_merge<T>(pp, s, ws, va32, nullptr, st, false, ml);
     if (r != AA_OK) return r;
-    // 3. broadcast-stage gradients
-    AA_CUDA(cudaMemsetAsync(dva, 0, BH * kd * 4, st));
-    AA_CUDA(cudaMemsetAsync(da, 0, BH * kd * 4, st));
-    BwdArgs g;
-    memset(&g, 0, sizeof(g));
-    g.x = q;
-    g.y = dout;
-    g.a = a32;
-    g.va = va32;
-    g.dq = dqa;
-    g.dva_acc = dva;
-    g.da_acc = da;
-    g.N = p.N;
-    g.n_agents = p.k;
-    g.d = p.d;
-    g.scale = p.scale;
-    g.scale_log2 = p.scale * kLog2e;
-    const size_t smem_b = bwd_smem_bytes(p.d);
-    const dim3 grid_b((unsigned)((p.N + kBwdRows - 1) / kBwdRows), (unsigned)BH);
-    r = ensure_smem(bwd_query_kernel<T>, smem_b, sizeof(T) == 4 ? g_bwd_q_f32 : g_bwd_q_bf16);
-    if (r != AA_OK) return r;
-    bwd_query_kernel<T><<<grid_b, kBwdThreads, smem_b, st>>>(g);
-    AA_CUDA(cudaGetLastError());
-    // 4. aggregation-stage gradients
-    g.x = k;
-    g.y = v;
-    g.dva = dva;
-    g.ml = ml;
-    g.dk = dk;
-    g.dv = dv;
-    r = ensure_smem(bwd_key_kernel<T>, smem_b, sizeof(T) == 4 ? g_bwd_k_f32 : g_bwd_k_bf16);
-    if (r != AA_OK) return r;
-    bwd_key_kernel<T><<<grid_b, kBwdThreads, smem_b, st>>>(g);
-    AA_CUDA(cudaGetLastError());
-    // 5. dQ (+ pooling adjoint) in the run dtype; the agents' own gradient
-    const dim3 grid_f((unsigned)(((long long)nd + 255) / 256), (unsigned)BH);
-    bwd_finish_kernel<T><<<grid_f, 256, 0, st>>>(dqa, da, static_cast<T*>(dq), p.N, p.d, p.grid_h,
-                                                 p.grid_w, p.pool_h, p.pool_w,
-                                                 agents == nullptr ? 1 : 0);
-    AA_CUDA(cudaGetLastError());
-    if (dagents) AA_CUDA(cudaMemcpyAsync(dagents, da, BH * kd * 4, cudaMemcpyDeviceToDevice, st));
-    return AA_OK;
+    return backward_gradients<T>(p, q, k, v, agents, dout, dq, dk, dv, dagents, a32, va32, ml,
+                                 dva, da, dqa, st);
   };
   rc = run();
   cudaError_t e = cudaFreeAsync(ws, st);
