@@ -45,8 +45,13 @@ struct BwdArgs {
   float scale_log2;     // s * log2 e
 };
 
+// Row stride of the staged [rows][d] tiles: d + 4 floats, so every row starts
+// on a 16-byte boundary (float4 reads along the channels) and consecutive
+// rows start 4 banks apart.
+__host__ __device__ __forceinline__ int bwd_row_stride(int d) { return d + 4; }
+
 __host__ __forceinline__ size_t bwd_smem_bytes(int d) {
-  const size_t dp = d + 1;
+  const size_t dp = bwd_row_stride(d);
   return sizeof(float) * (2 * kBwdRows * dp + 2 * kBwdCols * dp + 2 * kBwdRows * (kBwdCols + 1) +
                           (size_t)kBwdRows * d * 2 + 4 * kBwdRows + 2 * kBwdCols);
 }
@@ -69,30 +74,37 @@ __device__ __forceinline__ void bwd_load_agents(float* dst, const float* src, in
 }
 
 // dot products of the CTA's rows with a chunk's agents: out[r][j] = X_r . Y_j * mul.
-// Register-tiled: thread t owns rows 2(t/8), 2(t/8)+1 and columns 4(t%8) .. +3
-// (256 threads x 8 dots = 64 x 32), reading 6 shared values per 8 FMAs.
+// Register-tiled: thread t owns rows 2(t/8), 2(t/8)+1 and agents t%8 + 8q,
+// q = 0..3 (256 threads x 8 dots = 64 x 32); per 4 channels it reads 6 float4
+// (rows 16-byte aligned, d % 4 == 0) for 32 FMAs.  The 8 threads of a
+// quarter-warp read 8 consecutive agent rows d + 4 floats apart: 8 distinct
+// 4-bank groups (no conflict); their shared row is a broadcast.
+__device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc) {
+  return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
+}
 __device__ __forceinline__ void bwd_dots(float* out, const float* X, const float* Y, int d, int dp,
                                          float mul) {
   static_assert(kBwdRows * kBwdCols == kBwdThreads * 8, "2 x 4 dots per thread");
   const int t = threadIdx.x;
-  const int r = 2 * (t >> 3), j = 4 * (t & 7);
+  const int r = 2 * (t >> 3), j = t & 7;
   const float* x0 = X + r * dp;
   const float* x1 = x0 + dp;
   const float* y0 = Y + j * dp;
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  for (int c = 0; c < d; ++c) {
-    const float a0 = x0[c], a1 = x1[c];
+  for (int c = 0; c < d; c += 4) {
+    const float4 a0 = *reinterpret_cast<const float4*>(x0 + c);
+    const float4 a1 = *reinterpret_cast<const float4*>(x1 + c);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float bq = y0[q * dp + c];
-      acc[0][q] = fmaf(a0, bq, acc[0][q]);
-      acc[1][q] = fmaf(a1, bq, acc[1][q]);
+      const float4 bq = *reinterpret_cast<const float4*>(y0 + 8 * q * dp + c);
+      acc[0][q] = dot4(a0, bq, acc[0][q]);
+      acc[1][q] = dot4(a1, bq, acc[1][q]);
     }
   }
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    out[r * (kBwdCols + 1) + j + q] = acc[0][q] * mul;
-    out[(r + 1) * (kBwdCols + 1) + j + q] = acc[1][q] * mul;
+    out[r * (kBwdCols + 1) + j + 8 * q] = acc[0][q] * mul;
+    out[(r + 1) * (kBwdCols + 1) + j + 8 * q] = acc[1][q] * mul;
   }
 }
 
@@ -107,11 +119,12 @@ __device__ __forceinline__ void bwd_rows_acc(float* out, const float* W, const f
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j < valid; ++j) {
       const float w0 = W[r * (kBwdCols + 1) + j], w1 = W[(r + 1) * (kBwdCols + 1) + j];
+      const float4 m4 = *reinterpret_cast<const float4*>(M + j * dp + c);   // d % 4 == 0
+      const float m[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float m = (c + q < d) ? M[j * dp + c + q] : 0.f;
-        a0[q] = fmaf(w0, m, a0[q]);
-        a1[q] = fmaf(w1, m, a1[q]);
+        a0[q] = fmaf(w0, m[q], a0[q]);
+        a1[q] = fmaf(w1, m[q], a1[q]);
       }
     }
 #pragma unroll
@@ -136,11 +149,12 @@ __device__ __forceinline__ void bwd_agents_acc(float* dst, int j0, const float* 
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
     for (int r = 0; r < kBwdRows; ++r) {
       const float w0 = W[r * (kBwdCols + 1) + j], w1 = W[r * (kBwdCols + 1) + j + 1];
+      const float4 x4 = *reinterpret_cast<const float4*>(X + r * dp + c);   // d % 4 == 0
+      const float x[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float x = (c + q < d) ? X[r * dp + c + q] : 0.f;
-        a0[q] = fmaf(w0, x, a0[q]);
-        a1[q] = fmaf(w1, x, a1[q]);
+        a0[q] = fmaf(w0, x[q], a0[q]);
+        a1[q] = fmaf(w1, x[q], a1[q]);
       }
     }
 #pragma unroll
@@ -156,10 +170,10 @@ __device__ __forceinline__ void bwd_agents_acc(float* dst, int j0, const float* 
 template <typename T>
 __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
   extern __shared__ float sm[];
-  const int d = p.d, dp = d + 1;
-  float* s_x = sm;                                   // Q rows [64][d+1]
+  const int d = p.d, dp = bwd_row_stride(d);
+  float* s_x = sm;                                   // Q rows [64][d+4]
   float* s_y = s_x + kBwdRows * dp;                  // dO rows
-  float* s_a = s_y + kBwdRows * dp;                  // agent chunk [32][d+1]
+  float* s_a = s_y + kBwdRows * dp;                  // agent chunk [32][d+4]
   float* s_va = s_a + kBwdCols * dp;
   float* s_t = s_va + kBwdCols * dp;                 // scores / P2 [64][33]
   float* s_g = s_t + kBwdRows * (kBwdCols + 1);      // dP2 / dS2 [64][33]
@@ -185,30 +199,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
     s_D[r] = 0.f;
   }
   __syncthreads();
-  // pass 1: row max and sum of the scores over all agents (online, per chunk)
-  for (int j0 = 0; j0 < K; j0 += kBwdCols) {
-    const int valid = min(kBwdCols, K - j0);
-    bwd_load_agents(s_a, A, j0, K, d, dp);
-    __syncthreads();
-    bwd_dots(s_t, s_x, s_a, d, dp, p.scale_log2);
-    __syncthreads();
-    for (int r = warp; r < kBwdRows; r += kBwdThreads / 32) {
-      const float t = lane < valid ? s_t[r * (kBwdCols + 1) + lane] : -INFINITY;
-      float mx = t;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float m_new = fmaxf(s_m[r], mx);
-      float e = lane < valid ? exp2f(t - m_new) : 0.f;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-      if (lane == 0) {
-        s_l[r] = s_l[r] * exp2f(s_m[r] - m_new) + e;
-        s_m[r] = m_new;
-      }
-    }
-    __syncthreads();
-  }
-  // pass 2: D_i = sum_j P2_ij (dO_i . V_A_j)
+  // pass 1 (online over the chunks): each row's score max m and sum
+  // l = sum_j 2^(s_j - m), and D~ = sum_j 2^(s_j - m) (dO . V_A_j), both
+  // rescaled when m grows; D_i = D~ / l
   for (int j0 = 0; j0 < K; j0 += kBwdCols) {
     const int valid = min(kBwdCols, K - j0);
     bwd_load_agents(s_a, A, j0, K, d, dp);
@@ -218,16 +211,30 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
     bwd_dots(s_g, s_y, s_va, d, dp, 1.f);
     __syncthreads();
     for (int r = warp; r < kBwdRows; r += kBwdThreads / 32) {
-      float v = 0.f;
-      if (lane < valid)
-        v = exp2f(s_t[r * (kBwdCols + 1) + lane] - s_m[r]) / s_l[r] * s_g[r * (kBwdCols + 1) + lane];
+      const float t = lane < valid ? s_t[r * (kBwdCols + 1) + lane] : -INFINITY;
+      float mx = t;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) s_D[r] += v;
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float m_new = fmaxf(s_m[r], mx);
+      float e = lane < valid ? exp2f(t - m_new) : 0.f;
+      float eg = lane < valid ? e * s_g[r * (kBwdCols + 1) + lane] : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        e += __shfl_xor_sync(0xffffffffu, e, o);
+        eg += __shfl_xor_sync(0xffffffffu, eg, o);
+      }
+      if (lane == 0) {
+        const float rs = exp2f(s_m[r] - m_new);   // 0 on the first chunk (s_m = -inf)
+        s_l[r] = s_l[r] * rs + e;
+        s_D[r] = s_D[r] * rs + eg;
+        s_m[r] = m_new;
+      }
     }
     __syncthreads();
   }
-  // pass 3: dS2, dQ, and the chunk's contributions to dV_A and dA
+  for (int r = tid; r < kBwdRows; r += kBwdThreads) s_D[r] = s_D[r] / s_l[r];
+  __syncthreads();
+  // pass 2: dS2, dQ, and the chunk's contributions to dV_A and dA
   float* dva = p.dva_acc + bh * (long long)K * d;
   float* da = p.da_acc + bh * (long long)K * d;
   for (int j0 = 0; j0 < K; j0 += kBwdCols) {
@@ -265,7 +272,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
 template <typename T>
 __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
   extern __shared__ float sm[];
-  const int d = p.d, dp = d + 1;
+  const int d = p.d, dp = bwd_row_stride(d);
   float* s_x = sm;                                   // K rows
   float* s_y = s_x + kBwdRows * dp;                  // V rows
   float* s_a = s_y + kBwdRows * dp;                  // agent chunk
