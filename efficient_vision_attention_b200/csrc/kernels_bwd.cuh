@@ -137,6 +137,15 @@ __device__ __forceinline__ void bwd_rows_acc(float* out, const float* W, const f
   }
 }
 
+// Four consecutive floats added into global memory by one vector reduction
+// (16-byte aligned address): a quarter of the L2 atomic operations of four
+// scalar atomicAdds.
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float e) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(e)
+               : "memory");
+}
+
 // acc[j][c] = mul * sum_r W[r][j] X[r][c] for the chunk's agents j < valid,
 // added atomically into dst[(j0 + j) * d + c]: items = (agent pair, 4 channels).
 __device__ __forceinline__ void bwd_agents_acc(float* dst, int j0, const float* W, const float* X,
@@ -157,13 +166,12 @@ __device__ __forceinline__ void bwd_agents_acc(float* dst, int j0, const float* 
         a1[q] = fmaf(w1, x[q], a1[q]);
       }
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (c + q < d) {
-        atomicAdd(dst + (long long)(j0 + j) * d + c + q, mul * a0[q]);
-        if (j + 1 < valid) atomicAdd(dst + (long long)(j0 + j + 1) * d + c + q, mul * a1[q]);
-      }
-    }
+    // d % 4 == 0, so the 4 channels are in range and 16-byte aligned
+    red_add_v4(dst + (long long)(j0 + j) * d + c, mul * a0[0], mul * a0[1], mul * a0[2],
+               mul * a0[3]);
+    if (j + 1 < valid)
+      red_add_v4(dst + (long long)(j0 + j + 1) * d + c, mul * a1[0], mul * a1[1], mul * a1[2],
+                 mul * a1[3]);
   }
 }
 
