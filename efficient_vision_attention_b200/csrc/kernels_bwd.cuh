@@ -53,7 +53,7 @@ __host__ __device__ __forceinline__ int bwd_row_stride(int d) { return d + 4; }
 __host__ __forceinline__ size_t bwd_smem_bytes(int d) {
   const size_t dp = bwd_row_stride(d);
   return sizeof(float) * (2 * kBwdRows * dp + 2 * kBwdCols * dp + 2 * kBwdRows * (kBwdCols + 1) +
-                          (size_t)kBwdRows * d * 2 + 4 * kBwdRows + 2 * kBwdCols);
+                          (size_t)kBwdRows * dp * 2 + 4 * kBwdRows + 4 * kBwdCols);
 }
 
 template <typename T>
@@ -127,13 +127,14 @@ __device__ __forceinline__ void bwd_rows_acc(float* out, const float* W, const f
         a1[q] = fmaf(w1, m[q], a1[q]);
       }
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (c + q < d) {
-        out[r * d + c + q] += mul * a0[q];
-        out[(r + 1) * d + c + q] += mul * a1[q];
-      }
-    }
+    // out rows dp floats apart (16-byte aligned): one float4 update per row
+    float4* o0 = reinterpret_cast<float4*>(out + r * dp + c);
+    float4* o1 = reinterpret_cast<float4*>(out + (r + 1) * dp + c);
+    float4 u0 = *o0, u1 = *o1;
+    u0.x += mul * a0[0]; u0.y += mul * a0[1]; u0.z += mul * a0[2]; u0.w += mul * a0[3];
+    u1.x += mul * a1[0]; u1.y += mul * a1[1]; u1.z += mul * a1[2]; u1.w += mul * a1[3];
+    *o0 = u0;
+    *o1 = u1;
   }
 }
 
@@ -185,9 +186,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
   float* s_va = s_a + kBwdCols * dp;
   float* s_t = s_va + kBwdCols * dp;                 // scores / P2 [64][33]
   float* s_g = s_t + kBwdRows * (kBwdCols + 1);      // dP2 / dS2 [64][33]
-  float* s_acc = s_g + kBwdRows * (kBwdCols + 1);    // dQ accumulator [64][d]
-  float* s_red = s_acc + kBwdRows * d;               // chunk reductions [64][d] (2 x 32 x d)
-  float* s_m = s_red + kBwdRows * d;
+  float* s_acc = s_g + kBwdRows * (kBwdCols + 1);    // dQ accumulator [64][d+4]
+  float* s_m = s_acc + kBwdRows * dp;
   float* s_l = s_m + kBwdRows;
   float* s_D = s_l + kBwdRows;
   const long long bh = blockIdx.y;
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   bwd_load_rows(s_x, X, r0, n_rows, d, dp);
   bwd_load_rows(s_y, Y, r0, n_rows, d, dp);
-  for (int e = tid; e < kBwdRows * d; e += kBwdThreads) s_acc[e] = 0.f;
+  for (int e = tid; e < kBwdRows * dp; e += kBwdThreads) s_acc[e] = 0.f;
   for (int r = tid; r < kBwdRows; r += kBwdThreads) {
     s_m[r] = -INFINITY;
     s_l[r] = 0.f;
@@ -272,9 +272,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
   float* dq = p.dq + bh * (long long)p.N * d;
   for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {
     const int r = e / d, c = e - r * d;
-    if (r0 + r < n_rows) dq[(long long)(r0 + r) * d + c] = s_acc[e];
+    if (r0 + r < n_rows) dq[(long long)(r0 + r) * d + c] = s_acc[r * dp + c];
   }
-  (void)s_red;
 }
 
 template <typename T>
@@ -287,9 +286,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
   float* s_dva = s_a + kBwdCols * dp;                // dV_A chunk
   float* s_t = s_dva + kBwdCols * dp;                // P1 [64][33]
   float* s_g = s_t + kBwdRows * (kBwdCols + 1);      // dS1 [64][33]
-  float* s_dk = s_g + kBwdRows * (kBwdCols + 1);     // [64][d]
-  float* s_dv = s_dk + kBwdRows * d;                 // [64][d]
-  float* s_jm = s_dv + kBwdRows * d;                 // chunk: row max, sum, E (3 x 32)
+  float* s_dk = s_g + kBwdRows * (kBwdCols + 1);     // [64][d+4]
+  float* s_dv = s_dk + kBwdRows * dp;                // [64][d+4]
+  float* s_jm = s_dv + kBwdRows * dp;                // chunk: row max, sum, E (3 x 32)
   float* s_jl = s_jm + kBwdCols;
   float* s_je = s_jl + kBwdCols;
   const long long bh = blockIdx.y;
@@ -305,7 +304,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   bwd_load_rows(s_x, X, r0, n_rows, d, dp);
   bwd_load_rows(s_y, Y, r0, n_rows, d, dp);
-  for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {
+  for (int e = tid; e < kBwdRows * dp; e += kBwdThreads) {
     s_dk[e] = 0.f;
     s_dv[e] = 0.f;
   }
@@ -353,8 +352,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
   for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {
     const int r = e / d, c = e - r * d;
     if (r0 + r < n_rows) {
-      dk[(long long)(r0 + r) * d + c] = from_f32<T>(s_dk[e]);
-      dv[(long long)(r0 + r) * d + c] = from_f32<T>(s_dv[e]);
+      dk[(long long)(r0 + r) * d + c] = from_f32<T>(s_dk[r * dp + c]);
+      dv[(long long)(r0 + r) * d + c] = from_f32<T>(s_dv[r * dp + c]);
     }
   }
 }
