@@ -685,7 +685,7 @@ template <typename T>
 int backward_gradients(const Problem& p, const void* q, const void* k, const void* v,
                        const void* agents, const void* dout, void* dq, void* dk, void* dv,
                        float* dagents, float* a32, float* va32, float* ml, float* dva, float* da,
-                       float* dqa, cudaStream_t st) {
+                       float* dqa, float* ej, cudaStream_t st) {
   const long long BH = p.BH();
   const size_t kd = (size_t)p.k * p.d;
   const size_t nd = (size_t)p.N * p.d;
@@ -713,11 +713,19 @@ int backward_gradients(const Problem& p, const void* q, const void* k, const voi
   if (r != AA_OK) return r;
   bwd_query_kernel<T><<<grid_b, kBwdThreads, smem_b, st>>>(g);
   AA_CUDA(cudaGetLastError());
-  // 4. aggregation-stage gradients
+  // 4. aggregation-stage gradients, with E_j = dV_A_j . V_A_j computed once
+  // per (slice, agent)
+  {
+    const long long rows = BH * (long long)p.k;
+    bwd_agent_e_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(dva, va32, ej, rows,
+                                                                           p.d);
+    AA_CUDA(cudaGetLastError());
+  }
   g.x = k;
   g.y = v;
   g.dva = dva;
   g.ml = ml;
+  g.e = ej;
   g.dk = dk;
   g.dv = dv;
   r = ensure_smem(bwd_key_kernel<T>, smem_b, sizeof(T) == 4 ? g_bwd_k_f32 : g_bwd_k_bf16);
@@ -762,6 +770,7 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
   const size_t dva_off = off;   off += round256(BH * kd * 4);
   const size_t da_off = off;    off += round256(BH * kd * 4);
   const size_t dq_off = off;    off += round256(BH * nd * 4);
+  const size_t e_off = off;     off += round256(BH * (size_t)p.k * 4);
   char* ws = nullptr;
   rc = scratch_alloc(reinterpret_cast<void**>(&ws), off, st);
   if (rc != AA_OK) return rc;
@@ -771,6 +780,7 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
   float* dva = reinterpret_cast<float*>(ws + dva_off);
   float* da = reinterpret_cast<float*>(ws + da_off);
   float* dqa = reinterpret_cast<float*>(ws + dq_off);
+  float* ej = reinterpret_cast<float*>(ws + e_off);
   auto run = [&]() -> int {
     const long long n_ag = BH * (long long)kd;
     if (tc_recompute) {
@@ -800,7 +810,7 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
       int r = launch_merge<T>(pp, s, ws, va32, nullptr, st, false, ml);
       if (r != AA_OK) return r;
       return backward_gradients<T>(p, q, k, v, agents, dout, dq, dk, dv, dagents, a32, va32, ml,
-                                   dva, da, dqa, st);
+                                   dva, da, dqa, ej, st);
     }
     // 1. fp32 agents
     if (agents == nullptr) {
@@ -846,7 +856,7 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
     r = launch_merge<T>(pp, s, ws, va32, nullptr, st, false, ml);
     if (r != AA_OK) return r;
     return backward_gradients<T>(p, q, k, v, agents, dout, dq, dk, dv, dagents, a32, va32, ml,
-                                 dva, da, dqa, st);
+                                 dva, da, dqa, ej, st);
   };
   rc = run();
   cudaError_t e = cudaFreeAsync(ws, st);

@@ -35,6 +35,7 @@ struct BwdArgs {
   const float* va;      // V_A [BH][n_agents][d] fp32
   const float* dva;     // key kernel: dV_A [BH][n_agents][d]
   const float* ml;      // key kernel: aggregation row max (log2 units) and sum [BH][n_agents][2]
+  const float* e;       // key kernel: E_j = dV_A_j . V_A_j [BH][n_agents]
   float* dq;            // query kernel: dQ [BH][N][d] fp32
   float* dva_acc;       // query kernel: += dV_A
   float* da_acc;        // both: += dA
@@ -297,11 +298,11 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
   const T* X = static_cast<const T*>(p.x) + bh * (long long)p.N * d;
   const T* Y = static_cast<const T*>(p.y) + bh * (long long)p.N * d;
   const float* A = p.a + bh * (long long)K * d;
-  const float* VA = p.va + bh * (long long)K * d;
   const float* DVA = p.dva + bh * (long long)K * d;
   const float* ML = p.ml + bh * (long long)K * 2;
+  const float* EJ = p.e + bh * (long long)K;
   float* da = p.da_acc + bh * (long long)K * d;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   bwd_load_rows(s_x, X, r0, n_rows, d, dp);
   bwd_load_rows(s_y, Y, r0, n_rows, d, dp);
   for (int e = tid; e < kBwdRows * dp; e += kBwdThreads) {
@@ -313,19 +314,12 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
     __syncthreads();
     bwd_load_agents(s_a, A, j0, K, d, dp);
     bwd_load_agents(s_dva, DVA, j0, K, d, dp);
-    // E_j = dV_A_j . V_A_j, one warp per agent of the chunk
-    for (int j = warp; j < kBwdCols; j += kBwdThreads / 32) {
-      float e = 0.f;
-      if (j < valid)
-        for (int c = lane; c < d; c += 32)
-          e = fmaf(DVA[(long long)(j0 + j) * d + c], VA[(long long)(j0 + j) * d + c], e);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-      if (lane == 0) {
-        s_je[j] = e;
-        s_jm[j] = j < valid ? ML[(long long)(j0 + j) * 2] : 0.f;
-        s_jl[j] = j < valid ? ML[(long long)(j0 + j) * 2 + 1] : 1.f;
-      }
+    // the chunk's E_j (computed once per slice by bwd_agent_e_kernel) and
+    // the saved aggregation statistics
+    for (int j = tid; j < kBwdCols; j += kBwdThreads) {
+      s_je[j] = j < valid ? EJ[j0 + j] : 0.f;
+      s_jm[j] = j < valid ? ML[(long long)(j0 + j) * 2] : 0.f;
+      s_jl[j] = j < valid ? ML[(long long)(j0 + j) * 2 + 1] : 1.f;
     }
     __syncthreads();
     bwd_dots(s_t, s_x, s_a, d, dp, p.scale_log2);
@@ -356,6 +350,21 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
       dv[(long long)(r0 + r) * d + c] = from_f32<T>(s_dv[r * dp + c]);
     }
   }
+}
+
+// E_j = dV_A_j . V_A_j for every (slice, agent): a warp per agent row.
+__global__ void __launch_bounds__(256) bwd_agent_e_kernel(const float* __restrict__ dva,
+                                                          const float* __restrict__ va,
+                                                          float* __restrict__ e, long long rows,
+                                                          int d) {
+  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float acc = 0.f;
+  for (int c = lane; c < d; c += 32) acc = fmaf(dva[row * d + c], va[row * d + c], acc);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) e[row] = acc;
 }
 
 // dQ = dq_acc (+ the pooling adjoint of dA when the agents were pooled), in T.
