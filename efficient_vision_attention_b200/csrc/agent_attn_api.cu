@@ -494,19 +494,21 @@ int run_broadcast(const Problem& p, const void* q, const AgentsRef& ag, const vo
   return launch_simt_attend<T>(a, p.BH(), st, pdl);
 }
 
-// Small bf16 slices with pooled agents and no bias run the whole pass in one
-// kernel, one CTA per slice (agent_fused_small_tc).
-bool use_fused_small(const Problem& p, bool learnable) {
-  return !learnable && !p.force_simt && p.dtype == AA_BF16 && !has_bias(p) &&
+// Small bf16 slices (pooled or given agents, no bias) run the whole pass in
+// one kernel, one CTA per slice (agent_fused_small_tc).
+bool use_fused_small(const Problem& p) {
+  return !p.force_simt && p.dtype == AA_BF16 && !has_bias(p) &&
          tc::fused_small_fits(p.N, p.d, p.k);
 }
 
 template <typename T>
 int run_forward(const Problem& p, const Scratch& s, const void* q, const void* k, const void* v,
                 const AgentsRef* learnable, void* out, char* ws, cudaStream_t st) {
-  if (sizeof(T) == 2 && use_fused_small(p, learnable != nullptr)) {
-    cudaError_t e = tc_launch_fused_small(q, k, v, out, p.B, p.H, p.N, p.d, p.grid_h, p.grid_w,
-                                          p.pool_h, p.pool_w, p.scale * kLog2e, st);
+  if (sizeof(T) == 2 && use_fused_small(p)) {
+    cudaError_t e = tc_launch_fused_small(
+        q, k, v, out, p.B, p.H, p.N, p.d, p.grid_h, p.grid_w, p.pool_h, p.pool_w, p.k,
+        learnable ? learnable->ptr : nullptr, learnable ? learnable->bstride : 0,
+        p.scale * kLog2e, st);
     if (e != cudaSuccess) return cuda_fail(e, "agent forward (fused small slices) launch");
     return AA_OK;
   }

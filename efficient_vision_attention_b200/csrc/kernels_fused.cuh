@@ -1,13 +1,14 @@
 // Whole forward pass of one small slice in one CTA (bf16, N <= 256 tokens,
-// k <= 128 pooled agents, d <= 64): agent_fused_small_tc.
+// k <= 128 pooled or given agents, d <= 64): agent_fused_small_tc.
 //
 // For slices this small the three-kernel path is bound by its launches and
 // hand-offs (a pool, a split aggregation whose partials go through HBM, a
 // merge and a broadcast for a few hundred tokens).  Here one CTA per (b, h)
 // stages Q, K and V once by TMA and runs every step on chip:
 //
-//   1. pool     A[a] = mean of Q over agent a's bin (adaptive bins), written
-//               as bf16 in the 128-byte-swizzled operand layout;
+//   1. pool     A[a] = mean of Q over agent a's bin (adaptive bins), or the
+//               given agent rows, written as bf16 in the 128-byte-swizzled
+//               operand layout;
 //   2. S1 = A K^T             tcgen05 SS, M = 128 agent rows, N = N rounded
 //                              up to 16 (keys), into TMEM;
 //   3. softmax over the keys, P1 as bf16 over its scores (two passes: row
@@ -106,7 +107,9 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
                                 const __grid_constant__ CUtensorMap map_k,
                                 const __grid_constant__ CUtensorMap map_v,
                                 const __grid_constant__ CUtensorMap map_o, int N, int d,
-                                int grid_h, int grid_w, int pool_h, int pool_w, float c) {
+                                int grid_h, int grid_w, int pool_h, int pool_w, int k, int H,
+                                const __nv_bfloat16* __restrict__ agents, long long ag_bstride,
+                                float c) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const FusedLayout L = fused_layout(N);
@@ -121,7 +124,6 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x;
-  const int k = pool_h * pool_w;
   const int kpad = round16(k);
   const int npad = L.rows_alloc;                       // keys, rounded up to 16
   const int d16 = (d + 15) >> 4;
@@ -168,9 +170,19 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
   pdl_trigger();
   bool ok = fused_wait(&bars->tma_q, 0, abort, true);
 
-  // ---- 1. pool: thread per (agent row of the 128-row tile, 8-channel group)
+  // ---- 1. the agents: given ones (bf16 [H][k][d] per batch set) or pooled
+  // from the staged Q; thread per (agent row of the 128-row tile, 8-channel group)
+  const __nv_bfloat16* ag_rows =
+      agents ? agents + (long long)(bh / H) * ag_bstride + (long long)(bh % H) * k * d : nullptr;
   for (int it = threadIdx.x; it < kFusedMaxAgents * 8; it += kFusedThreads) {
     const int a = it >> 3, g = it & 7;
+    if (ag_rows) {
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (a < k && g < groups)
+        w = __ldg(reinterpret_cast<const uint4*>(ag_rows + (long long)a * d + g * 8));
+      *reinterpret_cast<uint4*>(sA + a * kRowBytes + ((g ^ (a & 7)) << 4)) = w;
+      continue;
+    }
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -381,10 +393,14 @@ __global__ void __launch_bounds__(kFusedThreads, 2)
 
 }  // namespace tc
 
-// Host launch of the fused small-slice forward pass (pooled agents, no bias).
+// Host launch of the fused small-slice forward pass (no bias): pooled agents
+// (agents = null) or given bf16 agents [H][n_agents][d] per batch set
+// (ag_bstride elements between sets, 0 = shared over the batch).
 inline cudaError_t tc_launch_fused_small(const void* q, const void* k, const void* v, void* out,
                                          int B, int H, int N, int d, int grid_h, int grid_w,
-                                         int pool_h, int pool_w, float c, cudaStream_t st) {
+                                         int pool_h, int pool_w, int n_agents,
+                                         const void* agents, long long ag_bstride, float c,
+                                         cudaStream_t st) {
   using namespace tc;
   const long long BH = (long long)B * H;
   if (BH > 0x7fffffffLL) return cudaErrorInvalidValue;
@@ -399,7 +415,7 @@ inline cudaError_t tc_launch_fused_small(const void* q, const void* k, const voi
   if (e != cudaSuccess) return e;
   return launch_kernel(agent_fused_small_tc_kernel, dim3((unsigned)BH), dim3(kFusedThreads),
                        L.smem, st, false, mq, mk, mv, mo, N, d, grid_h, grid_w, pool_h, pool_w,
-                       c);
+                       n_agents, H, static_cast<const __nv_bfloat16*>(agents), ag_bstride, c);
 }
 
 }  // namespace aa

@@ -84,8 +84,9 @@ typedef enum { AA_FP32 = 0, AA_BF16 = 1 } aa_dtype;
  * Scratch memory (agents, partial aggregation state, V_A) is taken from the
  * library's stream-ordered pool on `stream` and returned to it (freed in
  * stream order) before the call returns.  bf16 slices of at most 256 tokens
- * with at most 128 pooled agents and d <= 64 run as one fused kernel (one
- * CTA per slice, no scratch); the result is the same computation. */
+ * with at most 128 agents (pooled or given) and d <= 64 run as one fused
+ * kernel (one CTA per slice, no scratch); the result is the same
+ * computation. */
 AA_API int agent_attn_forward(const void* q, const void* k, const void* v, const void* agents_or_null,
                        void* out, int B, int H, int N, int d, int grid_h, int grid_w, int pool_h,
                        int pool_w, float scale, int dtype, void* stream);

@@ -214,6 +214,28 @@ def test_learnable_agents_batch_stride_and_permutation(dtype):
     assert_close(f64(out_p), ref, dtype, "permuted agents")
 
 
+@pytest.mark.parametrize("shared", [True, False])
+@pytest.mark.parametrize("N,n_ag,d", [(196, 49, 64), (143, 100, 40), (256, 128, 16)])
+def test_fused_small_slices_with_given_agents(shared, N, n_ag, d):
+    """Small bf16 slices with learnable agents (shared over the batch, or one
+    set per batch through the batch stride) also run as the one-kernel pass:
+    every output against the oracle."""
+    B, H = 2, 3
+    q, k, v = random_qkv((B, H, N, d), seed=N + n_ag, dtype=torch.bfloat16)
+    g = torch.Generator().manual_seed(N + 1)
+    if shared:
+        agents = (torch.randn((H, n_ag, d), generator=g) * 0.3).to(torch.bfloat16)
+        out = run_forward_agents(q, k, v, agents, 1 / math.sqrt(d), batch_stride=0)
+        ag_ref = agents.unsqueeze(0).expand(B, H, n_ag, d)
+    else:
+        agents = (torch.randn((B, H, n_ag, d), generator=g) * 0.3).to(torch.bfloat16)
+        out = run_forward_agents(q, k, v, agents, 1 / math.sqrt(d), batch_stride=H * n_ag * d)
+        ag_ref = agents
+    ref = oracle.agent_attn(f64(q), f64(k), f64(v), N, 1, 1, 1, 1 / math.sqrt(d),
+                            agents=f64(ag_ref.contiguous()))
+    assert_close(f64(out), ref, torch.bfloat16, f"given agents N={N} k={n_ag} d={d}")
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_joint_key_value_permutation(dtype):
     B, H, gh, gw, d = 1, 2, 30, 30, 64
