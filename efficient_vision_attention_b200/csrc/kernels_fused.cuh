@@ -1,7 +1,7 @@
 // Whole forward pass of one small slice in one CTA (bf16, N <= 256 tokens,
 // k <= 128 pooled or given agents, d <= 64): agent_fused_small_tc.
 //
-// For slices this small the three-kernel path is bound by its launches and
+// For slices this small the four-kernel path is bound by its launches and
 // hand-offs (a pool, a split aggregation whose partials go through HBM, a
 // merge and a broadcast for a few hundred tokens).  Here one CTA per (b, h)
 // stages Q, K and V once by TMA and runs every step on chip:
@@ -12,7 +12,7 @@
 //   2. S1 = A K^T             tcgen05 SS, M = 128 agent rows, N = N rounded
 //                              up to 16 (keys), into TMEM;
 //   3. softmax over the keys, P1 as bf16 over its scores (two passes: row
-//      maxima, then exponentials; the row sums add the rounded P);
+//      maxima, then exponentials, with the row sums of slab_exp);
 //   4. U = P1 V               tcgen05 TS (V as an MN-major operand);
 //   5. V_A = U / l1 as bf16 in shared memory (MN-major operand layout);
 //   6. S2 = Q A^T per 128-query tile, softmax over the agents, P2 over S2;
