@@ -411,6 +411,27 @@ def run_native(args, w):
            "achieved_gbs": dwc_bytes / (dwc_ms * 1e-3) / 1e9,
            "frac": dwc_bytes / (dwc_ms * 1e-3) / 1e9 / peak}
 
+    # The full module output (attention + DWC term) through its own entry
+    # point: the forward pass, then the DWC kernel accumulating into its output
+    # (chained by programmatic dependent launch).
+    def run_fwd_dwc(s):
+        eva.agent_attn_forward_dwc(s["q"], s["k"], s["v"], agents if w.learnable_agents else None,
+                                   dwc_w, dwc_b, s["out"], B, H, N, d, w.grid_h, w.grid_w,
+                                   w.pool_h, w.pool_w, w.scale, dt, stream)
+
+    for r in range(3):
+        run_fwd_dwc(sets[r % n_sets])
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for r in range(reps):
+        run_fwd_dwc(sets[r % n_sets])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    fd_ms = e0.elapsed_time(e1) / reps
+    fwd_dwc = {"ms_per_forward": fd_ms, "value": B * H * N / (fd_ms * 1e-3), "unit": UNIT,
+               "vs_forward": fd_ms / ms_max}
+
     # The forward pass with agent bias (row, column and block components in
     # both softmaxes) on the same workload (bias added inside the score tiles).
     gb_ = torch.Generator().manual_seed(w.seed + 78)
@@ -522,6 +543,7 @@ def run_native(args, w):
         "roofline": roofline,
         "sfu_roofline": sfu,
         "dwc_term": dwc,
+        "forward_dwc": fwd_dwc,
         "agent_bias_forward": bias_fwd,
         "backward": bwd,
         "cpu_baseline": base,
