@@ -307,8 +307,9 @@ int launch_pool(const Problem& p, const void* q, float* a_f32, T* a_lowp, cudaSt
       const long long nb = (p.BH() - b0 < 65535) ? p.BH() - b0 : 65535;
       const long long qoff = b0 * (long long)p.N * p.d;
       const long long aoff = b0 * (long long)p.k * p.d;
-      agent_pool_band_kernel<T><<<dim3((unsigned)grid_x, (unsigned)nb), bp.threads, bp.smem,
-                                  st>>>(
+      auto kernel = pool_band_batch(bp.rows) == 4 ? agent_pool_band_kernel<T, 4>
+                                                  : agent_pool_band_kernel<T, kPoolBandBatch>;
+      kernel<<<dim3((unsigned)grid_x, (unsigned)nb), bp.threads, bp.smem, st>>>(
           static_cast<const __nv_bfloat16*>(q) + qoff, a_f32 ? a_f32 + aoff : nullptr,
           a_lowp ? a_lowp + aoff : nullptr, p.N, p.d, p.grid_w, p.pool_h, p.pool_w, bp.rows,
           bp.bin_w, bp.chunk_cols);

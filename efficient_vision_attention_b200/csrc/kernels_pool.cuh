@@ -172,12 +172,18 @@ __global__ void __launch_bounds__(kPoolTmaThreads) agent_pool_tma_kernel(
 // When the bins tile the grid exactly (grid_h = R pool_h, grid_w = W pool_w)
 // every agent averages an R x W block, and a CTA takes one band of R grid
 // rows and a chunk of token columns of one slice: a thread per (token column,
-// 8-channel group) issues the R 16-byte loads of its column 16 at a time (in
-// flight together, straight into registers, no staging), sums them in fp32 into a
-// shared column sum, and a thread per (agent, 8-channel group) then adds the
-// W columns of its bin and divides by R W.
-constexpr int kPoolBandBatch = 16;      // rows of a column whose loads are in flight together
+// 8-channel group) issues the R 16-byte loads of its column kBatch at a time
+// (in flight together, straight into registers, no staging), sums them in
+// fp32 into a shared column sum, and a thread per (agent, 8-channel group)
+// then adds the W columns of its bin and divides by R W.  kBatch is 4 for
+// bins of up to 4 rows, else 8 (taller bins loop over 8-row batches): the
+// batch's registers bound how many CTAs share an SM, and with 16 rows' loads
+// in flight a thread needed about 108 registers (3 CTAs of 160 threads per
+// SM, 2.3 waves on the SD-latent grid) against 56 for 8 rows (7 CTAs, one
+// wave).
+constexpr int kPoolBandBatch = 8;       // largest batch of a column's loads in flight together
 constexpr int kPoolBandMaxRows = 64;
+inline int pool_band_batch(int rows) { return rows <= 4 ? 4 : kPoolBandBatch; }
 
 struct PoolBandPlan {
   int rows, bin_w, chunk_cols, threads;
@@ -210,8 +216,9 @@ inline PoolBandPlan pool_band_plan(int grid_h, int grid_w, int pool_h, int pool_
   return pl;
 }
 
-template <typename T>
-__global__ void agent_pool_band_kernel(const __nv_bfloat16* __restrict__ q,
+template <typename T, int kBatch>
+__global__ void __maxnreg__(kBatch <= 4 ? 40 : 56)
+    agent_pool_band_kernel(const __nv_bfloat16* __restrict__ q,
                                        float* __restrict__ a_f32, T* __restrict__ a_lowp, int N,
                                        int d, int grid_w, int pool_h, int pool_w, int rows,
                                        int bin_w, int chunk_cols) {
@@ -232,14 +239,18 @@ __global__ void agent_pool_band_kernel(const __nv_bfloat16* __restrict__ q,
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    if (rows <= kPoolBandBatch) {
-      // bins of up to 16 rows: every load of the column in flight at once
-      uint4 raw[kPoolBandBatch];
+    if (rows <= kBatch) {
+      // bins of up to kBatch rows: every load of the column in flight at once
+      // (32-bit offsets in 16-byte units from one base address: a band spans
+      // rows * grid_w * d elements < 2^31 here)
+      const uint4* base = reinterpret_cast<const uint4*>(src);
+      const uint32_t step = (uint32_t)(row_step >> 3);
+      uint4 raw[kBatch];
 #pragma unroll
-      for (int r = 0; r < kPoolBandBatch; ++r)
-        if (r < rows) raw[r] = __ldcs(reinterpret_cast<const uint4*>(src + r * row_step));
+      for (int r = 0; r < kBatch; ++r)
+        if (r < rows) raw[r] = __ldcs(base + r * step);
 #pragma unroll
-      for (int r = 0; r < kPoolBandBatch; ++r) {
+      for (int r = 0; r < kBatch; ++r) {
         if (r < rows) {
           const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[r]);
 #pragma unroll
@@ -251,15 +262,15 @@ __global__ void agent_pool_band_kernel(const __nv_bfloat16* __restrict__ q,
         }
       }
     } else {
-      // taller bins: 16 rows' loads in flight at a time
-      for (int rb = 0; rb < rows; rb += kPoolBandBatch) {
-        uint4 raw[kPoolBandBatch];
+      // taller bins: kBatch rows' loads in flight at a time
+      for (int rb = 0; rb < rows; rb += kBatch) {
+        uint4 raw[kBatch];
 #pragma unroll
-        for (int r = 0; r < kPoolBandBatch; ++r)
+        for (int r = 0; r < kBatch; ++r)
           if (rb + r < rows)
             raw[r] = __ldcs(reinterpret_cast<const uint4*>(src + (rb + r) * row_step));
 #pragma unroll
-        for (int r = 0; r < kPoolBandBatch; ++r) {
+        for (int r = 0; r < kBatch; ++r) {
           if (rb + r < rows) {
             const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[r]);
 #pragma unroll
