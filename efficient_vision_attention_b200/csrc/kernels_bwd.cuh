@@ -27,6 +27,10 @@ namespace aa {
 constexpr int kBwdRows = 64;     // query or key rows per CTA
 constexpr int kBwdCols = 32;     // agents per chunk
 constexpr int kBwdThreads = 256;
+// Row stride of the [rows][agents] score and gradient tiles: 36 floats, so a
+// row's 4 consecutive agents are one aligned float4 and the 4 row pairs a
+// warp writes in bwd_dots fall in 4 disjoint groups of 8 banks.
+constexpr int kBwdTStride = kBwdCols + 4;
 
 struct BwdArgs {
   const void* x;        // q (query kernel) or k (key kernel): [BH][N][d] of T
@@ -53,7 +57,7 @@ __host__ __device__ __forceinline__ int bwd_row_stride(int d) { return d + 4; }
 
 __host__ __forceinline__ size_t bwd_smem_bytes(int d) {
   const size_t dp = bwd_row_stride(d);
-  return sizeof(float) * (2 * kBwdRows * dp + 2 * kBwdCols * dp + 2 * kBwdRows * (kBwdCols + 1) +
+  return sizeof(float) * (2 * kBwdRows * dp + 2 * kBwdCols * dp + 2 * kBwdRows * kBwdTStride +
                           (size_t)kBwdRows * dp * 2 + 4 * kBwdRows + 4 * kBwdCols);
 }
 
@@ -75,42 +79,50 @@ __device__ __forceinline__ void bwd_load_agents(float* dst, const float* src, in
 }
 
 // dot products of the CTA's rows with a chunk's agents: out[r][j] = X_r . Y_j * mul.
-// Register-tiled: thread t owns rows 2(t/8), 2(t/8)+1 and agents t%8 + 8q,
-// q = 0..3 (256 threads x 8 dots = 64 x 32); per 4 channels it reads 6 float4
-// (rows 16-byte aligned, d % 4 == 0) for 32 FMAs.  The 8 threads of a
-// quarter-warp read 8 consecutive agent rows d + 4 floats apart: 8 distinct
-// 4-bank groups (no conflict); their shared row is a broadcast.
+// Register-tiled on the first 128 threads: thread t owns rows 4(t/8) .. +3
+// and agents t%8 + 8q, q = 0..3 (128 threads x 16 dots = 64 x 32); per 4
+// channels it reads 8 float4 (rows 16-byte aligned, d % 4 == 0) for 64 FMAs.
+// The 8 threads of a quarter-warp read 8 consecutive agent rows d + 4 floats
+// apart: 8 distinct 4-bank groups (no conflict); their shared rows are
+// broadcasts.  (Shared-memory reads bound these kernels: 8 reads per 64 FMAs
+// instead of 6 per 32 with all 256 threads on 2 x 4 tiles.)
 __device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc) {
   return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
 }
 __device__ __forceinline__ void bwd_dots(float* out, const float* X, const float* Y, int d, int dp,
                                          float mul) {
-  static_assert(kBwdRows * kBwdCols == kBwdThreads * 8, "2 x 4 dots per thread");
+  static_assert(kBwdRows * kBwdCols == 128 * 16, "4 x 4 dots per thread on 128 threads");
   const int t = threadIdx.x;
-  const int r = 2 * (t >> 3), j = t & 7;
+  if (t >= 128) return;
+  const int r = 4 * (t >> 3), j = t & 7;
   const float* x0 = X + r * dp;
-  const float* x1 = x0 + dp;
   const float* y0 = Y + j * dp;
-  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
   for (int c = 0; c < d; c += 4) {
-    const float4 a0 = *reinterpret_cast<const float4*>(x0 + c);
-    const float4 a1 = *reinterpret_cast<const float4*>(x1 + c);
+    float4 a[4], b[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 bq = *reinterpret_cast<const float4*>(y0 + 8 * q * dp + c);
-      acc[0][q] = dot4(a0, bq, acc[0][q]);
-      acc[1][q] = dot4(a1, bq, acc[1][q]);
-    }
+    for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(x0 + i * dp + c);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) b[q] = *reinterpret_cast<const float4*>(y0 + 8 * q * dp + c);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[i][q] = dot4(a[i], b[q], acc[i][q]);
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    out[r * (kBwdCols + 1) + j + 8 * q] = acc[0][q] * mul;
-    out[(r + 1) * (kBwdCols + 1) + j + 8 * q] = acc[1][q] * mul;
-  }
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) out[(r + i) * kBwdTStride + j + 8 * q] = acc[i][q] * mul;
 }
 
 // out[r][c] += mul * sum_{j < valid} W[r][j] M[j][c] for the CTA's 64 rows:
-// thread items = (row pair, 4 channels), 6 shared reads per 8 FMAs.
+// thread items = (row pair, 4 channels); per 4 agents, one float4 of W per
+// row and one float4 of M per agent feed 32 FMAs (6 shared reads).  Agents
+// past `valid` up to the next multiple of 4 have zero W (and zero M rows).
 __device__ __forceinline__ void bwd_rows_acc(float* out, const float* W, const float* M, int d,
                                              int dp, int valid, float mul) {
   const int nq = (d + 3) >> 2;
@@ -118,14 +130,19 @@ __device__ __forceinline__ void bwd_rows_acc(float* out, const float* W, const f
     const int rp = e / nq, c = 4 * (e - rp * nq);
     const int r = 2 * rp;
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < valid; ++j) {
-      const float w0 = W[r * (kBwdCols + 1) + j], w1 = W[(r + 1) * (kBwdCols + 1) + j];
-      const float4 m4 = *reinterpret_cast<const float4*>(M + j * dp + c);   // d % 4 == 0
-      const float m[4] = {m4.x, m4.y, m4.z, m4.w};
+    for (int j = 0; j < valid; j += 4) {
+      const float4 w0 = *reinterpret_cast<const float4*>(W + r * kBwdTStride + j);
+      const float4 w1 = *reinterpret_cast<const float4*>(W + (r + 1) * kBwdTStride + j);
+      const float wa[4] = {w0.x, w0.y, w0.z, w0.w}, wb[4] = {w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        a0[q] = fmaf(w0, m[q], a0[q]);
-        a1[q] = fmaf(w1, m[q], a1[q]);
+        const float4 m4 = *reinterpret_cast<const float4*>(M + (j + q) * dp + c);   // d % 4 == 0
+        const float m[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          a0[i] = fmaf(wa[q], m[i], a0[i]);
+          a1[i] = fmaf(wb[q], m[i], a1[i]);
+        }
       }
     }
     // out rows dp floats apart (16-byte aligned): one float4 update per row
@@ -149,32 +166,44 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 }
 
 // acc[j][c] = mul * sum_r W[r][j] X[r][c] for the chunk's agents j < valid,
-// added atomically into dst[(j0 + j) * d + c]: items = (agent pair, 4 channels).
+// added atomically into dst[(j0 + j) * d + c].  Items = (4 agents, 4
+// channels): per row one float4 of W (the 4 agents) and one of X (the 4
+// channels) feed 16 FMAs.  The 64 rows are split between up to 3 groups of
+// items (as many as the block holds), each adding its own partial sums.
+constexpr int kBwdAccGroups = 3;
 __device__ __forceinline__ void bwd_agents_acc(float* dst, int j0, const float* W, const float* X,
                                                int d, int dp, int valid, float mul) {
-  const int nq = (d + 3) >> 2;
-  for (int e = threadIdx.x; e < (kBwdCols / 2) * nq; e += kBwdThreads) {
-    const int jp = e / nq, c = 4 * (e - jp * nq);
-    const int j = 2 * jp;
-    if (j >= valid) continue;
-    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int r = 0; r < kBwdRows; ++r) {
-      const float w0 = W[r * (kBwdCols + 1) + j], w1 = W[r * (kBwdCols + 1) + j + 1];
-      const float4 x4 = *reinterpret_cast<const float4*>(X + r * dp + c);   // d % 4 == 0
-      const float x[4] = {x4.x, x4.y, x4.z, x4.w};
+  const int nq = d >> 2;                       // d % 8 == 0
+  const int items = (kBwdCols / 4) * nq;
+  const int groups = min(kBwdAccGroups, kBwdThreads / items);
+  const int t = threadIdx.x;
+  if (t >= groups * items) return;
+  const int grp = t / items, it = t - grp * items;
+  const int jq = it / nq, c = 4 * (it - jq * nq);
+  const int j = 4 * jq;
+  if (j >= valid) return;
+  const int rb = grp * kBwdRows / groups, re = (grp + 1) * kBwdRows / groups;
+  float a[4][4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        a0[q] = fmaf(w0, x[q], a0[q]);
-        a1[q] = fmaf(w1, x[q], a1[q]);
-      }
-    }
-    // d % 4 == 0, so the 4 channels are in range and 16-byte aligned
-    red_add_v4(dst + (long long)(j0 + j) * d + c, mul * a0[0], mul * a0[1], mul * a0[2],
-               mul * a0[3]);
-    if (j + 1 < valid)
-      red_add_v4(dst + (long long)(j0 + j + 1) * d + c, mul * a1[0], mul * a1[1], mul * a1[2],
-                 mul * a1[3]);
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) a[q][e] = 0.f;
+  for (int r = rb; r < re; ++r) {
+    const float4 w4 = *reinterpret_cast<const float4*>(W + r * kBwdTStride + j);
+    const float4 x4 = *reinterpret_cast<const float4*>(X + r * dp + c);
+    const float w[4] = {w4.x, w4.y, w4.z, w4.w}, x[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a[q][e] = fmaf(w[q], x[e], a[q][e]);
   }
+  // W is zero for agents >= valid (the chunk's tail), but their rows of dst
+  // may not exist
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (j + q < valid)
+      red_add_v4(dst + (long long)(j0 + j + q) * d + c, mul * a[q][0], mul * a[q][1],
+                 mul * a[q][2], mul * a[q][3]);
 }
 
 template <typename T>
@@ -185,9 +214,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
   float* s_y = s_x + kBwdRows * dp;                  // dO rows
   float* s_a = s_y + kBwdRows * dp;                  // agent chunk [32][d+4]
   float* s_va = s_a + kBwdCols * dp;
-  float* s_t = s_va + kBwdCols * dp;                 // scores / P2 [64][33]
-  float* s_g = s_t + kBwdRows * (kBwdCols + 1);      // dP2 / dS2 [64][33]
-  float* s_acc = s_g + kBwdRows * (kBwdCols + 1);    // dQ accumulator [64][d+4]
+  float* s_t = s_va + kBwdCols * dp;                 // scores / P2 [64][36]
+  float* s_g = s_t + kBwdRows * kBwdTStride;      // dP2 / dS2 [64][36]
+  float* s_acc = s_g + kBwdRows * kBwdTStride;    // dQ accumulator [64][d+4]
   float* s_m = s_acc + kBwdRows * dp;
   float* s_l = s_m + kBwdRows;
   float* s_D = s_l + kBwdRows;
@@ -220,13 +249,13 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
     bwd_dots(s_g, s_y, s_va, d, dp, 1.f);
     __syncthreads();
     for (int r = warp; r < kBwdRows; r += kBwdThreads / 32) {
-      const float t = lane < valid ? s_t[r * (kBwdCols + 1) + lane] : -INFINITY;
+      const float t = lane < valid ? s_t[r * kBwdTStride + lane] : -INFINITY;
       float mx = t;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       const float m_new = fmaxf(s_m[r], mx);
       float e = lane < valid ? exp2f(t - m_new) : 0.f;
-      float eg = lane < valid ? e * s_g[r * (kBwdCols + 1) + lane] : 0.f;
+      float eg = lane < valid ? e * s_g[r * kBwdTStride + lane] : 0.f;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         e += __shfl_xor_sync(0xffffffffu, e, o);
@@ -258,11 +287,11 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
       const int r = e / kBwdCols, j = e - r * kBwdCols;
       float pr = 0.f, ds = 0.f;
       if (j < valid && r0 + r < n_rows) {
-        pr = exp2f(s_t[r * (kBwdCols + 1) + j] - s_m[r]) / s_l[r];
-        ds = pr * (s_g[r * (kBwdCols + 1) + j] - s_D[r]);
+        pr = exp2f(s_t[r * kBwdTStride + j] - s_m[r]) / s_l[r];
+        ds = pr * (s_g[r * kBwdTStride + j] - s_D[r]);
       }
-      s_t[r * (kBwdCols + 1) + j] = pr;
-      s_g[r * (kBwdCols + 1) + j] = ds;
+      s_t[r * kBwdTStride + j] = pr;
+      s_g[r * kBwdTStride + j] = ds;
     }
     __syncthreads();
     bwd_rows_acc(s_acc, s_g, s_a, d, dp, valid, p.scale);       // dQ_r += s sum_j ds A_j
@@ -285,9 +314,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
   float* s_y = s_x + kBwdRows * dp;                  // V rows
   float* s_a = s_y + kBwdRows * dp;                  // agent chunk
   float* s_dva = s_a + kBwdCols * dp;                // dV_A chunk
-  float* s_t = s_dva + kBwdCols * dp;                // P1 [64][33]
-  float* s_g = s_t + kBwdRows * (kBwdCols + 1);      // dS1 [64][33]
-  float* s_dk = s_g + kBwdRows * (kBwdCols + 1);     // [64][d+4]
+  float* s_t = s_dva + kBwdCols * dp;                // P1 [64][36]
+  float* s_g = s_t + kBwdRows * kBwdTStride;      // dS1 [64][36]
+  float* s_dk = s_g + kBwdRows * kBwdTStride;     // [64][d+4]
   float* s_dv = s_dk + kBwdRows * dp;                // [64][d+4]
   float* s_jm = s_dv + kBwdRows * dp;                // chunk: row max, sum, E (3 x 32)
   float* s_jl = s_jm + kBwdCols;
@@ -329,11 +358,11 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
       const int r = e / kBwdCols, j = e - r * kBwdCols;
       float pr = 0.f, ds = 0.f;
       if (j < valid && r0 + r < n_rows) {
-        pr = exp2f(s_t[r * (kBwdCols + 1) + j] - s_jm[j]) / s_jl[j];
-        ds = pr * (s_g[r * (kBwdCols + 1) + j] - s_je[j]);
+        pr = exp2f(s_t[r * kBwdTStride + j] - s_jm[j]) / s_jl[j];
+        ds = pr * (s_g[r * kBwdTStride + j] - s_je[j]);
       }
-      s_t[r * (kBwdCols + 1) + j] = pr;
-      s_g[r * (kBwdCols + 1) + j] = ds;
+      s_t[r * kBwdTStride + j] = pr;
+      s_g[r * kBwdTStride + j] = ds;
     }
     __syncthreads();
     bwd_rows_acc(s_dk, s_g, s_a, d, dp, valid, p.scale);        // dK_r += s sum_j dS1 A_j
