@@ -79,22 +79,24 @@ __device__ __forceinline__ void bwd_load_agents(float* dst, const float* src, in
 }
 
 // dot products of the CTA's rows with a chunk's agents: out[r][j] = X_r . Y_j * mul.
-// Register-tiled on the first 128 threads: thread t owns rows 4(t/8) .. +3
-// and agents t%8 + 8q, q = 0..3 (128 threads x 16 dots = 64 x 32); per 4
+// Register-tiled on the first 128 threads: thread t owns rows t/8 + 16i and
+// agents t%8 + 8q, i, q = 0..3 (128 threads x 16 dots = 64 x 32); per 4
 // channels it reads 8 float4 (rows 16-byte aligned, d % 4 == 0) for 64 FMAs.
 // The 8 threads of a quarter-warp read 8 consecutive agent rows d + 4 floats
-// apart: 8 distinct 4-bank groups (no conflict); their shared rows are
-// broadcasts.  (Shared-memory reads bound these kernels: 8 reads per 64 FMAs
+// apart: 8 distinct 4-bank groups (no conflict), and a warp's 4 row groups
+// read 4 consecutive rows (also distinct bank groups; rows 4 apart would
+// collide in pairs for d + 4 = 44); the threads sharing a row get a
+// broadcast.  (Shared-memory reads bound these kernels: 8 reads per 64 FMAs
 // instead of 6 per 32 with all 256 threads on 2 x 4 tiles.)
 __device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc) {
   return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
 }
 __device__ __forceinline__ void bwd_dots(float* out, const float* X, const float* Y, int d, int dp,
                                          float mul) {
-  static_assert(kBwdRows * kBwdCols == 128 * 16, "4 x 4 dots per thread on 128 threads");
+  static_assert(kBwdRows == 64 && kBwdCols == 32, "4 x 4 dots per thread on 128 threads");
   const int t = threadIdx.x;
   if (t >= 128) return;
-  const int r = 4 * (t >> 3), j = t & 7;
+  const int r = t >> 3, j = t & 7;
   const float* x0 = X + r * dp;
   const float* y0 = Y + j * dp;
   float acc[4][4];
@@ -105,7 +107,7 @@ __device__ __forceinline__ void bwd_dots(float* out, const float* X, const float
   for (int c = 0; c < d; c += 4) {
     float4 a[4], b[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(x0 + i * dp + c);
+    for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(x0 + 16 * i * dp + c);
 #pragma unroll
     for (int q = 0; q < 4; ++q) b[q] = *reinterpret_cast<const float4*>(y0 + 8 * q * dp + c);
 #pragma unroll
@@ -116,7 +118,7 @@ __device__ __forceinline__ void bwd_dots(float* out, const float* X, const float
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) out[(r + i) * kBwdTStride + j + 8 * q] = acc[i][q] * mul;
+    for (int q = 0; q < 4; ++q) out[(r + 16 * i) * kBwdTStride + j + 8 * q] = acc[i][q] * mul;
 }
 
 // out[r][c] += mul * sum_{j < valid} W[r][j] M[j][c] for the CTA's 64 rows:
