@@ -736,7 +736,7 @@ int backward_gradients(const Problem& p, const void* q, const void* k, const voi
   bwd_key_kernel<T><<<grid_b, kBwdThreads, smem_b, st>>>(g);
   AA_CUDA(cudaGetLastError());
   // 5. dQ (+ pooling adjoint) in the run dtype; the agents' own gradient
-  const dim3 grid_f((unsigned)(((long long)nd + 255) / 256), (unsigned)BH);
+  const dim3 grid_f((unsigned)(((long long)nd / 8 + 255) / 256), (unsigned)BH);
   bwd_finish_kernel<T><<<grid_f, 256, 0, st>>>(dqa, da, static_cast<T*>(dq), p.N, p.d, p.grid_h,
                                                p.grid_w, p.pool_h, p.pool_w,
                                                agents == nullptr ? 1 : 0);

@@ -399,33 +399,82 @@ __global__ void __launch_bounds__(256) bwd_agent_e_kernel(const float* __restric
 }
 
 // dQ = dq_acc (+ the pooling adjoint of dA when the agents were pooled), in T.
-// Thread per (token, channel); grid (ceil(N*d / 256), BH).
+// Thread per (token, 8-channel group); grid (ceil(N*d/8 / 256), BH).  The
+// bins holding a token are found once per axis: the floor cell c = y P / G
+// and its two neighbours are the only candidates (adaptive bins overlap by at
+// most one token), and a token lies in one or two bins per axis.  Each bin
+// adds its dA row divided by the bin's token count.
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_finish_kernel(const float* __restrict__ dq_acc,
                                                          const float* __restrict__ da, T* dq,
                                                          int N, int d, int grid_h, int grid_w,
                                                          int pool_h, int pool_w, int pooled) {
   const long long bh = blockIdx.y;
+  const int groups = d >> 3;
   const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= (long long)N * d) return;
-  const int n = (int)(e / d), c = (int)(e - (long long)n * d);
-  float g = dq_acc[bh * (long long)N * d + e];
+  if (e >= (long long)N * groups) return;
+  const int n = (int)(e / groups), g = (int)(e - (long long)n * groups);
+  const long long off = (bh * N + n) * (long long)d + g * 8;
+  const float4 s0 = *reinterpret_cast<const float4*>(dq_acc + off);
+  const float4 s1 = *reinterpret_cast<const float4*>(dq_acc + off + 4);
+  float acc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
   if (pooled) {
     const int y = n / grid_w, x = n - y * grid_w;
-    const long long n_agents = (long long)pool_h * pool_w;
-    const float* D = da + bh * n_agents * d;
+    // first and last bin holding the token along each axis, with their sizes
+    int by0 = -1, by1 = -1, sy0 = 1, sy1 = 1, bx0 = -1, bx1 = -1, sx0 = 1, sx1 = 1;
     const int cy = (int)(((long long)y * pool_h) / grid_h), cx = (int)(((long long)x * pool_w) / grid_w);
     for (int py = max(0, cy - 1); py <= min(pool_h - 1, cy + 1); ++py) {
       const int y0 = bin_start(py, grid_h, pool_h), y1 = bin_end(py, grid_h, pool_h);
-      if (y < y0 || y >= y1) continue;
-      for (int px = max(0, cx - 1); px <= min(pool_w - 1, cx + 1); ++px) {
-        const int x0 = bin_start(px, grid_w, pool_w), x1 = bin_end(px, grid_w, pool_w);
-        if (x < x0 || x >= x1) continue;
-        g += D[((long long)py * pool_w + px) * d + c] / (float)((y1 - y0) * (x1 - x0));
+      if (y >= y0 && y < y1) {
+        if (by0 < 0) {
+          by0 = py;
+          sy0 = y1 - y0;
+        } else {
+          by1 = py;
+          sy1 = y1 - y0;
+        }
+      }
+    }
+    for (int px = max(0, cx - 1); px <= min(pool_w - 1, cx + 1); ++px) {
+      const int x0 = bin_start(px, grid_w, pool_w), x1 = bin_end(px, grid_w, pool_w);
+      if (x >= x0 && x < x1) {
+        if (bx0 < 0) {
+          bx0 = px;
+          sx0 = x1 - x0;
+        } else {
+          bx1 = px;
+          sx1 = x1 - x0;
+        }
+      }
+    }
+    const float* D = da + bh * (long long)pool_h * pool_w * d + g * 8;
+#pragma unroll
+    for (int iy = 0; iy < 2; ++iy) {
+      const int py = iy ? by1 : by0, hy = iy ? sy1 : sy0;
+#pragma unroll
+      for (int ix = 0; ix < 2; ++ix) {
+        const int px = ix ? bx1 : bx0, hx = ix ? sx1 : sx0;
+        if (py < 0 || px < 0) continue;
+        const float* row = D + ((long long)py * pool_w + px) * d;
+        const float4 d0 = *reinterpret_cast<const float4*>(row);
+        const float4 d1 = *reinterpret_cast<const float4*>(row + 4);
+        const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+        const float size = (float)(hy * hx);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += dv[i] / size;
       }
     }
   }
-  dq[bh * (long long)N * d + e] = from_f32<T>(g);
+  T* o = dq + off;                           // 16-byte aligned: d % 8 == 0
+  if constexpr (sizeof(T) == 4) {
+    reinterpret_cast<float4*>(o)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    reinterpret_cast<float4*>(o)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  } else {
+    __nv_bfloat162 h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(h);
+  }
 }
 
 }  // namespace aa

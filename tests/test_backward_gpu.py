@@ -41,7 +41,8 @@ def run_backward(q, k, v, dout, gh, gw, ph, pw, scale, agents=None):
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("B,H,gh,gw,ph,pw,d", [(1, 1, 8, 8, 2, 2, 32), (2, 3, 14, 14, 7, 7, 64),
                                                (1, 2, 13, 11, 4, 3, 40), (1, 1, 32, 32, 16, 16, 16),
-                                               (1, 2, 9, 20, 1, 1, 8), (1, 1, 12, 12, 3, 3, 128)])
+                                               (1, 2, 9, 20, 1, 1, 8), (1, 1, 12, 12, 3, 3, 128),
+                                               (1, 1, 50, 37, 12, 9, 16)])
 def test_backward_matches_oracle(dtype, B, H, gh, gw, ph, pw, d):
     N = gh * gw
     q, k, v = random_qkv((B, H, N, d), seed=N + 7 * d, dtype=dtype)
