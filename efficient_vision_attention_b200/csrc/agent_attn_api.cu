@@ -301,18 +301,18 @@ template <typename T>
 int launch_pool(const Problem& p, const void* q, float* a_f32, T* a_lowp, cudaStream_t st) {
   const PoolBandPlan bp = pool_band_plan(p.grid_h, p.grid_w, p.pool_h, p.pool_w, p.d);
   if (sizeof(T) == 2 && bp.ok) {
-    const long long grid_x = (long long)p.pool_h * (p.grid_w / bp.chunk_cols);
+    const long long grid_x = (long long)p.pool_h * (p.pool_w / bp.bins);
     if (grid_x > 0x7fffffffLL) return AA_ERR_SHAPE;
     for (long long b0 = 0; b0 < p.BH(); b0 += 65535) {   // grid.y limit: slices in chunks
       const long long nb = (p.BH() - b0 < 65535) ? p.BH() - b0 : 65535;
       const long long qoff = b0 * (long long)p.N * p.d;
       const long long aoff = b0 * (long long)p.k * p.d;
-      auto kernel = pool_band_batch(bp.rows) == 4 ? agent_pool_band_kernel<T, 4>
-                                                  : agent_pool_band_kernel<T, kPoolBandBatch>;
+      auto kernel = pool_band_batch(bp.rows_max) == 4 ? agent_pool_band_kernel<T, 4>
+                                                      : agent_pool_band_kernel<T, kPoolBandBatch>;
       kernel<<<dim3((unsigned)grid_x, (unsigned)nb), bp.threads, bp.smem, st>>>(
           static_cast<const __nv_bfloat16*>(q) + qoff, a_f32 ? a_f32 + aoff : nullptr,
-          a_lowp ? a_lowp + aoff : nullptr, p.N, p.d, p.grid_w, p.pool_h, p.pool_w, bp.rows,
-          bp.bin_w, bp.chunk_cols);
+          a_lowp ? a_lowp + aoff : nullptr, p.N, p.d, p.grid_h, p.grid_w, p.pool_h, p.pool_w,
+          bp.bins);
       AA_CUDA(cudaGetLastError());
     }
     return AA_OK;

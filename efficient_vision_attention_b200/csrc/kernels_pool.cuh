@@ -168,47 +168,64 @@ __global__ void __launch_bounds__(kPoolTmaThreads) agent_pool_tma_kernel(
 }
 
 
-// ------------------------------------------------ uniform bins, bf16 Q
-// When the bins tile the grid exactly (grid_h = R pool_h, grid_w = W pool_w)
-// every agent averages an R x W block, and a CTA takes one band of R grid
-// rows and a chunk of token columns of one slice: a thread per (token column,
-// 8-channel group) issues the R 16-byte loads of its column kBatch at a time
-// (in flight together, straight into registers, no staging), sums them in
-// fp32 into a shared column sum, and a thread per (agent, 8-channel group)
-// then adds the W columns of its bin and divides by R W.  kBatch is 4 for
-// bins of up to 4 rows, else 8 (taller bins loop over 8-row batches): the
-// batch's registers bound how many CTAs share an SM, and with 16 rows' loads
-// in flight a thread needed about 108 registers (3 CTAs of 160 threads per
-// SM, 2.3 waves on the SD-latent grid) against 56 for 8 rows (7 CTAs, one
-// wave).
+// ------------------------------------------------ bins of at most 64 rows, bf16 Q
+// A CTA takes the grid rows [y0, y1) of one agent row py (the bin rows, 64 at
+// most) and the token columns of a chunk of consecutive agent columns of one
+// slice: a thread per (token column, 8-channel group) issues the loads of its
+// column kBatch rows at a time (in flight together, straight into registers,
+// no staging), sums them in fp32 into a shared column sum, and a thread per
+// (agent, 8-channel group) then adds the columns [x0, x1) of its bin and
+// divides by its token count.  Adaptive bins [floor(iG/P), ceil((i+1)G/P))
+// may overlap by one token: a column shared by two bins of the chunk is
+// summed once and used by both.  kBatch is 4 for bins of up to 4 rows, else
+// 8 (taller bins loop over 8-row batches): the batch's registers bound how
+// many CTAs share an SM, and with 16 rows' loads in flight a thread needed
+// about 108 registers (3 CTAs of 160 threads per SM, 2.3 waves on the
+// SD-latent grid) against 56 for 8 rows (7 CTAs, one wave).
 constexpr int kPoolBandBatch = 8;       // largest batch of a column's loads in flight together
 constexpr int kPoolBandMaxRows = 64;
+constexpr int kPoolBandMaxSide = 46340;   // grid sides whose bin products fit 32 bits
 inline int pool_band_batch(int rows) { return rows <= 4 ? 4 : kPoolBandBatch; }
+// The adaptive bin bounds in 32-bit arithmetic (exact for sides <= 46340:
+// (i + 1) g + p - 1 <= g^2 + g < 2^31).
+__device__ __forceinline__ int band_bin_start(int i, int g, int p) { return (i * g) / p; }
+__device__ __forceinline__ int band_bin_end(int i, int g, int p) { return ((i + 1) * g + p - 1) / p; }
 
 struct PoolBandPlan {
-  int rows, bin_w, chunk_cols, threads;
+  int rows_max;      // tallest bin
+  int bins;          // agent columns per chunk (a divisor of pool_w, or pool_w)
+  int threads;
   size_t smem;
   bool ok;
 };
 
 inline PoolBandPlan pool_band_plan(int grid_h, int grid_w, int pool_h, int pool_w, int d) {
-  PoolBandPlan pl{0, 0, 0, 0, 0, false};
-  if (grid_h % pool_h != 0 || grid_w % pool_w != 0 || d % 8 != 0) return pl;
-  pl.rows = grid_h / pool_h;
-  pl.bin_w = grid_w / pool_w;
-  if (pl.rows > kPoolBandMaxRows) return pl;
+  PoolBandPlan pl{0, 0, 0, 0, false};
+  if (d % 8 != 0 || pool_h < 1 || pool_w < 1 || pool_h > grid_h || pool_w > grid_w ||
+      grid_h > kPoolBandMaxSide || grid_w > kPoolBandMaxSide)
+    return pl;
+  for (int py = 0; py < pool_h; ++py) {
+    const int h = bin_end(py, grid_h, pool_h) - bin_start(py, grid_h, pool_h);
+    if (h > pl.rows_max) pl.rows_max = h;
+  }
+  if (pl.rows_max > kPoolBandMaxRows) return pl;
   const int groups = d / 8;
   // whole bins per chunk: the fewest that divide pool_w and span at least
   // 32 token columns (all of them when no smaller divisor does)
-  const int want = (32 + pl.bin_w - 1) / pl.bin_w;
-  int bins = pool_w;
+  const int min_w = grid_w / pool_w;                 // narrowest bin, >= 1
+  const int want = (32 + min_w - 1) / min_w;
+  pl.bins = pool_w;
   for (int b = 1; b < pool_w; ++b)
     if (pool_w % b == 0 && b >= want) {
-      bins = b;
+      pl.bins = b;
       break;
     }
-  pl.chunk_cols = bins * pl.bin_w;
-  const int items = pl.chunk_cols * groups;
+  int cols_max = 0;
+  for (int px0 = 0; px0 < pool_w; px0 += pl.bins) {
+    const int c = bin_end(px0 + pl.bins - 1, grid_w, pool_w) - bin_start(px0, grid_w, pool_w);
+    if (c > cols_max) cols_max = c;
+  }
+  const int items = cols_max * groups;
   pl.threads = ((items + 31) / 32) * 32;
   if (pl.threads > 1024) return pl;
   pl.smem = (size_t)items * 8 * sizeof(float);
@@ -217,34 +234,37 @@ inline PoolBandPlan pool_band_plan(int grid_h, int grid_w, int pool_h, int pool_
 }
 
 template <typename T, int kBatch>
-__global__ void __maxnreg__(kBatch <= 4 ? 40 : 56)
+__global__ void __maxnreg__(kBatch <= 4 ? 48 : 64)
     agent_pool_band_kernel(const __nv_bfloat16* __restrict__ q,
                                        float* __restrict__ a_f32, T* __restrict__ a_lowp, int N,
-                                       int d, int grid_w, int pool_h, int pool_w, int rows,
-                                       int bin_w, int chunk_cols) {
+                                       int d, int grid_h, int grid_w, int pool_h, int pool_w,
+                                       int bins) {
   extern __shared__ float band_colsum[];
   pdl_trigger();
-  const int n_chunks = grid_w / chunk_cols;
+  const int n_chunks = pool_w / bins;
   const int py = blockIdx.x / n_chunks, ch = blockIdx.x - py * n_chunks;
   const long long bh = blockIdx.y;
   const int groups = d >> 3;
-  const int xs = ch * chunk_cols;
-  const int items = chunk_cols * groups;
+  const int y0 = band_bin_start(py, grid_h, pool_h);
+  const int rows = band_bin_end(py, grid_h, pool_h) - y0;
+  const int px0 = ch * bins;
+  const int xs = band_bin_start(px0, grid_w, pool_w);
+  const int items = (band_bin_end(px0 + bins - 1, grid_w, pool_w) - xs) * groups;
   const int it = threadIdx.x;
   if (it < items) {
     const int x = it / groups, g = it - x * groups;
     const __nv_bfloat16* src =
-        q + (bh * (long long)N + (long long)py * rows * grid_w + xs + x) * d + g * 8;
+        q + (bh * (long long)N + (long long)y0 * grid_w + xs + x) * d + g * 8;
     const long long row_step = (long long)grid_w * d;
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    // 32-bit offsets in 16-byte units from one base address: a band spans
+    // at most 64 x 46340 x 128 elements / 8 < 2^32 such units
+    const uint4* base = reinterpret_cast<const uint4*>(src);
+    const uint32_t step = (uint32_t)(row_step >> 3);
     if (rows <= kBatch) {
       // bins of up to kBatch rows: every load of the column in flight at once
-      // (32-bit offsets in 16-byte units from one base address: a band spans
-      // rows * grid_w * d elements < 2^31 here)
-      const uint4* base = reinterpret_cast<const uint4*>(src);
-      const uint32_t step = (uint32_t)(row_step >> 3);
       uint4 raw[kBatch];
 #pragma unroll
       for (int r = 0; r < kBatch; ++r)
@@ -267,8 +287,7 @@ __global__ void __maxnreg__(kBatch <= 4 ? 40 : 56)
         uint4 raw[kBatch];
 #pragma unroll
         for (int r = 0; r < kBatch; ++r)
-          if (rb + r < rows)
-            raw[r] = __ldcs(reinterpret_cast<const uint4*>(src + (rb + r) * row_step));
+          if (rb + r < rows) raw[r] = __ldcs(base + (uint32_t)(rb + r) * step);
 #pragma unroll
         for (int r = 0; r < kBatch; ++r) {
           if (rb + r < rows) {
@@ -288,20 +307,21 @@ __global__ void __maxnreg__(kBatch <= 4 ? 40 : 56)
     cs[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
   __syncthreads();
-  const int per = chunk_cols / bin_w;            // agents of this chunk
-  if (it < per * groups) {
+  if (it < bins * groups) {
     const int pxl = it / groups, g = it - pxl * groups;
+    const int px = px0 + pxl;
+    const int x0 = band_bin_start(px, grid_w, pool_w) - xs;
+    const int x1 = band_bin_end(px, grid_w, pool_w) - xs;
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int x = pxl * bin_w; x < (pxl + 1) * bin_w; ++x) {
+    for (int x = x0; x < x1; ++x) {
       const float4* cs = reinterpret_cast<const float4*>(band_colsum + ((size_t)x * groups + g) * 8);
       const float4 a = cs[0], b = cs[1];
       acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
       acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
     }
-    const float inv = 1.f / (float)(rows * bin_w);
-    const int px = ch * per + pxl;
+    const float inv = 1.f / (float)(rows * (x1 - x0));
     const long long off = (bh * pool_h * (long long)pool_w + (long long)py * pool_w + px) * d + g * 8;
     float m[8];
 #pragma unroll
