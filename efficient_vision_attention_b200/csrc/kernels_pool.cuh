@@ -9,9 +9,10 @@
 // 16-byte shared loads) and phase 2 adds the columns of each agent's bin and
 // divides by its token count.  fp32 sums.  Bins follow the adaptive-pool
 // convention [floor(iG/P), ceil((i+1)G/P)) (they may overlap by one token).
-// The host uses this kernel when the tile of one agent column fits the
-// shared-memory budget and falls back to agent_pool_kernel otherwise; bf16 Q
-// on a grid that the bins divide exactly goes to agent_pool_band_kernel.
+// The host sends bf16 Q with bins of at most 64 rows (grid sides up to 46340)
+// to agent_pool_band_kernel below; otherwise it uses this kernel when the
+// tile of one agent column fits the shared-memory budget, else
+// agent_pool_kernel.
 #pragma once
 
 #include "common.cuh"
