@@ -132,6 +132,27 @@ def test_stage_pool_uniform_bins(gh, gw, ph, pw, d):
                                rtol=2 ** -7, atol=1e-6)
 
 
+@pytest.mark.parametrize("gh,gw,ph,pw,d", [(256, 256, 12, 12, 64), (128, 16, 2, 3, 24),
+                                         (50, 37, 12, 9, 16), (3, 300, 3, 7, 8),
+                                         (130, 20, 2, 3, 8)])
+def test_stage_pool_adaptive_bins(gh, gw, ph, pw, d):
+    """Bins that do not divide the grid (adaptive bounds, neighbours sharing a
+    token row or column): the high-res 256/12 shape (21-22-token bins), 64-row
+    bins (the band kernel's limit) with overlapping columns, many small
+    overlapping bins, one-row bins, and 65-row bins (past the band kernel's
+    limit: the fallback kernel)."""
+    B, H = 2, 2
+    q, _, _ = random_qkv((B, H, gh * gw, d), seed=gh * pw + d, dtype=torch.bfloat16)
+    a32 = torch.empty((B, H, ph * pw, d), dtype=torch.float32, device="cuda")
+    alow = torch.empty((B, H, ph * pw, d), dtype=torch.bfloat16, device="cuda")
+    eva.agent_attn_stage_pool(q.cuda(), a32, alow, B, H, gh * gw, d, gh, gw, ph, pw, eva.AA_BF16)
+    torch.cuda.synchronize()
+    ref = oracle.agent_pool(f64(q), gh, gw, ph, pw)
+    np.testing.assert_allclose(f64(a32), ref, rtol=0, atol=2e-6)
+    np.testing.assert_allclose(f64(alow), f64(torch.from_numpy(ref).to(torch.bfloat16)),
+                               rtol=2 ** -7, atol=1e-6)
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("N,n_agents,d", [(3136, 49, 32), (1000, 256, 40), (196, 49, 64),
                                           (4100, 144, 64), (77, 3, 16)])
