@@ -688,7 +688,8 @@ template <typename T>
 int backward_gradients(const Problem& p, const void* q, const void* k, const void* v,
                        const void* agents, const void* dout, void* dq, void* dk, void* dv,
                        float* dagents, float* a32, float* va32, float* ml, float* dva, float* da,
-                       float* dqa, float* ej, cudaStream_t st) {
+                       float* dqa, float* ej, cudaStream_t st,
+                       const tc::BcStats* qstats = nullptr) {
   const long long BH = p.BH();
   const size_t kd = (size_t)p.k * p.d;
   const size_t nd = (size_t)p.N * p.d;
@@ -710,6 +711,11 @@ int backward_gradients(const Problem& p, const void* q, const void* k, const voi
   g.d = p.d;
   g.scale = p.scale;
   g.scale_log2 = p.scale * kLog2e;
+  if (qstats) {
+    g.st_m = qstats->m;
+    g.st_l = qstats->l;
+    g.st_D = qstats->D;
+  }
   const size_t smem_b = bwd_smem_bytes(p.d);
   const dim3 grid_b((unsigned)((p.N + kBwdRows - 1) / kBwdRows), (unsigned)BH);
   r = ensure_smem(bwd_query_kernel<T>, smem_b, sizeof(T) == 4 ? g_bwd_q_f32 : g_bwd_q_bf16);
@@ -724,6 +730,7 @@ int backward_gradients(const Problem& p, const void* q, const void* k, const voi
                                                                            p.d);
     AA_CUDA(cudaGetLastError());
   }
+  g.st_m = g.st_l = g.st_D = nullptr;
   g.x = k;
   g.y = v;
   g.dva = dva;
@@ -774,6 +781,8 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
   const size_t da_off = off;    off += round256(BH * kd * 4);
   const size_t dq_off = off;    off += round256(BH * nd * 4);
   const size_t e_off = off;     off += round256(BH * (size_t)p.k * 4);
+  // the broadcast's per-query statistics (max, sum, D) from the tensor cores
+  const size_t st_off = off;    off += tc_recompute ? 3 * round256(BH * (size_t)p.N * 4) : 0;
   char* ws = nullptr;
   rc = scratch_alloc(reinterpret_cast<void**>(&ws), off, st);
   if (rc != AA_OK) return rc;
@@ -810,10 +819,21 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
                                           reinterpret_cast<float*>(ws + s.pu_off),
                                           reinterpret_cast<float*>(ws + s.pml_off), st, false);
       if (e != cudaSuccess) return cuda_fail(e, "agent_aggregate (backward recompute) launch");
-      int r = launch_merge<T>(pp, s, ws, va32, nullptr, st, false, ml);
+      T* va_low = reinterpret_cast<T*>(ws + s.va_off);
+      int r = launch_merge<T>(pp, s, ws, va32, va_low, st, false, ml);
       if (r != AA_OK) return r;
+      // 3. the broadcast on the tensor cores, writing each query's max, sum
+      // and D = dO . O instead of O (the gradient kernel's first sweep)
+      const size_t st_bytes = round256(BH * (size_t)p.N * 4);
+      const tc::BcStats qs{static_cast<const __nv_bfloat16*>(dout),
+                           reinterpret_cast<float*>(ws + st_off),
+                           reinterpret_cast<float*>(ws + st_off + st_bytes),
+                           reinterpret_cast<float*>(ws + st_off + 2 * st_bytes)};
+      e = tc_launch_broadcast(q, ag, ag_bstride, va_low, const_cast<void*>(q), p.B, p.H, p.N, p.d,
+                              p.k, p.scale * kLog2e, sms, st, false, nullptr, &qs);
+      if (e != cudaSuccess) return cuda_fail(e, "agent_broadcast (backward statistics) launch");
       return backward_gradients<T>(p, q, k, v, agents, dout, dq, dk, dv, dagents, a32, va32, ml,
-                                   dva, da, dqa, ej, st);
+                                   dva, da, dqa, ej, st, &qs);
     }
     // 1. fp32 agents
     if (agents == nullptr) {

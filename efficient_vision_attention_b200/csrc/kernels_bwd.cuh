@@ -4,7 +4,8 @@
 //   P2 = softmax_rows(s Q A^T) (N x k), O = P2 V_A
 // and an output gradient dO:
 //   bwd_query_kernel  per query row i: P2_i (two passes over agent chunks for
-//                     its max and sum), dP2_ij = dO_i . V_A_j, D_i = sum_j
+//                     its max and sum, or one when the tensor-core broadcast
+//                     supplied them with D_i), dP2_ij = dO_i . V_A_j, D_i = sum_j
 //                     P2_ij dP2_ij, dS2 = P2 (dP2 - D_i); writes dQ_i = s sum_j
 //                     dS2_ij A_j (fp32) and adds the CTA's sums of
 //                     P2_ij dO_i (-> dV_A_j) and s dS2_ij Q_i (-> dA_j) into
@@ -40,6 +41,9 @@ struct BwdArgs {
   const float* dva;     // key kernel: dV_A [BH][n_agents][d]
   const float* ml;      // key kernel: aggregation row max (log2 units) and sum [BH][n_agents][2]
   const float* e;       // key kernel: E_j = dV_A_j . V_A_j [BH][n_agents]
+  const float* st_m;    // query kernel, or null: each query's score max (log2 units),
+  const float* st_l;    //   sum of 2^(s - m) and D = dO . O [BH][N], computed
+  const float* st_D;    //   beforehand (then the first sweep is skipped)
   float* dq;            // query kernel: dQ [BH][N][d] fp32
   float* dva_acc;       // query kernel: += dV_A
   float* da_acc;        // both: += dA
@@ -233,16 +237,19 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
   bwd_load_rows(s_x, X, r0, n_rows, d, dp);
   bwd_load_rows(s_y, Y, r0, n_rows, d, dp);
   for (int e = tid; e < kBwdRows * dp; e += kBwdThreads) s_acc[e] = 0.f;
+  const bool given = p.st_m != nullptr;
   for (int r = tid; r < kBwdRows; r += kBwdThreads) {
-    s_m[r] = -INFINITY;
-    s_l[r] = 0.f;
-    s_D[r] = 0.f;
+    const bool in = r0 + r < n_rows;
+    const long long i = bh * (long long)n_rows + r0 + r;
+    s_m[r] = given ? (in ? p.st_m[i] : 0.f) : -INFINITY;
+    s_l[r] = given ? (in ? p.st_l[i] : 1.f) : 0.f;
+    s_D[r] = given ? (in ? p.st_D[i] : 0.f) : 0.f;
   }
   __syncthreads();
-  // pass 1 (online over the chunks): each row's score max m and sum
-  // l = sum_j 2^(s_j - m), and D~ = sum_j 2^(s_j - m) (dO . V_A_j), both
-  // rescaled when m grows; D_i = D~ / l
-  for (int j0 = 0; j0 < K; j0 += kBwdCols) {
+  // pass 1 (online over the chunks, unless the statistics are given): each
+  // row's score max m and sum l = sum_j 2^(s_j - m), and D~ = sum_j 2^(s_j -
+  // m) (dO . V_A_j), both rescaled when m grows; D_i = D~ / l
+  for (int j0 = 0; j0 < (given ? 0 : K); j0 += kBwdCols) {
     const int valid = min(kBwdCols, K - j0);
     bwd_load_agents(s_a, A, j0, K, d, dp);
     bwd_load_agents(s_va, VA, j0, K, d, dp);
@@ -272,8 +279,10 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
     }
     __syncthreads();
   }
-  for (int r = tid; r < kBwdRows; r += kBwdThreads) s_D[r] = s_D[r] / s_l[r];
-  __syncthreads();
+  if (!given) {
+    for (int r = tid; r < kBwdRows; r += kBwdThreads) s_D[r] = s_D[r] / s_l[r];
+    __syncthreads();
+  }
   // pass 2: dS2, dQ, and the chunk's contributions to dV_A and dA
   float* dva = p.dva_acc + bh * (long long)K * d;
   float* da = p.da_acc + bh * (long long)K * d;

@@ -90,6 +90,17 @@ struct AggParams {
   BiasParams bias;           // B1 (agents x keys), all null when absent
 };
 
+// Per-query statistics of the broadcast for the backward pass (the stats
+// instantiation writes these instead of O): the row max of the scores in log2
+// units (m), the row sum of 2^(s - m) (l), and D = dO . O with O the
+// normalised output row.  dout [BH][N][d] bf16; m, l, D [BH][N] fp32.
+struct BcStats {
+  const __nv_bfloat16* dout;
+  float* m;
+  float* l;
+  float* D;
+};
+
 struct BcParams {
   int H, N, d, k;
   float c;
@@ -97,6 +108,7 @@ struct BcParams {
   long long total_tiles;
   int ctas;
   BiasParams bias;           // B2 (queries x agents), all null when absent
+  BcStats stats;             // read only by the stats instantiation
 };
 
 struct AggBars {
@@ -907,8 +919,10 @@ __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int
   }
 }
 
-// kBias: the agent bias B2 is added in the max pass (a separate instantiation).
-template <bool kBias>
+// kBias: the agent bias B2 is added in the max pass; kStats: the epilogue
+// writes the backward pass's per-query statistics (p.stats) instead of O
+// (separate instantiations).
+template <bool kBias, bool kStats = false>
 __global__ void __launch_bounds__(kThreads, 1)
     agent_broadcast_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                               const __grid_constant__ CUtensorMap map_a,
@@ -1130,7 +1144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         t1 = row4_max(t1) * ce;
       }
       bc_slab_exp(s_col, p.k, kpad, j4, wide, ce, -t0, -t1, l0, l1, ok, bars->p_chunk[g]);
-      const float inv0 = 1.f / row4_sum(l0), inv1 = 1.f / row4_sum(l1);
+      const float sum0 = row4_sum(l0), sum1 = row4_sum(l1);
+      const float inv0 = 1.f / sum0, inv1 = 1.f / sum1;
       // epilogue: O = (P V_A) / l -> bf16 -> swizzled staging tile -> TMA store
       if (ok) ok = warp_wait(&bars->o_full[g], u & 1, abort);
       tc_fence_after();
@@ -1145,6 +1160,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       warp_arrive(&bars->o_free[g]);           // the buffer may take the next S now
+      if constexpr (kStats) {
+        // D = dO . O over the row's columns (this thread's pairs, then the 4
+        // threads of the row), and the row's max and sum, by its first thread
+        const bool in0 = q0 + r0 < p.N, in1 = q0 + r1 < p.N;
+        const long long row0 = bh * p.N + q0 + r0, row1 = row0 + 8;
+        const __nv_bfloat16* g0 = p.stats.dout + row0 * p.d + 2 * j4;
+        const __nv_bfloat16* g1 = p.stats.dout + row1 * p.d + 2 * j4;
+        float dd0 = 0.f, dd1 = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int ch = 2 * q + h;
+            if (ch * 8 < p.d) {
+              if (in0) {
+                const uint32_t w = __ldg(reinterpret_cast<const unsigned int*>(g0 + ch * 8));
+                dd0 = fmaf(bf16x2_lo(w), o[q][4 * h] * inv0, dd0);
+                dd0 = fmaf(bf16x2_hi(w), o[q][4 * h + 1] * inv0, dd0);
+              }
+              if (in1) {
+                const uint32_t w = __ldg(reinterpret_cast<const unsigned int*>(g1 + ch * 8));
+                dd1 = fmaf(bf16x2_lo(w), o[q][4 * h + 2] * inv1, dd1);
+                dd1 = fmaf(bf16x2_hi(w), o[q][4 * h + 3] * inv1, dd1);
+              }
+            }
+          }
+        }
+        dd0 = row4_sum(dd0);
+        dd1 = row4_sum(dd1);
+        if (ok && j4 == 0) {
+          if (in0) {
+            p.stats.m[row0] = t0;
+            p.stats.l[row0] = sum0;
+            p.stats.D[row0] = dd0;
+          }
+          if (in1) {
+            p.stats.m[row1] = t1;
+            p.stats.l[row1] = sum1;
+            p.stats.D[row1] = dd1;
+          }
+        }
+        continue;                              // no O tile to stage or store
+      }
       if (leader) tma_store_wait_read();
       named_barrier(3 + g, kSoftmaxThreads);
 #pragma unroll
@@ -1271,6 +1329,10 @@ inline std::atomic<int>* smem_flags_bc() {
   static std::atomic<int> f[64];
   return f;
 }
+inline std::atomic<int>* smem_flags_bc_stats() {
+  static std::atomic<int> f[64];
+  return f;
+}
 
 inline cudaError_t ensure_tc_smem(const void* kernel, int bytes, std::atomic<int>* flags) {
   int dev = 0;
@@ -1328,7 +1390,8 @@ inline cudaError_t tc_launch_aggregate(const void* agents, long long a_bstride, 
 inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long long a_bstride,
                                        const void* va, void* out, int B, int H, int N, int d,
                                        int n_agents, float c, int sm_count, cudaStream_t st,
-                                       bool pdl, const tc::BiasParams* bias = nullptr) {
+                                       bool pdl, const tc::BiasParams* bias = nullptr,
+                                       const tc::BcStats* stats = nullptr) {
   using namespace tc;
   CUtensorMap mq, ma, mva, mo;
   int a_sets = 1;
@@ -1339,12 +1402,16 @@ inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long l
       !make_map_agents(&ma, agents, d, n_agents, H, B, a_bstride, kpad, &a_sets))
     return cudaErrorInvalidValue;
   const bool biased = bias != nullptr && bias->any();
-  cudaError_t e = biased ? ensure_tc_smem(reinterpret_cast<const void*>(
-                                              agent_broadcast_tc_kernel<true>),
-                                          (int)kBcSmemBytes, smem_flags_bc_bias())
-                         : ensure_tc_smem(reinterpret_cast<const void*>(
-                                              agent_broadcast_tc_kernel<false>),
-                                          (int)kBcSmemBytes, smem_flags_bc());
+  const bool with_stats = stats != nullptr;
+  if (biased && with_stats) return cudaErrorInvalidValue;   // no instantiation takes both
+  const void* kernel = biased       ? reinterpret_cast<const void*>(agent_broadcast_tc_kernel<true>)
+                       : with_stats ? reinterpret_cast<const void*>(
+                                          agent_broadcast_tc_kernel<false, true>)
+                                    : reinterpret_cast<const void*>(agent_broadcast_tc_kernel<false>);
+  cudaError_t e = ensure_tc_smem(kernel, (int)kBcSmemBytes,
+                                 biased       ? smem_flags_bc_bias()
+                                 : with_stats ? smem_flags_bc_stats()
+                                              : smem_flags_bc());
   if (e != cudaSuccess) return e;
   BcParams p;
   p.H = H;
@@ -1356,7 +1423,10 @@ inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long l
   p.total_tiles = BH * p.tiles_per_slice;
   p.ctas = (int)(p.total_tiles < sm_count ? p.total_tiles : sm_count);
   p.bias = bias ? *bias : BiasParams{nullptr, nullptr, nullptr, 1, 1, 1, 1, 0};
-  return launch_kernel(biased ? agent_broadcast_tc_kernel<true> : agent_broadcast_tc_kernel<false>,
+  p.stats = with_stats ? *stats : BcStats{nullptr, nullptr, nullptr, nullptr};
+  return launch_kernel(biased       ? agent_broadcast_tc_kernel<true>
+                       : with_stats ? agent_broadcast_tc_kernel<false, true>
+                                    : agent_broadcast_tc_kernel<false>,
                        dim3(p.ctas), dim3(kThreads), kBcSmemBytes, st, pdl, mq, ma, mva, mo,
                        a_sets, p);
 }
