@@ -667,6 +667,7 @@ int validate_dwc(const void* v, const float* w, const void* out, int B, int H, i
 
 // ------------------------------------------------------------ backward pass
 std::atomic<int> g_bwd_q_f32[kMaxDevices], g_bwd_q_bf16[kMaxDevices];
+std::atomic<int> g_bwd_qr_f32[kMaxDevices], g_bwd_qr_bf16[kMaxDevices];
 std::atomic<int> g_bwd_k_f32[kMaxDevices], g_bwd_k_bf16[kMaxDevices];
 std::atomic<int> g_simt_f32rows_f32[kMaxDevices], g_simt_f32rows_bf16[kMaxDevices];
 
@@ -718,9 +719,17 @@ int backward_gradients(const Problem& p, const void* q, const void* k, const voi
   }
   const size_t smem_b = bwd_smem_bytes(p.d);
   const dim3 grid_b((unsigned)((p.N + kBwdRows - 1) / kBwdRows), (unsigned)BH);
-  r = ensure_smem(bwd_query_kernel<T>, smem_b, sizeof(T) == 4 ? g_bwd_q_f32 : g_bwd_q_bf16);
-  if (r != AA_OK) return r;
-  bwd_query_kernel<T><<<grid_b, kBwdThreads, smem_b, st>>>(g);
+  if (p.d <= 64) {   // dQ accumulated in registers: 16 (d / 4) <= 256 threads
+    const size_t smem_q = bwd_query_reg_smem_bytes(p.d);
+    r = ensure_smem(bwd_query_kernel<T, true>, smem_q,
+                    sizeof(T) == 4 ? g_bwd_qr_f32 : g_bwd_qr_bf16);
+    if (r != AA_OK) return r;
+    bwd_query_kernel<T, true><<<grid_b, kBwdThreads, smem_q, st>>>(g);
+  } else {
+    r = ensure_smem(bwd_query_kernel<T>, smem_b, sizeof(T) == 4 ? g_bwd_q_f32 : g_bwd_q_bf16);
+    if (r != AA_OK) return r;
+    bwd_query_kernel<T><<<grid_b, kBwdThreads, smem_b, st>>>(g);
+  }
   AA_CUDA(cudaGetLastError());
   // 4. aggregation-stage gradients, with E_j = dV_A_j . V_A_j computed once
   // per (slice, agent)

@@ -59,6 +59,13 @@ struct BwdArgs {
 // rows start 4 banks apart.
 __host__ __device__ __forceinline__ int bwd_row_stride(int d) { return d + 4; }
 
+// Shared memory of bwd_query_kernel<T, true> (dQ accumulated in registers,
+// d <= 64): the staged tiles and the row statistics only.
+__host__ __forceinline__ size_t bwd_query_reg_smem_bytes(int d) {
+  const size_t dp = bwd_row_stride(d);
+  return sizeof(float) * (2 * kBwdRows * dp + 2 * kBwdCols * dp + 2 * kBwdRows * kBwdTStride +
+                          4 * kBwdRows);
+}
 __host__ __forceinline__ size_t bwd_smem_bytes(int d) {
   const size_t dp = bwd_row_stride(d);
   return sizeof(float) * (2 * kBwdRows * dp + 2 * kBwdCols * dp + 2 * kBwdRows * kBwdTStride +
@@ -162,6 +169,37 @@ __device__ __forceinline__ void bwd_rows_acc(float* out, const float* W, const f
   }
 }
 
+// acc[i][e] += sum_{j < valid} W[rq + 16 i][j] M[j][c + e] for the CTA's 64
+// rows held in registers across the agent chunks (d <= 64): thread t < 16 nq
+// owns rows rq + 16 i (i = 0..3, rq = t / nq) and channels c = 4 (t % nq) ..
+// + 3; per 4 agents, 4 float4 of W and 4 of M feed 64 FMAs.  Agents past
+// `valid` up to the next multiple of 4 have zero W (and zero M rows).  A
+// warp's row groups read consecutive rows (distinct bank groups).
+__device__ __forceinline__ void bwd_rows_acc_reg(float (&acc)[4][4], const float* W,
+                                                 const float* M, int d, int dp, int valid) {
+  const int nq = d >> 2;
+  const int t = threadIdx.x;
+  if (t >= 16 * nq) return;
+  const int rq = t / nq, c = 4 * (t - rq * nq);
+  for (int j = 0; j < valid; j += 4) {
+    float4 w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      w[i] = *reinterpret_cast<const float4*>(W + (rq + 16 * i) * kBwdTStride + j);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 m4 = *reinterpret_cast<const float4*>(M + (j + q) * dp + c);
+      const float m[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float wq = q == 0 ? w[i].x : q == 1 ? w[i].y : q == 2 ? w[i].z : w[i].w;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][e] = fmaf(wq, m[e], acc[i][e]);
+      }
+    }
+  }
+}
+
 // Four consecutive floats added into global memory by one vector reduction
 // (16-byte aligned address): a quarter of the L2 atomic operations of four
 // scalar atomicAdds.
@@ -212,8 +250,11 @@ __device__ __forceinline__ void bwd_agents_acc(float* dst, int j0, const float* 
                  mul * a[q][2], mul * a[q][3]);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
+// kRegAcc (d <= 64): the dQ accumulator lives in registers (no shared
+// accumulator; 80 registers, 3 CTAs per SM: bounding it to 4 CTAs at 64
+// registers spilled and measured slower).
+template <typename T, bool kRegAcc = false>
+__global__ void __launch_bounds__(kBwdThreads, kRegAcc ? 3 : 1) bwd_query_kernel(BwdArgs p) {
   extern __shared__ float sm[];
   const int d = p.d, dp = bwd_row_stride(d);
   float* s_x = sm;                                   // Q rows [64][d+4]
@@ -222,8 +263,13 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
   float* s_va = s_a + kBwdCols * dp;
   float* s_t = s_va + kBwdCols * dp;                 // scores / P2 [64][36]
   float* s_g = s_t + kBwdRows * kBwdTStride;      // dP2 / dS2 [64][36]
-  float* s_acc = s_g + kBwdRows * kBwdTStride;    // dQ accumulator [64][d+4]
-  float* s_m = s_acc + kBwdRows * dp;
+  float* s_acc = s_g + kBwdRows * kBwdTStride;    // dQ accumulator [64][d+4] (not kRegAcc)
+  float* s_m = kRegAcc ? s_acc : s_acc + kBwdRows * dp;
+  float racc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) racc[i][e] = 0.f;
   float* s_l = s_m + kBwdRows;
   float* s_D = s_l + kBwdRows;
   const long long bh = blockIdx.y;
@@ -236,7 +282,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   bwd_load_rows(s_x, X, r0, n_rows, d, dp);
   bwd_load_rows(s_y, Y, r0, n_rows, d, dp);
-  for (int e = tid; e < kBwdRows * dp; e += kBwdThreads) s_acc[e] = 0.f;
+  if (!kRegAcc)
+    for (int e = tid; e < kBwdRows * dp; e += kBwdThreads) s_acc[e] = 0.f;
   const bool given = p.st_m != nullptr;
   for (int r = tid; r < kBwdRows; r += kBwdThreads) {
     const bool in = r0 + r < n_rows;
@@ -305,15 +352,33 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_query_kernel(BwdArgs p) {
       s_g[r * kBwdTStride + j] = ds;
     }
     __syncthreads();
-    bwd_rows_acc(s_acc, s_g, s_a, d, dp, valid, p.scale);       // dQ_r += s sum_j ds A_j
+    if constexpr (kRegAcc)                                      // dQ_r += sum_j ds A_j
+      bwd_rows_acc_reg(racc, s_g, s_a, d, dp, valid);
+    else
+      bwd_rows_acc(s_acc, s_g, s_a, d, dp, valid, p.scale);     // dQ_r += s sum_j ds A_j
     bwd_agents_acc(dva, j0, s_t, s_y, d, dp, valid, 1.f);       // dV_A_j += sum_r P2 dO_r
     bwd_agents_acc(da, j0, s_g, s_x, d, dp, valid, p.scale);    // dA_j += s sum_r dS2 Q_r
     __syncthreads();
   }
   float* dq = p.dq + bh * (long long)p.N * d;
-  for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {
-    const int r = e / d, c = e - r * d;
-    if (r0 + r < n_rows) dq[(long long)(r0 + r) * d + c] = s_acc[r * dp + c];
+  if constexpr (kRegAcc) {
+    const int nq = d >> 2;
+    if (tid < 16 * nq) {
+      const int rq = tid / nq, c = 4 * (tid - rq * nq);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = rq + 16 * i;
+        if (r0 + r < n_rows)
+          *reinterpret_cast<float4*>(dq + (long long)(r0 + r) * d + c) =
+              make_float4(p.scale * racc[i][0], p.scale * racc[i][1], p.scale * racc[i][2],
+                          p.scale * racc[i][3]);
+      }
+    }
+  } else {
+    for (int e = tid; e < kBwdRows * d; e += kBwdThreads) {
+      const int r = e / d, c = e - r * d;
+      if (r0 + r < n_rows) dq[(long long)(r0 + r) * d + c] = s_acc[r * dp + c];
+    }
   }
 }
 
