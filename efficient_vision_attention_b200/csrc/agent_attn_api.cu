@@ -716,6 +716,8 @@ int backward_gradients(const Problem& p, const void* q, const void* k, const voi
     g.st_m = qstats->m;
     g.st_l = qstats->l;
     g.st_D = qstats->D;
+    g.st_p = reinterpret_cast<const uint32_t*>(qstats->p);
+    g.st_kpad = (p.k + 15) / 16 * 16;
   }
   const size_t smem_b = bwd_smem_bytes(p.d);
   const dim3 grid_b((unsigned)((p.N + kBwdRows - 1) / kBwdRows), (unsigned)BH);
@@ -740,6 +742,7 @@ int backward_gradients(const Problem& p, const void* q, const void* k, const voi
     AA_CUDA(cudaGetLastError());
   }
   g.st_m = g.st_l = g.st_D = nullptr;
+  g.st_p = nullptr;
   g.x = k;
   g.y = v;
   g.dva = dva;
@@ -790,8 +793,11 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
   const size_t da_off = off;    off += round256(BH * kd * 4);
   const size_t dq_off = off;    off += round256(BH * nd * 4);
   const size_t e_off = off;     off += round256(BH * (size_t)p.k * 4);
-  // the broadcast's per-query statistics (max, sum, D) from the tensor cores
+  // the broadcast's per-query statistics (max, sum, D) and exponentials
+  // 2^(s - m) (bf16, k padded to 16) from the tensor cores
+  const size_t kpad16 = (size_t)(p.k + 15) / 16 * 16;
   const size_t st_off = off;    off += tc_recompute ? 3 * round256(BH * (size_t)p.N * 4) : 0;
+  const size_t sp_off = off;    off += tc_recompute ? round256(BH * (size_t)p.N * kpad16 * 2) : 0;
   char* ws = nullptr;
   rc = scratch_alloc(reinterpret_cast<void**>(&ws), off, st);
   if (rc != AA_OK) return rc;
@@ -831,13 +837,15 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
       T* va_low = reinterpret_cast<T*>(ws + s.va_off);
       int r = launch_merge<T>(pp, s, ws, va32, va_low, st, false, ml);
       if (r != AA_OK) return r;
-      // 3. the broadcast on the tensor cores, writing each query's max, sum
-      // and D = dO . O instead of O (the gradient kernel's first sweep)
+      // 3. the broadcast on the tensor cores, writing each query's max, sum,
+      // D = dO . O and exponentials instead of O (the gradient kernel's first
+      // sweep and its score dot products)
       const size_t st_bytes = round256(BH * (size_t)p.N * 4);
       const tc::BcStats qs{static_cast<const __nv_bfloat16*>(dout),
                            reinterpret_cast<float*>(ws + st_off),
                            reinterpret_cast<float*>(ws + st_off + st_bytes),
-                           reinterpret_cast<float*>(ws + st_off + 2 * st_bytes)};
+                           reinterpret_cast<float*>(ws + st_off + 2 * st_bytes),
+                           reinterpret_cast<__nv_bfloat16*>(ws + sp_off)};
       e = tc_launch_broadcast(q, ag, ag_bstride, va_low, const_cast<void*>(q), p.B, p.H, p.N, p.d,
                               p.k, p.scale * kLog2e, sms, st, false, nullptr, &qs);
       if (e != cudaSuccess) return cuda_fail(e, "agent_broadcast (backward statistics) launch");

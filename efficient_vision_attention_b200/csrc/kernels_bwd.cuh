@@ -5,9 +5,11 @@
 // and an output gradient dO:
 //   bwd_query_kernel  per query row i: P2_i (two passes over agent chunks for
 //                     its max and sum, or one when the tensor-core broadcast
-//                     supplied them with D_i), dP2_ij = dO_i . V_A_j, D_i = sum_j
-//                     P2_ij dP2_ij, dS2 = P2 (dP2 - D_i); writes dQ_i = s sum_j
-//                     dS2_ij A_j (fp32) and adds the CTA's sums of
+//                     supplied them with D_i and the bf16 exponentials, which
+//                     then replace the score dot products), dP2_ij = dO_i .
+//                     V_A_j, D_i = sum_j P2_ij dP2_ij, dS2 = P2 (dP2 - D_i);
+//                     writes dQ_i = s sum_j dS2_ij A_j (fp32) and adds the
+//                     CTA's sums of
 //                     P2_ij dO_i (-> dV_A_j) and s dS2_ij Q_i (-> dA_j) into
 //                     global fp32 accumulators.
 //   bwd_key_kernel    per key row n: P1_jn from the aggregation's stored row
@@ -44,6 +46,8 @@ struct BwdArgs {
   const float* st_m;    // query kernel, or null: each query's score max (log2 units),
   const float* st_l;    //   sum of 2^(s - m) and D = dO . O [BH][N], computed
   const float* st_D;    //   beforehand (then the first sweep is skipped)
+  const uint32_t* st_p; // query kernel, or null: 2^(s - m) as bf16 pairs, [BH][N][st_kpad]
+  int st_kpad;          //   bf16 (even; columns >= n_agents hold 0), given with st_m
   float* dq;            // query kernel: dQ [BH][N][d] fp32
   float* dva_acc;       // query kernel: += dV_A
   float* da_acc;        // both: += dA
@@ -330,26 +334,56 @@ __global__ void __launch_bounds__(kBwdThreads, kRegAcc ? 3 : 1) bwd_query_kernel
     for (int r = tid; r < kBwdRows; r += kBwdThreads) s_D[r] = s_D[r] / s_l[r];
     __syncthreads();
   }
-  // pass 2: dS2, dQ, and the chunk's contributions to dV_A and dA
+  // pass 2: dS2, dQ, and the chunk's contributions to dV_A and dA.  With
+  // the exponentials given, P2 = 2^(s - m) / l comes from them (thread items
+  // = 4 bf16 pairs: rows e / 16, agents 2 (e % 16), e = tid + 256 i) and the
+  // score dot products are skipped.
   float* dva = p.dva_acc + bh * (long long)K * d;
   float* da = p.da_acc + bh * (long long)K * d;
+  static_assert(kBwdRows * kBwdCols == 8 * kBwdThreads, "4 P pairs per thread");
+  const bool p_given = p.st_p != nullptr;
+  const uint32_t* Pw = p_given ? p.st_p + (bh * n_rows + r0) * (long long)(p.st_kpad / 2) : nullptr;
   for (int j0 = 0; j0 < K; j0 += kBwdCols) {
     const int valid = min(kBwdCols, K - j0);
+    uint32_t pw[4] = {0u, 0u, 0u, 0u};
+    if (p_given) {                     // issued before the dot products hide the latency
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = tid + kBwdThreads * i, r = e >> 4, j = 2 * (e & 15);
+        if (j < valid && r0 + r < n_rows)
+          pw[i] = __ldg(Pw + (long long)r * (p.st_kpad / 2) + ((j0 + j) >> 1));
+      }
+    }
     bwd_load_agents(s_a, A, j0, K, d, dp);
     bwd_load_agents(s_va, VA, j0, K, d, dp);
     __syncthreads();
-    bwd_dots(s_t, s_x, s_a, d, dp, p.scale_log2);
+    if (!p_given) bwd_dots(s_t, s_x, s_a, d, dp, p.scale_log2);
     bwd_dots(s_g, s_y, s_va, d, dp, 1.f);
     __syncthreads();
-    for (int e = tid; e < kBwdRows * kBwdCols; e += kBwdThreads) {
-      const int r = e / kBwdCols, j = e - r * kBwdCols;
-      float pr = 0.f, ds = 0.f;
-      if (j < valid && r0 + r < n_rows) {
-        pr = exp2f(s_t[r * kBwdTStride + j] - s_m[r]) / s_l[r];
-        ds = pr * (s_g[r * kBwdTStride + j] - s_D[r]);
+    if (p_given) {
+      // a pair's second agent past the chunk is a padding column (0)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = tid + kBwdThreads * i, r = e >> 4, j = 2 * (e & 15);
+        const float inv = 1.f / s_l[r], Dr = s_D[r];
+        const float2 g2 = *reinterpret_cast<const float2*>(s_g + r * kBwdTStride + j);
+        const float p0 = __uint_as_float(pw[i] << 16) * inv;           // bf16 -> fp32
+        const float p1 = __uint_as_float(pw[i] & 0xffff0000u) * inv;
+        *reinterpret_cast<float2*>(s_t + r * kBwdTStride + j) = make_float2(p0, p1);
+        *reinterpret_cast<float2*>(s_g + r * kBwdTStride + j) =
+            make_float2(p0 * (g2.x - Dr), p1 * (g2.y - Dr));
       }
-      s_t[r * kBwdTStride + j] = pr;
-      s_g[r * kBwdTStride + j] = ds;
+    } else {
+      for (int e = tid; e < kBwdRows * kBwdCols; e += kBwdThreads) {
+        const int r = e / kBwdCols, j = e - r * kBwdCols;
+        float pr = 0.f, ds = 0.f;
+        if (j < valid && r0 + r < n_rows) {
+          pr = exp2f(s_t[r * kBwdTStride + j] - s_m[r]) / s_l[r];
+          ds = pr * (s_g[r * kBwdTStride + j] - s_D[r]);
+        }
+        s_t[r * kBwdTStride + j] = pr;
+        s_g[r * kBwdTStride + j] = ds;
+      }
     }
     __syncthreads();
     if constexpr (kRegAcc)                                      // dQ_r += sum_j ds A_j

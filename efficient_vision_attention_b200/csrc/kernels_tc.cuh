@@ -92,13 +92,15 @@ struct AggParams {
 
 // Per-query statistics of the broadcast for the backward pass (the stats
 // instantiation writes these instead of O): the row max of the scores in log2
-// units (m), the row sum of 2^(s - m) (l), and D = dO . O with O the
-// normalised output row.  dout [BH][N][d] bf16; m, l, D [BH][N] fp32.
+// units (m), the row sum of 2^(s - m) (l), D = dO . O with O the normalised
+// output row, and the row's 2^(s - m) themselves as bf16 (p).  dout
+// [BH][N][d] bf16; m, l, D [BH][N] fp32; p [BH][N][kpad] bf16.
 struct BcStats {
   const __nv_bfloat16* dout;
   float* m;
   float* l;
   float* D;
+  __nv_bfloat16* p;          // [BH][N][kpad]: 2^(s - m) as bf16 (not normalised)
 };
 
 struct BcParams {
@@ -876,9 +878,26 @@ __device__ __forceinline__ int bc_p_col(int ch, bool wide) { return (wide && ch 
 // 0), placed by bc_p_col.  Adds the exponentials to the partial row sums l0,
 // l1.  After each 64-column chunk the warp arrives on that chunk's barrier
 // (whether or not it did the work).
+// kStoreP: the packed bf16 P words of the thread's two rows also go to global
+// memory, rows g0 and g1 (bf16x2 words of a [kpad]-wide row; null: the row
+// is past the slice), for the backward pass's query gradient kernel.
+template <int R, bool kStoreP>
+__device__ __forceinline__ void bc_store_p(uint32_t* g0, uint32_t* g1, int c, int j4,
+                                           const uint32_t (&pk)[2 * R]) {
+  if constexpr (kStoreP) {
+#pragma unroll
+    for (int g = 0; g < R; ++g) {
+      if (g0) g0[(c + 8 * g) / 2 + j4] = pk[2 * g];
+      if (g1) g1[(c + 8 * g) / 2 + j4] = pk[2 * g + 1];
+    }
+  }
+}
+
+template <bool kStoreP = false>
 __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int j4, bool wide,
                                             float c_scale, float neg_m0, float neg_m1, float& l0,
-                                            float& l1, bool run, uint64_t* chunk_bar) {
+                                            float& l1, bool run, uint64_t* chunk_bar,
+                                            uint32_t* g0 = nullptr, uint32_t* g1 = nullptr) {
   int c = 0, ch = 0;
 #pragma unroll 1
   for (; c + 64 <= kpad; c += 64, ++ch) {
@@ -889,6 +908,7 @@ __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int
       if (c + 64 > k) slab_mask<8>(v, c, j4, k);
       slab_exp<8>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
       slab_st_p32(s_col + bc_p_col(ch, wide), pk);
+      bc_store_p<8, kStoreP>(g0, g1, c, j4, pk);
       tmem_wait_st();
     }
     warp_arrive(&chunk_bar[ch]);
@@ -903,6 +923,7 @@ __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int
         if (c + 32 > k) slab_mask<4>(v, c, j4, k);
         slab_exp<4>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
         slab_st_p16(pc, pk);
+        bc_store_p<4, kStoreP>(g0, g1, c, j4, pk);
       }
       const int c16 = c + ((kpad - c) & 32);
       if (c16 < kpad) {
@@ -912,6 +933,7 @@ __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int
         if (c16 + 16 > k) slab_mask<2>(v, c16, j4, k);
         slab_exp<2>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
         slab_st_p8(pc + (c16 - c) / 2, pk);
+        bc_store_p<2, kStoreP>(g0, g1, c16, j4, pk);
       }
       tmem_wait_st();
     }
@@ -1143,7 +1165,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         t0 = row4_max(t0) * ce;
         t1 = row4_max(t1) * ce;
       }
-      bc_slab_exp(s_col, p.k, kpad, j4, wide, ce, -t0, -t1, l0, l1, ok, bars->p_chunk[g]);
+      if constexpr (kStats) {
+        uint32_t* g0 = q0 + r0 < p.N ? reinterpret_cast<uint32_t*>(
+                                           p.stats.p + (bh * p.N + q0 + r0) * (long long)kpad)
+                                     : nullptr;
+        uint32_t* g1 = q0 + r1 < p.N ? reinterpret_cast<uint32_t*>(
+                                           p.stats.p + (bh * p.N + q0 + r1) * (long long)kpad)
+                                     : nullptr;
+        bc_slab_exp<true>(s_col, p.k, kpad, j4, wide, ce, -t0, -t1, l0, l1, ok, bars->p_chunk[g],
+                          g0, g1);
+      } else {
+        bc_slab_exp(s_col, p.k, kpad, j4, wide, ce, -t0, -t1, l0, l1, ok, bars->p_chunk[g]);
+      }
       const float sum0 = row4_sum(l0), sum1 = row4_sum(l1);
       const float inv0 = 1.f / sum0, inv1 = 1.f / sum1;
       // epilogue: O = (P V_A) / l -> bf16 -> swizzled staging tile -> TMA store
