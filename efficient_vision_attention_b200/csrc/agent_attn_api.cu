@@ -177,22 +177,25 @@ int validate_grid(int N, int grid_h, int grid_w, int pool_h, int pool_w) {
 }
 
 bool has_bias(const Problem& p) { return (p.b1 && p.b1->any()) || (p.b2 && p.b2->any()); }
-// The tensor-core kernels take the agent bias while its cell tables fit in
-// shared memory; larger grids run the biased problem on the SIMT kernels.
+// Shared memory of the B1 dense-copy builder: one agent row's row, column and
+// block terms and the grid's cell tables.
+__host__ __device__ inline size_t bias_tokens_smem_bytes(int gh, int gw, int ph, int pw) {
+  return sizeof(float) * (2 * ((size_t)gh + gw) + (size_t)ph * pw);
+}
+constexpr size_t kBiasSmemMax = 160 * 1024;
+// The tensor-core kernels take the agent bias through dense copies while the
+// builder's tables fit in shared memory (grid_h + grid_w up to about 20000);
+// larger grids run the biased problem on the SIMT kernels.
 bool use_tensor_cores(const Problem& p) {
   if (p.force_simt || p.dtype != AA_BF16 || !tc_supported(p.d, p.k)) return false;
-  return !has_bias(p) || (long long)p.grid_h + p.grid_w <= tc::kBiasGridMax;
+  return !has_bias(p) ||
+         bias_tokens_smem_bytes(p.grid_h, p.grid_w, p.pool_h, p.pool_w) <= kBiasSmemMax;
 }
 
-tc::BiasParams tc_bias(const Problem& p, const AgentBiasRef* b) {
-  tc::BiasParams r{nullptr, nullptr, nullptr, p.grid_h, p.grid_w, p.pool_h, p.pool_w, 0};
-  if (b) {
-    r.row = b->row;
-    r.col = b->col;
-    r.block = b->block;
-  }
-  return r;
-}
+// Row lengths of the tensor-core kernels' dense bias copies: B1 [H][k][ld]
+// (tokens, 16-byte rows), B2 [H][N][ld] (agents, k rounded up to 16).
+int bias_ld_b1(const Problem& p) { return (p.N + 7) & ~7; }
+int bias_ld_b2(const Problem& p) { return (p.k + 15) & ~15; }
 
 void set_bias(SimtAttendArgs& a, const Problem& p, const AgentBiasRef* b, bool tok_is_col) {
   if (!b || !b->any()) return;
@@ -210,7 +213,7 @@ void set_bias(SimtAttendArgs& a, const Problem& p, const AgentBiasRef* b, bool t
 // Scratch layout.  Every region starts on a 256-byte boundary.
 struct Scratch {
   size_t a_off, va_off, pu_off, pml_off, total;
-  size_t b2t_off;            // agent-contiguous copy of B2's components (tensor-core bias)
+  size_t b1d_off, b2d_off;   // dense fp16 copies of B1 and B2 (tensor-core bias)
   SplitPlan plan;
   int simt_row_blocks;
   int simt_cols_per_split;
@@ -247,26 +250,150 @@ void plan_scratch(const Problem& p, int sm_count, Scratch* s) {
   off += round256((size_t)BH * s->plan.slots * p.k * p.d * sizeof(float));
   s->pml_off = off;
   off += round256((size_t)BH * s->plan.slots * p.k * 2 * sizeof(float));
-  s->b2t_off = off;
-  if (use_tensor_cores(p) && p.b2 && p.b2->any()) {
-    const size_t kp = (size_t)((p.k + 15) & ~15);
-    off += round256((size_t)p.H * ((size_t)p.grid_h + p.grid_w + (size_t)p.pool_h * p.pool_w) *
-                    kp * sizeof(float));
-  }
+  s->b1d_off = off;
+  if (use_tensor_cores(p) && p.b1 && p.b1->any())
+    off += round256((size_t)p.H * p.k * bias_ld_b1(p) * sizeof(__half));
+  s->b2d_off = off;
+  if (use_tensor_cores(p) && p.b2 && p.b2->any())
+    off += round256((size_t)p.H * p.N * bias_ld_b2(p) * sizeof(__half));
   s->total = off;
 }
 
-// B2's components [H][k][L] -> [H][L][kp] (agents contiguous, kp = k rounded
-// up to 16, zero padding), so a query row of the tensor-core broadcast reads
-// its agents' bias as coalesced float2 runs.  Thread per destination element.
-__global__ void bias_transpose_kernel(const float* __restrict__ src, float* __restrict__ dst,
-                                      int H, int k, int L, int kp) {
-  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= (long long)H * L * kp) return;
-  const int a = (int)(e % kp);
-  const long long hl = e / kp;
-  const int l = (int)(hl % L), h = (int)(hl / L);
-  dst[e] = a < k ? src[((long long)h * k + a) * L + l] : 0.f;
+// Dense agent bias for the tensor-core kernels: (row + col + block) * log2(e)
+// as fp16, saturated to the largest finite value, for agent a and grid token
+// n = (y, x) of head h, the block term from the floor-partition cell
+// (floor(y pool_h / grid_h), floor(x pool_w / grid_w)).
+//   bias_dense_tokens_kernel: B1 [H][k][ld] (ld >= N, zero for n >= N);
+//   bias_dense_agents_kernel: B2 [H][N][ld] (ld = k rounded up to 16, zero
+//                             for a >= k).
+// Both read the components along their token axis (coalesced) and write
+// whole rows of the dense copy.  fits32: every index product (grid side x
+// pool side, the thread count) is below 2^31, so 32-bit divisions suffice.
+__device__ __forceinline__ float bias_sum(const AgentBiasRef& b, long long ha, int y, int x,
+                                          long long cell, int gh, int gw, long long n_cells) {
+  float s = 0.f;
+  if (b.row) s += __ldg(b.row + ha * gh + y);
+  if (b.col) s += __ldg(b.col + ha * gw + x);
+  if (b.block) s += __ldg(b.block + ha * n_cells + cell);
+  return s;
+}
+__device__ __forceinline__ float bias_logit(float v) {
+  return fminf(fmaxf(v * kLog2e, -65504.f), 65504.f);
+}
+
+__device__ __forceinline__ long long floor_div(long long a, int b, bool fits32) {
+  return fits32 ? (long long)((int)a / b) : a / b;
+}
+
+// Block per agent row r = h k + a (grid-stride over the rows), 256 threads:
+// the row's components (row terms [grid_h], column terms [grid_w], block
+// terms [pool_h * pool_w]) are staged in shared memory beside the cell
+// tables (cell row offset cy * pool_w per grid row, cell column per grid
+// column), then each thread writes token pairs 512 apart, tracking (y, x)
+// by adding the stride's quotient and remainder (no division per token).
+__global__ void __launch_bounds__(256) bias_dense_tokens_kernel(AgentBiasRef b,
+                                                                __half* __restrict__ out, int H,
+                                                                int k, int N, int gh, int gw,
+                                                                int ph, int pw, int ld,
+                                                                bool fits32) {
+  extern __shared__ float bsm[];
+  const int n_cells = ph * pw;
+  float* s_row = bsm;
+  float* s_col = s_row + gh;
+  float* s_blk = s_col + gw;
+  int* s_cyo = reinterpret_cast<int*>(s_blk + n_cells);
+  int* s_cx = s_cyo + gh;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < gh; i += blockDim.x)
+    s_cyo[i] = (int)floor_div((long long)i * ph, gh, fits32) * pw;
+  for (int i = tid; i < gw; i += blockDim.x) s_cx[i] = (int)floor_div((long long)i * pw, gw, fits32);
+  const int step = 2 * blockDim.x;           // tokens between a thread's pairs
+  const int qy = step / gw, qx = step - qy * gw;
+  const int y0 = (2 * tid) / gw, x0 = 2 * tid - y0 * gw;
+  const long long rows = (long long)H * k;
+  for (long long r = blockIdx.x; r < rows; r += gridDim.x) {
+    __syncthreads();                         // the previous row's terms are read
+    for (int i = tid; i < gh; i += blockDim.x) s_row[i] = b.row ? __ldg(b.row + r * gh + i) : 0.f;
+    for (int i = tid; i < gw; i += blockDim.x) s_col[i] = b.col ? __ldg(b.col + r * gw + i) : 0.f;
+    for (int i = tid; i < n_cells; i += blockDim.x)
+      s_blk[i] = b.block ? __ldg(b.block + r * n_cells + i) : 0.f;
+    __syncthreads();
+    __half2* o = reinterpret_cast<__half2*>(out + r * ld);
+    int y = y0, x = x0;
+    for (int n = 2 * tid; n < ld; n += step) {
+      float v0 = 0.f, v1 = 0.f;
+      if (n < N) v0 = s_row[y] + s_col[x] + s_blk[s_cyo[y] + s_cx[x]];
+      int x1 = x + 1, y1 = y;
+      if (x1 == gw) {
+        x1 = 0;
+        ++y1;
+      }
+      if (n + 1 < N) v1 = s_row[y1] + s_col[x1] + s_blk[s_cyo[y1] + s_cx[x1]];
+      o[n / 2] = __floats2half2_rn(bias_logit(v0), bias_logit(v1));
+      x += qx;
+      y += qy;
+      if (x >= gw) {
+        x -= gw;
+        ++y;
+      }
+    }
+  }
+}
+
+// Block per (head, 32 consecutive tokens), 256 threads: the tile [32 tokens]
+// [ld agents] is summed into shared memory with a warp's lanes on 32
+// consecutive tokens (row stride 257 floats: lane t of agent a hits bank
+// (t + a) % 32), then each warp writes whole token rows, lanes on agent pairs.
+constexpr int kBiasTileTokens = 32;
+constexpr int kBiasTileStride = 257;
+__global__ void __launch_bounds__(256) bias_dense_agents_kernel(AgentBiasRef b,
+                                                                __half* __restrict__ out, int H,
+                                                                int k, int N, int gh, int gw,
+                                                                int ph, int pw, int ld,
+                                                                bool fits32) {
+  __shared__ float tile[kBiasTileTokens * kBiasTileStride];
+  const int tiles = (N + kBiasTileTokens - 1) / kBiasTileTokens;
+  const int h = blockIdx.x / tiles;
+  const int n0 = (blockIdx.x - h * tiles) * kBiasTileTokens;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int n = n0 + tx;
+  const bool in = n < N;
+  int y = 0, x = 0;
+  long long cell = 0;
+  if (in) {
+    y = n / gw;
+    x = n - y * gw;
+    cell = floor_div((long long)y * ph, gh, fits32) * pw + floor_div((long long)x * pw, gw, fits32);
+  }
+  const long long n_cells = (long long)ph * pw;
+  // agents a = ty + 8 i (ld <= 256): the components' offsets advance by 8 rows
+  long long ro = ((long long)h * k + ty) * gh + y;
+  long long co = ((long long)h * k + ty) * gw + x;
+  long long bo = ((long long)h * k + ty) * n_cells + cell;
+  const long long sr = 8LL * gh, sc = 8LL * gw, sb = 8 * n_cells;
+#pragma unroll 8
+  for (int i = 0; i < 32; ++i) {
+    const int a = ty + 8 * i;
+    if (a < ld) {
+      float v = 0.f;
+      if (in && a < k) {
+        if (b.row) v += __ldg(b.row + ro);
+        if (b.col) v += __ldg(b.col + co);
+        if (b.block) v += __ldg(b.block + bo);
+      }
+      tile[tx * kBiasTileStride + a] = v;
+    }
+    ro += sr;
+    co += sc;
+    bo += sb;
+  }
+  __syncthreads();
+  for (int j = ty; j < kBiasTileTokens && n0 + j < N; j += 8) {
+    __half2* row = reinterpret_cast<__half2*>(out + ((long long)h * N + n0 + j) * ld);
+    for (int a = 2 * tx; a < ld; a += 64)
+      row[a / 2] = __floats2half2_rn(bias_logit(tile[j * kBiasTileStride + a]),
+                                     bias_logit(tile[j * kBiasTileStride + a + 1]));
+  }
 }
 
 std::mutex g_smem_attr_mutex;   // serialises raising a kernel's shared-memory limit
@@ -378,6 +505,29 @@ int launch_simt_attend(const SimtAttendArgs& args, long long BH, cudaStream_t st
   return AA_OK;
 }
 
+std::atomic<int> g_bias_tokens_smem[kMaxDevices];
+
+int launch_bias_dense(const Problem& p, const AgentBiasRef& b, __half* out, bool tokens_minor,
+                      cudaStream_t st) {
+  const long long lim = 0x7fffffffLL;
+  bool fits32 = (long long)p.grid_h * p.pool_h <= lim && (long long)p.grid_w * p.pool_w <= lim;
+  if (tokens_minor) {
+    const size_t smem = bias_tokens_smem_bytes(p.grid_h, p.grid_w, p.pool_h, p.pool_w);
+    int rc = ensure_smem(bias_dense_tokens_kernel, smem, g_bias_tokens_smem);
+    if (rc != AA_OK) return rc;
+    const long long rows = (long long)p.H * p.k;
+    bias_dense_tokens_kernel<<<(unsigned)(rows < 65535 ? rows : 65535), 256, smem, st>>>(
+        b, out, p.H, p.k, p.N, p.grid_h, p.grid_w, p.pool_h, p.pool_w, bias_ld_b1(p), fits32);
+  } else {
+    const long long blocks = (long long)p.H * ((p.N + kBiasTileTokens - 1) / kBiasTileTokens);
+    if (blocks > lim) return AA_ERR_SHAPE;
+    bias_dense_agents_kernel<<<(unsigned)blocks, 256, 0, st>>>(
+        b, out, p.H, p.k, p.N, p.grid_h, p.grid_w, p.pool_h, p.pool_w, bias_ld_b2(p), fits32);
+  }
+  AA_CUDA(cudaGetLastError());
+  return AA_OK;
+}
+
 template <typename T>
 int launch_merge(const Problem& p, const Scratch& s, char* ws, float* va_f32, T* va_lowp,
                  cudaStream_t st, bool pdl, float* ml_out = nullptr) {
@@ -399,7 +549,9 @@ int run_aggregate(const Problem& p, const Scratch& s, const AgentsRef& ag, const
                   bool pdl = false) {
   const long long qstride_h = (long long)p.N * p.d, qstride_b = qstride_h * p.H;
   if (use_tensor_cores(p)) {
-    const tc::BiasParams b1 = tc_bias(p, p.b1);
+    tc::BiasParams b1{nullptr, 0};
+    if (p.b1 && p.b1->any())
+      b1 = tc::BiasParams{reinterpret_cast<const __half*>(ws + s.b1d_off), bias_ld_b1(p)};
     cudaError_t e = tc_launch_aggregate(ag.ptr, ag.bstride, ag.hstride, k, v, p.B, p.H, p.N, p.d,
                                         p.k, p.scale * kLog2e, s.plan,
                                         reinterpret_cast<float*>(ws + s.pu_off),
@@ -437,32 +589,18 @@ int run_aggregate(const Problem& p, const Scratch& s, const AgentsRef& ag, const
 
 template <typename T>
 int run_broadcast(const Problem& p, const void* q, const AgentsRef& ag, const void* va,
-                  void* out, cudaStream_t st, bool pdl = false, float* b2t = nullptr) {
+                  void* out, cudaStream_t st, bool pdl = false,
+                  const __half* b2d = nullptr) {
   const long long qstride_h = (long long)p.N * p.d, qstride_b = qstride_h * p.H;
   const long long vstride_h = (long long)p.k * p.d, vstride_b = vstride_h * p.H;
   if (use_tensor_cores(p)) {
     int sms = 0;
     int rc = device_sm_count(&sms);
     if (rc != AA_OK) return rc;
-    tc::BiasParams b2 = tc_bias(p, p.b2);
-    if (b2.any()) {
-      if (b2t == nullptr) return AA_ERR_WORKSPACE;
-      const int kp = (p.k + 15) & ~15;
-      const int lens[3] = {p.grid_h, p.grid_w, p.pool_h * p.pool_w};
-      const float* srcs[3] = {b2.row, b2.col, b2.block};
-      float* dst = b2t;
-      const float** outs[3] = {&b2.row, &b2.col, &b2.block};
-      for (int c = 0; c < 3; ++c) {
-        if (srcs[c] == nullptr) continue;
-        const long long n = (long long)p.H * lens[c] * kp;
-        bias_transpose_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(srcs[c], dst, p.H, p.k,
-                                                                         lens[c], kp);
-        AA_CUDA(cudaGetLastError());
-        *outs[c] = dst;
-        dst += n;
-      }
-      b2.agent_minor = kp;
-      pdl = false;    // the broadcast follows the transposes, not the merge
+    tc::BiasParams b2{nullptr, 0};
+    if (p.b2 && p.b2->any()) {
+      if (b2d == nullptr) return AA_ERR_WORKSPACE;
+      b2 = tc::BiasParams{b2d, bias_ld_b2(p)};
     }
     cudaError_t e = tc_launch_broadcast(q, ag.ptr, ag.bstride, va, out, p.B, p.H, p.N, p.d, p.k,
                                         p.scale * kLog2e, sms, st, pdl, &b2);
@@ -513,6 +651,18 @@ int run_forward(const Problem& p, const Scratch& s, const void* q, const void* k
     if (e != cudaSuccess) return cuda_fail(e, "agent forward (fused small slices) launch");
     return AA_OK;
   }
+  if (use_tensor_cores(p)) {
+    // the dense bias copies, before the pool: every later kernel of the pass
+    // starts after they have completed (the pool launches without overlap)
+    if (p.b1 && p.b1->any()) {
+      int rc = launch_bias_dense(p, *p.b1, reinterpret_cast<__half*>(ws + s.b1d_off), true, st);
+      if (rc != AA_OK) return rc;
+    }
+    if (p.b2 && p.b2->any()) {
+      int rc = launch_bias_dense(p, *p.b2, reinterpret_cast<__half*>(ws + s.b2d_off), false, st);
+      if (rc != AA_OK) return rc;
+    }
+  }
   AgentsRef ag;
   const long long ahs = (long long)p.k * p.d;
   if (learnable) {
@@ -538,7 +688,7 @@ int run_forward(const Problem& p, const Scratch& s, const void* q, const void* k
                : run_aggregate<T>(p, s, ag, k, v, ws, nullptr, va_ws, st, pdl_agg);
   if (rc != AA_OK) return rc;
   return run_broadcast<T>(p, q, ag, va_ws, out, st, true,
-                          reinterpret_cast<float*>(ws + s.b2t_off));
+                          reinterpret_cast<const __half*>(ws + s.b2d_off));
 }
 
 int forward_impl(const Problem& p, const void* q, const void* k, const void* v,
@@ -1142,7 +1292,7 @@ int agent_attn_stage_aggregate_static(const void* agents, long long agents_batch
   const size_t need = s.total - s.pu_off;
   if (need > (size_t)AA_STATIC_SCRATCH_BYTES) return AA_ERR_WORKSPACE;
   Scratch r = s;
-  r.a_off = r.va_off = r.b2t_off = 0;
+  r.a_off = r.va_off = r.b1d_off = r.b2d_off = 0;
   r.pml_off = s.pml_off - s.pu_off;
   r.pu_off = 0;
   r.total = need;

@@ -64,18 +64,16 @@ constexpr int kMaxAgents = 256;
 constexpr int kAgentBufBytes = kMaxAgents * kRowBytes;   // one agent tile (all agents of a slice)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale only when the max grows by > 2^8
 
-// Agent bias in the score tiles: for agent a and grid token (y, x) of head h,
-// row[h][a][y] + col[h][a][x] + block[h][a][cell(y, x)] (fp32 components, any
-// may be null), cell = cell_y[y] * pool_w + cell_x[x] from tables the kernel
-// builds in shared memory (grid_h + grid_w <= kBiasGridMax).
-constexpr int kBiasGridMax = 4096;
+// Agent bias in the score tiles: a dense fp16 copy of B * log2(e) (logits in
+// log2 units), made per call from the row, column and block components.  B1
+// (aggregation): [H][k][ld] with the tokens contiguous (ld >= N, even, zero
+// past N); B2 (broadcast): [H][N][ld] with the agents contiguous (ld = k
+// rounded up to 16, zero past k).  A thread's score column pair reads its two
+// logits as one 32-bit word.
 struct BiasParams {
-  const float* row;
-  const float* col;
-  const float* block;
-  int grid_h, grid_w, pool_h, pool_w;
-  int agent_minor;           // 0: components [H][k][L]; kp > 0: [H][L][kp] (agents contiguous)
-  __host__ __device__ bool any() const { return row || col || block; }
+  const __half* dense;       // null: no bias
+  int ld;                    // row length of the dense copy, in elements
+  __host__ __device__ bool any() const { return dense != nullptr; }
 };
 
 struct AggParams {
@@ -166,64 +164,15 @@ __device__ __forceinline__ void drain_commits(uint64_t* bar) {
 }
 
 // ============================================================== aggregation
-// Cell tables of the agent bias: cell_y[grid_h], cell_x[grid_w] as int16.
-__device__ __forceinline__ void build_cell_tables(int16_t* cy, int16_t* cx, const BiasParams& b,
-                                                  int tid, int nthreads) {
-  for (int i = tid; i < b.grid_h; i += nthreads)
-    cy[i] = (int16_t)(((long long)i * b.pool_h) / b.grid_h);
-  for (int i = tid; i < b.grid_w; i += nthreads)
-    cx[i] = (int16_t)(((long long)i * b.pool_w) / b.grid_w);
-}
-
-// Per-agent-row bases of the three components (null where a component is absent).
-struct BiasRowPtrs {
-  const float* row;
-  const float* col;
-  const float* block;
-};
-__device__ __forceinline__ BiasRowPtrs bias_row_ptrs(const BiasParams& b, long long ra) {
-  BiasRowPtrs r;
-  r.row = b.row ? b.row + ra * b.grid_h : nullptr;
-  r.col = b.col ? b.col + ra * b.grid_w : nullptr;
-  r.block = b.block ? b.block + ra * ((long long)b.pool_h * b.pool_w) : nullptr;
-  return r;
-}
-// Bias of one agent row for the token pair (y, x), (y, x+1) of one grid row:
-// one row term, the two column terms as one float2 (8-byte aligned), two cells.
-__device__ __forceinline__ float2 agent_bias_pair(const BiasRowPtrs& r, const BiasParams& b,
-                                                  const int16_t* cy, const int16_t* cx, int y,
-                                                  int x) {
-  float2 v = make_float2(0.f, 0.f);
-  if (r.row) {
-    const float t = __ldg(r.row + y);
-    v.x = t;
-    v.y = t;
-  }
-  if (r.col) {
-    const float2 t = __ldg(reinterpret_cast<const float2*>(r.col + x));
-    v.x += t.x;
-    v.y += t.y;
-  }
-  if (r.block) {
-    const float* br = r.block + (int)cy[y] * b.pool_w;
-    v.x += __ldg(br + cx[x]);
-    v.y += __ldg(br + cx[x + 1]);
-  }
-  return v;
-}
-__device__ __forceinline__ float agent_bias_one(const BiasRowPtrs& r, const BiasParams& b,
-                                                const int16_t* cy, const int16_t* cx, int y,
-                                                int x) {
-  float v = 0.f;
-  if (r.row) v += __ldg(r.row + y);
-  if (r.col) v += __ldg(r.col + x);
-  if (r.block) v += __ldg(r.block + (int)cy[y] * b.pool_w + cx[x]);
-  return v;
+// The two fp16 logits of a bias word as floats.
+__device__ __forceinline__ float2 bias_pair(uint32_t w) {
+  __half2 h;
+  memcpy(&h, &w, sizeof(h));
+  return __half22float2(h);
 }
 
 constexpr size_t kAggSmemBytes = 1024 + 2 * (size_t)kAgentBufBytes +
-                                 2 * (size_t)kAggStages * kKTileBytes + sizeof(AggBars) +
-                                 2 * (size_t)kBiasGridMax;
+                                 2 * (size_t)kAggStages * kKTileBytes + sizeof(AggBars);
 
 // kBias: the agent bias B1 is added to the score tiles (a separate
 // instantiation, so the unbiased kernel carries none of its code).
@@ -239,8 +188,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK = sA + 2 * kAgentBufBytes;
   uint8_t* sV = sK + kAggStages * kKTileBytes;
   AggBars* bars = reinterpret_cast<AggBars*>(sV + kAggStages * kKTileBytes);
-  int16_t* cell_y = reinterpret_cast<int16_t*>(reinterpret_cast<uint8_t*>(bars) + sizeof(AggBars));
-  int16_t* cell_x = cell_y + p.bias.grid_h;
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -282,7 +229,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   constexpr bool biased = kBias;
-  if (biased) build_cell_tables(cell_y, cell_x, p.bias, threadIdx.x, blockDim.x);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -458,6 +404,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = J % kSBuf;
         const uint32_t s_col = tmem + slab_off + g * 256 + b * 64;
         const int valid = min(kKeyTile, p.N - (int)(t + i - bh * tps) * kKeyTile);
+        // the tile's B1 logits of this thread's column pairs (two fp16 per
+        // word), loaded before the wait for the scores so that their latency
+        // overlaps it; columns past the slice (and padding agents) add 0
+        uint32_t bw0[8], bw1[8];
+        if constexpr (kBias) {
+          const int n0 = (int)(t + i - bh * tps) * kKeyTile;
+          const long long ra0 = (long long)(bh % p.H) * p.k + row_base + r0;
+          const bool in0 = ok && row_base + r0 < p.k, in1 = ok && row_base + r1 < p.k;
+          const uint32_t* w0p =
+              reinterpret_cast<const uint32_t*>(p.bias.dense + ra0 * p.bias.ld + n0);
+          const uint32_t* w1p = w0p + 4LL * p.bias.ld;     // 8 agent rows further
+#pragma unroll
+          for (int g8 = 0; g8 < 8; ++g8) {
+            const int col = 8 * g8 + 2 * j4;
+            bw0[g8] = (in0 && col < valid) ? __ldg(w0p + col / 2) : 0u;
+            bw1[g8] = (in1 && col < valid) ? __ldg(w1p + col / 2) : 0u;
+          }
+        }
         if (ok) ok = warp_wait(&bars->s_full[g][b], (uint32_t)(J / kSBuf) & 1, abort);
         tc_fence_after();
         // A tile's scores are only written after the P V of the buffer's
@@ -469,101 +433,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           slab_ld64(s_col, v);
           if (valid < kKeyTile) slab_mask<8>(v, 0, j4, valid);   // ragged last tile
           if (biased) {
-            // scores become log2-unit logits: S*c + bias*log2(e), then ce = 1.
-            // The tile's first key is split into (y, x) once.  A thread's
-            // columns come in pairs (x, x+1); on an even-width grid a pair
-            // starts at an even x, so it never straddles two grid rows and
-            // shares the row term and the cell row (the column terms as one
-            // float2 when the column component is 8-byte aligned).
-            const int n0 = (int)(t + i - bh * tps) * kKeyTile;
-            const int h = (int)(bh % p.H);
-            const long long ra0 = (long long)h * p.k + row_base + r0;
-            const bool in0 = row_base + r0 < p.k, in1 = row_base + r1 < p.k;
-            const BiasRowPtrs br0 = bias_row_ptrs(p.bias, ra0);
-            const BiasRowPtrs br1 = bias_row_ptrs(p.bias, ra0 + 8);
-            const int gw = p.bias.grid_w;
-            const int ty0 = n0 / gw, tx0 = n0 - ty0 * gw;
-            const bool pairs = (gw & 1) == 0 && (reinterpret_cast<uintptr_t>(p.bias.col) & 7u) == 0;
-            if (pairs && tx0 + kKeyTile <= gw) {
-              // the whole tile lies in grid row ty0: each agent row's row term
-              // and cell row are loaded once; a pair's block term once when
-              // both of its tokens fall in the same cell
-              const int cyo = (int)cell_y[ty0] * p.bias.pool_w;
-              const float rw0 = (in0 && br0.row) ? __ldg(br0.row + ty0) : 0.f;
-              const float rw1 = (in1 && br1.row) ? __ldg(br1.row + ty0) : 0.f;
-#pragma unroll
-              for (int g8 = 0; g8 < 8; ++g8) {
-                const int col = 8 * g8 + 2 * j4;
-                if (col >= valid) continue;
-                const int x = tx0 + col;
-                float2 b0 = make_float2(rw0, rw0), b1 = make_float2(rw1, rw1);
-                if (p.bias.col) {
-                  if (in0) {
-                    const float2 t0 = __ldg(reinterpret_cast<const float2*>(br0.col + x));
-                    b0.x += t0.x;
-                    b0.y += t0.y;
-                  }
-                  if (in1) {
-                    const float2 t1 = __ldg(reinterpret_cast<const float2*>(br1.col + x));
-                    b1.x += t1.x;
-                    b1.y += t1.y;
-                  }
-                }
-                if (p.bias.block) {
-                  const int c0 = cyo + cell_x[x], c1 = cyo + cell_x[x + 1];
-                  if (in0) {
-                    const float k0 = __ldg(br0.block + c0);
-                    b0.x += k0;
-                    b0.y += (c1 == c0) ? k0 : __ldg(br0.block + c1);
-                  }
-                  if (in1) {
-                    const float k1 = __ldg(br1.block + c0);
-                    b1.x += k1;
-                    b1.y += (c1 == c0) ? k1 : __ldg(br1.block + c1);
-                  }
-                }
-                v[4 * g8] = fmaf(v[4 * g8], p.c, b0.x * kLog2e);
-                v[4 * g8 + 1] = fmaf(v[4 * g8 + 1], p.c, b0.y * kLog2e);
-                v[4 * g8 + 2] = fmaf(v[4 * g8 + 2], p.c, b1.x * kLog2e);
-                v[4 * g8 + 3] = fmaf(v[4 * g8 + 3], p.c, b1.y * kLog2e);
-              }
-            } else
+            // scores become log2-unit logits S*c + B1*log2(e), then ce = 1
 #pragma unroll
             for (int g8 = 0; g8 < 8; ++g8) {
-              const int col = 8 * g8 + 2 * j4;
-              if (col >= valid) continue;
-              int x = tx0 + col, y = ty0;
-              if (x >= gw) {
-                const int q = x / gw;
-                y += q;
-                x -= q * gw;
-              }
-              if (pairs) {   // valid is even here (N = grid_h * gw is even)
-                const float2 b0 = in0 ? agent_bias_pair(br0, p.bias, cell_y, cell_x, y, x)
-                                      : make_float2(0.f, 0.f);
-                const float2 b1 = in1 ? agent_bias_pair(br1, p.bias, cell_y, cell_x, y, x)
-                                      : make_float2(0.f, 0.f);
-                v[4 * g8] = fmaf(v[4 * g8], p.c, b0.x * kLog2e);
-                v[4 * g8 + 1] = fmaf(v[4 * g8 + 1], p.c, b0.y * kLog2e);
-                v[4 * g8 + 2] = fmaf(v[4 * g8 + 2], p.c, b1.x * kLog2e);
-                v[4 * g8 + 3] = fmaf(v[4 * g8 + 3], p.c, b1.y * kLog2e);
-              } else {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                  if (col + e >= valid) continue;
-                  int xe = x + e, ye = y;
-                  if (xe >= gw) {   // x < gw, so x + 1 wraps at most once
-                    xe -= gw;
-                    ++ye;
-                  }
-                  float& va = v[4 * g8 + e];
-                  float& vb = v[4 * g8 + 2 + e];
-                  va = fmaf(va, p.c,
-                            in0 ? agent_bias_one(br0, p.bias, cell_y, cell_x, ye, xe) * kLog2e : 0.f);
-                  vb = fmaf(vb, p.c,
-                            in1 ? agent_bias_one(br1, p.bias, cell_y, cell_x, ye, xe) * kLog2e : 0.f);
-                }
-              }
+              const float2 b0 = bias_pair(bw0[g8]), b1 = bias_pair(bw1[g8]);
+              v[4 * g8] = fmaf(v[4 * g8], p.c, b0.x);
+              v[4 * g8 + 1] = fmaf(v[4 * g8 + 1], p.c, b0.y);
+              v[4 * g8 + 2] = fmaf(v[4 * g8 + 2], p.c, b1.x);
+              v[4 * g8 + 3] = fmaf(v[4 * g8 + 3], p.c, b1.y);
             }
           }
           const float ce = biased ? 1.f : p.c;
@@ -733,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ================================================================ broadcast
 constexpr size_t kBcSmemBytes = 1024 + 2 * (size_t)kMaxAgents * kRowBytes +
                                 (size_t)kBcStages * kQTileBytes + 2 * (size_t)kQTileBytes +
-                                sizeof(BcBars) + 2 * (size_t)kBiasGridMax;
+                                sizeof(BcBars);
 
 // Row maxima of a slab's two rows (this thread's columns) over score columns
 // [0, kpad), columns >= k masked; 64 columns per TMEM load, then 32 and 16.
@@ -762,102 +639,78 @@ __device__ __forceinline__ void bc_slab_max(uint32_t s_col, int k, int kpad, int
   }
 }
 
-// The agent bias of a slab's two query rows: token (y, x) and cell per row.
+// The B2 logits of a slab's two query rows: the rows of the dense copy as
+// 32-bit words (two fp16 agents each), null for a row past the slice.
 struct BcRowBias {
-  int y0, x0, cell0, y1, x1, cell1;
-  bool in0, in1;             // the row is a real token
-  long long h;               // head
-  long long hk;              // h * k: agent rows of this head
+  const uint32_t* w0;
+  const uint32_t* w1;
 };
 
-// Scores of a block (16x256b layout, first column c) become log2-unit logits
-// S*c + B2*log2(e); masked columns stay -inf.  With the agent-contiguous
-// component layout a row's two agents of a column pair come as one float2.
-__device__ __forceinline__ float2 ld_pair(const float* p) {
-  return __ldg(reinterpret_cast<const float2*>(p));
-}
+// The words of a 16x256b register block (first column c): agents
+// c + 8 g + 2 j4 and the next one.
 template <int R>
-__device__ __forceinline__ void bc_bias_block(float (&v)[4 * R], int c, int k, int j4, float cs,
-                                              const BiasParams& b, const BcRowBias& rb) {
-  if (b.agent_minor > 0) {
-    const long long kp = b.agent_minor;
-    const long long h = rb.h;
-    const long long nb = (long long)b.pool_h * b.pool_w;
-#pragma unroll
-    for (int g = 0; g < R; ++g) {
-      const int a = c + 8 * g + 2 * j4;       // even; a + 1 < kp (zero padding)
-      float2 b0 = make_float2(0.f, 0.f), b1 = make_float2(0.f, 0.f);
-      if (rb.in0) {
-        if (b.row) { const float2 t = ld_pair(b.row + (h * b.grid_h + rb.y0) * kp + a); b0.x += t.x; b0.y += t.y; }
-        if (b.col) { const float2 t = ld_pair(b.col + (h * b.grid_w + rb.x0) * kp + a); b0.x += t.x; b0.y += t.y; }
-        if (b.block) { const float2 t = ld_pair(b.block + (h * nb + rb.cell0) * kp + a); b0.x += t.x; b0.y += t.y; }
-      }
-      if (rb.in1) {
-        if (b.row) { const float2 t = ld_pair(b.row + (h * b.grid_h + rb.y1) * kp + a); b1.x += t.x; b1.y += t.y; }
-        if (b.col) { const float2 t = ld_pair(b.col + (h * b.grid_w + rb.x1) * kp + a); b1.x += t.x; b1.y += t.y; }
-        if (b.block) { const float2 t = ld_pair(b.block + (h * nb + rb.cell1) * kp + a); b1.x += t.x; b1.y += t.y; }
-      }
-      // columns >= k keep their -inf (their fma stays -inf as cs > 0)
-      v[4 * g] = fmaf(v[4 * g], cs, b0.x * kLog2e);
-      v[4 * g + 1] = fmaf(v[4 * g + 1], cs, b0.y * kLog2e);
-      v[4 * g + 2] = fmaf(v[4 * g + 2], cs, b1.x * kLog2e);
-      v[4 * g + 3] = fmaf(v[4 * g + 3], cs, b1.y * kLog2e);
-    }
-    return;
-  }
+__device__ __forceinline__ void bc_bias_load(uint32_t (&w0)[R], uint32_t (&w1)[R], int c, int j4,
+                                             const BcRowBias& rb) {
 #pragma unroll
   for (int g = 0; g < R; ++g) {
+    const int w = (c + 8 * g) / 2 + j4;
+    w0[g] = rb.w0 ? __ldg(rb.w0 + w) : 0u;
+    w1[g] = rb.w1 ? __ldg(rb.w1 + w) : 0u;
+  }
+}
+// Scores of the block become log2-unit logits S*c + B2*log2(e); masked
+// columns stay -inf (their bias words are the zero padding).
+template <int R>
+__device__ __forceinline__ void bc_bias_add(float (&v)[4 * R], const uint32_t (&w0)[R],
+                                            const uint32_t (&w1)[R], float cs) {
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int a = c + 8 * g + 2 * j4 + e;
-      if (a >= k) continue;
-      const long long ra = rb.hk + a;
-      float b0 = 0.f, b1 = 0.f;
-      if (rb.in0) {
-        if (b.row) b0 += __ldg(b.row + ra * b.grid_h + rb.y0);
-        if (b.col) b0 += __ldg(b.col + ra * b.grid_w + rb.x0);
-        if (b.block) b0 += __ldg(b.block + ra * ((long long)b.pool_h * b.pool_w) + rb.cell0);
-      }
-      if (rb.in1) {
-        if (b.row) b1 += __ldg(b.row + ra * b.grid_h + rb.y1);
-        if (b.col) b1 += __ldg(b.col + ra * b.grid_w + rb.x1);
-        if (b.block) b1 += __ldg(b.block + ra * ((long long)b.pool_h * b.pool_w) + rb.cell1);
-      }
-      v[4 * g + e] = fmaf(v[4 * g + e], cs, b0 * kLog2e);
-      v[4 * g + 2 + e] = fmaf(v[4 * g + 2 + e], cs, b1 * kLog2e);
-    }
+  for (int g = 0; g < R; ++g) {
+    const float2 b0 = bias_pair(w0[g]), b1 = bias_pair(w1[g]);
+    v[4 * g] = fmaf(v[4 * g], cs, b0.x);
+    v[4 * g + 1] = fmaf(v[4 * g + 1], cs, b0.y);
+    v[4 * g + 2] = fmaf(v[4 * g + 2], cs, b1.x);
+    v[4 * g + 3] = fmaf(v[4 * g + 3], cs, b1.y);
   }
 }
 
 // Biased max pass: adds B2 to every score, writes the logits back over the
 // scores (the exponential pass then uses scale 1) and returns the row maxima.
+// w0, w1 hold the first 64-column block's bias words (loaded by the caller
+// before it waited for the scores, when kpad >= 64); each later block's words
+// are requested as soon as the previous block has used its own.
 __device__ __forceinline__ void bc_slab_bias_max(uint32_t s_col, int k, int kpad, int j4,
-                                                 float cs, const BiasParams& b,
-                                                 const BcRowBias& rb, float& t0, float& t1) {
+                                                 float cs, const BcRowBias& rb, float& t0,
+                                                 float& t1, uint32_t (&w0)[8],
+                                                 uint32_t (&w1)[8]) {
   int c = 0;
 #pragma unroll 1
   for (; c + 64 <= kpad; c += 64) {
     float v[32];
     slab_ld64(s_col + c, v);
     if (c + 64 > k) slab_mask<8>(v, c, j4, k);
-    bc_bias_block<8>(v, c, k, j4, cs, b, rb);
+    bc_bias_add<8>(v, w0, w1, cs);
+    if (c + 128 <= kpad) bc_bias_load<8>(w0, w1, c + 64, j4, rb);
     slab_st64(s_col + c, v);
     slab_max<8>(v, t0, t1);
   }
   if (c + 32 <= kpad) {
+    uint32_t u0[4], u1[4];
+    bc_bias_load<4>(u0, u1, c, j4, rb);
     float v[16];
     slab_ld32(s_col + c, v);
     if (c + 32 > k) slab_mask<4>(v, c, j4, k);
-    bc_bias_block<4>(v, c, k, j4, cs, b, rb);
+    bc_bias_add<4>(v, u0, u1, cs);
     slab_st32(s_col + c, v);
     slab_max<4>(v, t0, t1);
     c += 32;
   }
   if (c < kpad) {
+    uint32_t u0[2], u1[2];
+    bc_bias_load<2>(u0, u1, c, j4, rb);
     float v[8];
     slab_ld16(s_col + c, v);
     if (c + 16 > k) slab_mask<2>(v, c, j4, k);
-    bc_bias_block<2>(v, c, k, j4, cs, b, rb);
+    bc_bias_add<2>(v, u0, u1, cs);
     slab_st16(s_col + c, v);
     slab_max<2>(v, t0, t1);
   }
@@ -958,8 +811,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = sVA + kMaxAgents * kRowBytes;
   uint8_t* sO = sQ + kBcStages * kQTileBytes;
   BcBars* bars = reinterpret_cast<BcBars*>(sO + 2 * kQTileBytes);
-  int16_t* cell_y = reinterpret_cast<int16_t*>(reinterpret_cast<uint8_t*>(bars) + sizeof(BcBars));
-  int16_t* cell_x = cell_y + p.bias.grid_h;
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1000,7 +851,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
-  if (kBias) build_cell_tables(cell_y, cell_x, p.bias, threadIdx.x, blockDim.x);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1140,25 +990,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long t = t_begin + j;
       const long long bh = t / tps;
       const int q0 = (int)(t - bh * tps) * kQTile;
+      // biased: the rows' B2 words of the first 64 agents are requested
+      // before the wait, so that their latency overlaps it
+      BcRowBias rb;
+      uint32_t bw0[8], bw1[8];
+      if constexpr (kBias) {
+        const __half* hb = p.bias.dense + (long long)(bh % p.H) * p.N * p.bias.ld;
+        rb.w0 = q0 + r0 < p.N
+                    ? reinterpret_cast<const uint32_t*>(hb + (long long)(q0 + r0) * p.bias.ld)
+                    : nullptr;
+        rb.w1 = q0 + r1 < p.N
+                    ? reinterpret_cast<const uint32_t*>(hb + (long long)(q0 + r1) * p.bias.ld)
+                    : nullptr;
+        if (kpad >= 64) bc_bias_load<8>(bw0, bw1, 0, j4, rb);
+      }
       if (ok) ok = warp_wait(&bars->s_full[g], u & 1, abort);
       tc_fence_after();
       float l0 = 0.f, l1 = 0.f, t0 = -INFINITY, t1 = -INFINITY;
       const float ce = kBias ? 1.f : p.c;     // biased scores are already logits
       if (ok) {
         if constexpr (kBias) {
-          BcRowBias rb;
-          const int n0 = q0 + r0, n1 = q0 + r1;
-          rb.in0 = n0 < p.N;
-          rb.in1 = n1 < p.N;
-          rb.y0 = rb.in0 ? n0 / p.bias.grid_w : 0;
-          rb.x0 = rb.in0 ? n0 - rb.y0 * p.bias.grid_w : 0;
-          rb.y1 = rb.in1 ? n1 / p.bias.grid_w : 0;
-          rb.x1 = rb.in1 ? n1 - rb.y1 * p.bias.grid_w : 0;
-          rb.cell0 = (int)cell_y[rb.y0] * p.bias.pool_w + cell_x[rb.x0];
-          rb.cell1 = (int)cell_y[rb.y1] * p.bias.pool_w + cell_x[rb.x1];
-          rb.h = (long long)(bh % p.H);
-          rb.hk = rb.h * p.k;
-          bc_slab_bias_max(s_col, p.k, kpad, j4, p.c, p.bias, rb, t0, t1);
+          bc_slab_bias_max(s_col, p.k, kpad, j4, p.c, rb, t0, t1, bw0, bw1);
         } else {
           bc_slab_max(s_col, p.k, kpad, j4, t0, t1);
         }
@@ -1414,7 +1266,7 @@ inline cudaError_t tc_launch_aggregate(const void* agents, long long a_bstride, 
   p.slots = plan.slots;
   p.part_u = part_u;
   p.part_ml = part_ml;
-  p.bias = bias ? *bias : BiasParams{nullptr, nullptr, nullptr, 1, 1, 1, 1, 0};
+  p.bias = bias ? *bias : BiasParams{nullptr, 0};
   return launch_kernel(biased ? agent_aggregate_tc_kernel<true> : agent_aggregate_tc_kernel<false>,
                        dim3(plan.ctas), dim3(kThreads), kAggSmemBytes,
                        st, pdl, mk, mv, ma, a_sets, p);
@@ -1455,7 +1307,7 @@ inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long l
   p.tiles_per_slice = (N + kQTile - 1) / kQTile;
   p.total_tiles = BH * p.tiles_per_slice;
   p.ctas = (int)(p.total_tiles < sm_count ? p.total_tiles : sm_count);
-  p.bias = bias ? *bias : BiasParams{nullptr, nullptr, nullptr, 1, 1, 1, 1, 0};
+  p.bias = bias ? *bias : BiasParams{nullptr, 0};
   p.stats = with_stats ? *stats : BcStats{nullptr, nullptr, nullptr, nullptr};
   return launch_kernel(biased       ? agent_broadcast_tc_kernel<true>
                        : with_stats ? agent_broadcast_tc_kernel<false, true>

@@ -196,10 +196,12 @@ AA_API int agent_attn_stage_aggregate_static(const void* agents, long long agent
  * Components are fp32 device buffers shared over the batch (4-byte aligned):
  *   *_row [H, k, grid_h], *_col [H, k, grid_w], *_block [H, k, pool_h*pool_w],
  * k = pool_h*pool_w; each may be NULL (contributes zero).  Other arguments as
- * in agent_attn_forward.  bf16 problems add the bias inside the tensor-core
- * score tiles (grid_h + grid_w <= 4096); fp32 problems and larger grids run on
- * the SIMT kernels.  Scratch for a transposed copy of B2's components comes
- * from the library's stream-ordered pool. */
+ * in agent_attn_forward.  bf16 problems first build a dense copy of each bias
+ * (B * log2(e) as fp16: 11-bit significands, values saturated at +-65504,
+ * i.e. |B| up to about 45000) and add it inside the tensor-core score tiles;
+ * fp32 problems add the fp32 components on the SIMT kernels.  Scratch for the
+ * dense copies (2 bytes per agent and token and head, for each of B1 and B2)
+ * comes from the library's stream-ordered pool. */
 AA_API int agent_attn_forward_bias(const void* q, const void* k, const void* v,
                                    const void* agents_or_null, const float* b1_row,
                                    const float* b1_col, const float* b1_block,

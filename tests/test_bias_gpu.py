@@ -59,16 +59,21 @@ def test_bias_matches_oracle(dtype, B, H, gh, gw, ph, pw, d, drop1, drop2):
     assert_close(f64(out), ref, dtype, "biased O")
 
 
-def test_bias_admitting_one_token_selects_its_value_on_gpu():
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_bias_admitting_one_token_selects_its_value_on_gpu(dtype):
+    """B1 = -1e4 everywhere but one token: every agent's V_A is that token's
+    V row, and so is every output row (bf16: the -1e4 components sum to
+    -2e4, inside the dense copy's fp16 range)."""
     gh, gw, ph, pw, d, ys, xs = 9, 7, 3, 3, 16, 4, 2
-    q, kk, v = random_qkv((1, 2, gh * gw, d), seed=3)
+    q, kk, v = random_qkv((1, 2, gh * gw, d), seed=3, dtype=dtype)
     row = torch.full((2, 9, gh), -1e4)
     row[:, :, ys] = 0.0
     col = torch.full((2, 9, gw), -1e4)
     col[:, :, xs] = 0.0
-    out = run(q, kk, v, gh, gw, ph, pw, 0.25, [row, col, None], parts(2, 9, gh, gw, 5), torch.float32)
+    out = run(q, kk, v, gh, gw, ph, pw, 0.25, [row, col, None], parts(2, 9, gh, gw, 5), dtype)
     want = v[:, :, ys * gw + xs][:, :, None, :].expand_as(out.cpu())
-    assert torch.allclose(out.cpu(), want, atol=1e-6, rtol=0)
+    atol = 1e-6 if dtype == torch.float32 else 1e-2
+    assert torch.allclose(out.cpu().float(), want.float(), atol=atol, rtol=0)
 
 
 def test_bias_at_the_sd_latent_size_on_sampled_slices():
@@ -93,8 +98,8 @@ def test_bias_at_the_sd_latent_size_on_sampled_slices():
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16])
 def test_bias_with_a_column_component_on_a_4_byte_boundary(dtype):
-    """An even-width grid whose column component starts 4 bytes past an
-    8-byte boundary takes the per-element path of the biased aggregation."""
+    """A column component that starts 4 bytes past an 8-byte boundary (the
+    boundary the entry point accepts) reads correctly."""
     B, H, gh, gw, ph, pw, d = 1, 2, 16, 16, 4, 4, 32
     N, k = gh * gw, ph * pw
     q, kk, v = random_qkv((B, H, N, d), seed=5, dtype=dtype)
@@ -114,3 +119,18 @@ def test_bias_with_a_column_component_on_a_4_byte_boundary(dtype):
     ref = oracle.agent_attn_bias(f64(q), f64(kk), f64(v), gh, gw, ph, pw, 1 / math.sqrt(d),
                                  full(b1, gh, gw, ph, pw), full(b2, gh, gw, ph, pw))
     assert_close(f64(out), ref, dtype, "biased O")
+
+
+def test_bias_on_a_grid_wider_than_4096_tokens():
+    """A 2 x 4100 grid (8200 tokens, 1 x 4 agent cells, odd cell widths of
+    1025 tokens) takes the tensor-core kernels with the dense bias copies; the
+    B1 rows (8200 tokens) and B2 rows (4 agents, padded to 16) end mid-tile."""
+    B, H, gh, gw, ph, pw, d = 1, 2, 2, 4100, 1, 4, 16
+    N = gh * gw
+    q, kk, v = random_qkv((B, H, N, d), seed=9, dtype=torch.bfloat16)
+    b1 = parts(H, ph * pw, gh, gw, 41)
+    b2 = parts(H, ph * pw, gh, gw, 42)
+    out = run(q, kk, v, gh, gw, ph, pw, 1 / math.sqrt(d), b1, b2, torch.bfloat16)
+    ref = oracle.agent_attn_bias(f64(q), f64(kk), f64(v), gh, gw, ph, pw, 1 / math.sqrt(d),
+                                 full(b1, gh, gw, ph, pw), full(b2, gh, gw, ph, pw))
+    assert_close(f64(out), ref, torch.bfloat16, "biased O")
