@@ -835,12 +835,23 @@ __global__ void expand_agents_f32_kernel(const T* __restrict__ ag, float* __rest
 // row's softmax max and sum: the broadcast-stage gradients, the
 // aggregation-stage gradients, then dQ with the pooling adjoint and the
 // agents' own gradient.
+// The tensor-core pass over K that gives the key kernel its exponentials:
+// the bf16 agents and V_A the broadcast reads, and the SM count it sizes its
+// grid by.
+struct KeyExpLaunch {
+  const void* agents;
+  long long agents_bstride;
+  const void* va_low;
+  int sms;
+};
+
 template <typename T>
 int backward_gradients(const Problem& p, const void* q, const void* k, const void* v,
                        const void* agents, const void* dout, void* dq, void* dk, void* dv,
                        float* dagents, float* a32, float* va32, float* ml, float* dva, float* da,
                        float* dqa, float* ej, cudaStream_t st,
-                       const tc::BcStats* qstats = nullptr) {
+                       const tc::BcStats* qstats = nullptr,
+                       const KeyExpLaunch* kexp = nullptr) {
   const long long BH = p.BH();
   const size_t kd = (size_t)p.k * p.d;
   const size_t nd = (size_t)p.N * p.d;
@@ -893,6 +904,18 @@ int backward_gradients(const Problem& p, const void* q, const void* k, const voi
   }
   g.st_m = g.st_l = g.st_D = nullptr;
   g.st_p = nullptr;
+  if (qstats && kexp) {
+    // the broadcast over K in column mode: 2^(s - m_j) for every (key, agent
+    // j), m_j the aggregation's max, into the buffer the query kernel has
+    // finished with
+    const tc::BcStats ks{nullptr, nullptr, nullptr, nullptr, qstats->p, ml};
+    cudaError_t e = tc_launch_broadcast(k, kexp->agents, kexp->agents_bstride, kexp->va_low,
+                                        const_cast<void*>(k), p.B, p.H, p.N, p.d, p.k,
+                                        p.scale * kLog2e, kexp->sms, st, false, nullptr, &ks);
+    if (e != cudaSuccess) return cuda_fail(e, "agent_broadcast (backward key exponentials) launch");
+    g.st_p = reinterpret_cast<const uint32_t*>(qstats->p);
+    g.st_kpad = (p.k + 15) / 16 * 16;
+  }
   g.x = k;
   g.y = v;
   g.dva = dva;
@@ -999,8 +1022,9 @@ int backward_impl(const Problem& p, const void* q, const void* k, const void* v,
       e = tc_launch_broadcast(q, ag, ag_bstride, va_low, const_cast<void*>(q), p.B, p.H, p.N, p.d,
                               p.k, p.scale * kLog2e, sms, st, false, nullptr, &qs);
       if (e != cudaSuccess) return cuda_fail(e, "agent_broadcast (backward statistics) launch");
+      const KeyExpLaunch kx{ag, ag_bstride, va_low, sms};
       return backward_gradients<T>(p, q, k, v, agents, dout, dq, dk, dv, dagents, a32, va32, ml,
-                                   dva, da, dqa, ej, st, &qs);
+                                   dva, da, dqa, ej, st, &qs, &kx);
     }
     // 1. fp32 agents
     if (agents == nullptr) {

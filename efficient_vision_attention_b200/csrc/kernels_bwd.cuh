@@ -13,7 +13,9 @@
 //                     P2_ij dO_i (-> dV_A_j) and s dS2_ij Q_i (-> dA_j) into
 //                     global fp32 accumulators.
 //   bwd_key_kernel    per key row n: P1_jn from the aggregation's stored row
-//                     max and sum, dP1_jn = dV_A_j . V_n, dS1 = P1 (dP1 - E_j)
+//                     max and sum (the exponentials from a tensor-core pass
+//                     over K when given), dP1_jn = dV_A_j . V_n, dS1 = P1
+//                     (dP1 - E_j)
 //                     with E_j = dV_A_j . V_A_j; writes dK_n = s sum_j dS1_jn
 //                     A_j and dV_n = sum_j P1_jn dV_A_j and adds s dS1_jn K_n
 //                     into dA_j.
@@ -46,8 +48,9 @@ struct BwdArgs {
   const float* st_m;    // query kernel, or null: each query's score max (log2 units),
   const float* st_l;    //   sum of 2^(s - m) and D = dO . O [BH][N], computed
   const float* st_D;    //   beforehand (then the first sweep is skipped)
-  const uint32_t* st_p; // query kernel, or null: 2^(s - m) as bf16 pairs, [BH][N][st_kpad]
-  int st_kpad;          //   bf16 (even; columns >= n_agents hold 0), given with st_m
+  const uint32_t* st_p; // or null: 2^(s - m) as bf16 pairs, [BH][N][st_kpad] bf16 (even;
+  int st_kpad;          //   columns >= n_agents hold 0): the query kernel's with st_m (m
+                        //   the query's max), the key kernel's with m the agent's max
   float* dq;            // query kernel: dQ [BH][N][d] fp32
   float* dva_acc;       // query kernel: += dV_A
   float* da_acc;        // both: += dA
@@ -416,8 +419,10 @@ __global__ void __launch_bounds__(kBwdThreads, kRegAcc ? 3 : 1) bwd_query_kernel
   }
 }
 
+// Three CTAs per SM (the shared-memory limit too): the given-exponential path
+// would otherwise take 110 registers and two.
 template <typename T>
-__global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
+__global__ void __launch_bounds__(kBwdThreads, 3) bwd_key_kernel(BwdArgs p) {
   extern __shared__ float sm[];
   const int d = p.d, dp = bwd_row_stride(d);
   float* s_x = sm;                                   // K rows
@@ -448,8 +453,23 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
     s_dk[e] = 0.f;
     s_dv[e] = 0.f;
   }
+  // With the exponentials given (the broadcast run over K, each agent's max
+  // subtracted), P1 = 2^(s - m_j) / l_j comes from them (thread items = 4
+  // bf16 pairs: rows e / 16, agents 2 (e % 16), e = tid + 256 i) and the
+  // score dot products are skipped.
+  const bool p_given = p.st_p != nullptr;
+  const uint32_t* Pw = p_given ? p.st_p + (bh * n_rows + r0) * (long long)(p.st_kpad / 2) : nullptr;
   for (int j0 = 0; j0 < K; j0 += kBwdCols) {
     const int valid = min(kBwdCols, K - j0);
+    uint32_t pw[4] = {0u, 0u, 0u, 0u};
+    if (p_given) {                     // issued before the dot products hide the latency
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = tid + kBwdThreads * i, r = e >> 4, j = 2 * (e & 15);
+        if (j < valid && r0 + r < n_rows)
+          pw[i] = __ldg(Pw + (long long)r * (p.st_kpad / 2) + ((j0 + j) >> 1));
+      }
+    }
     __syncthreads();
     bwd_load_agents(s_a, A, j0, K, d, dp);
     bwd_load_agents(s_dva, DVA, j0, K, d, dp);
@@ -461,18 +481,32 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_key_kernel(BwdArgs p) {
       s_jl[j] = j < valid ? ML[(long long)(j0 + j) * 2 + 1] : 1.f;
     }
     __syncthreads();
-    bwd_dots(s_t, s_x, s_a, d, dp, p.scale_log2);
+    if (!p_given) bwd_dots(s_t, s_x, s_a, d, dp, p.scale_log2);
     bwd_dots(s_g, s_y, s_dva, d, dp, 1.f);
     __syncthreads();
-    for (int e = tid; e < kBwdRows * kBwdCols; e += kBwdThreads) {
-      const int r = e / kBwdCols, j = e - r * kBwdCols;
-      float pr = 0.f, ds = 0.f;
-      if (j < valid && r0 + r < n_rows) {
-        pr = exp2f(s_t[r * kBwdTStride + j] - s_jm[j]) / s_jl[j];
-        ds = pr * (s_g[r * kBwdTStride + j] - s_je[j]);
+    if (p_given) {
+      // padding agents (j >= valid) have l = 1, E = 0 and zero words
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = tid + kBwdThreads * i, r = e >> 4, j = 2 * (e & 15);
+        const float2 g2 = *reinterpret_cast<const float2*>(s_g + r * kBwdTStride + j);
+        const float p0 = __uint_as_float(pw[i] << 16) / s_jl[j];             // bf16 -> fp32
+        const float p1 = __uint_as_float(pw[i] & 0xffff0000u) / s_jl[j + 1];
+        *reinterpret_cast<float2*>(s_t + r * kBwdTStride + j) = make_float2(p0, p1);
+        *reinterpret_cast<float2*>(s_g + r * kBwdTStride + j) =
+            make_float2(p0 * (g2.x - s_je[j]), p1 * (g2.y - s_je[j + 1]));
       }
-      s_t[r * kBwdTStride + j] = pr;
-      s_g[r * kBwdTStride + j] = ds;
+    } else {
+      for (int e = tid; e < kBwdRows * kBwdCols; e += kBwdThreads) {
+        const int r = e / kBwdCols, j = e - r * kBwdCols;
+        float pr = 0.f, ds = 0.f;
+        if (j < valid && r0 + r < n_rows) {
+          pr = exp2f(s_t[r * kBwdTStride + j] - s_jm[j]) / s_jl[j];
+          ds = pr * (s_g[r * kBwdTStride + j] - s_je[j]);
+        }
+        s_t[r * kBwdTStride + j] = pr;
+        s_g[r * kBwdTStride + j] = ds;
+      }
     }
     __syncthreads();
     bwd_rows_acc(s_dk, s_g, s_a, d, dp, valid, p.scale);        // dK_r += s sum_j dS1 A_j

@@ -99,6 +99,11 @@ struct BcStats {
   float* l;
   float* D;
   __nv_bfloat16* p;          // [BH][N][kpad]: 2^(s - m) as bf16 (not normalised)
+  // Column mode (the key side: the broadcast run over K): non-null col_ml
+  // [BH][k][2] holds each agent's aggregation max (log2 units) and sum; the
+  // pass then stores 2^(s - m_agent) for every (key, agent) into p and
+  // nothing else (dout, m, l, D unused).
+  const float* col_ml;
 };
 
 struct BcParams {
@@ -746,11 +751,35 @@ __device__ __forceinline__ void bc_store_p(uint32_t* g0, uint32_t* g1, int c, in
   }
 }
 
+// Column mode (colm non-null, kStoreP): the exponent subtracts the column's
+// max colm[2 a] (log2 units) instead of the row's: v = S*c_scale - m_a.
+template <int R>
+__device__ __forceinline__ void bc_col_shift(float (&v)[4 * R], int c, int j4, int k,
+                                             float c_scale, const float* colm) {
+#pragma unroll
+  for (int g = 0; g < R; ++g) {
+    const int a = c + 8 * g + 2 * j4;
+    const float m0 = a < k ? __ldg(colm + 2 * a) : 0.f;
+    const float m1 = a + 1 < k ? __ldg(colm + 2 * a + 2) : 0.f;
+    v[4 * g] = fmaf(v[4 * g], c_scale, -m0);
+    v[4 * g + 1] = fmaf(v[4 * g + 1], c_scale, -m1);
+    v[4 * g + 2] = fmaf(v[4 * g + 2], c_scale, -m0);
+    v[4 * g + 3] = fmaf(v[4 * g + 3], c_scale, -m1);
+  }
+}
+
 template <bool kStoreP = false>
 __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int j4, bool wide,
                                             float c_scale, float neg_m0, float neg_m1, float& l0,
                                             float& l1, bool run, uint64_t* chunk_bar,
-                                            uint32_t* g0 = nullptr, uint32_t* g1 = nullptr) {
+                                            uint32_t* g0 = nullptr, uint32_t* g1 = nullptr,
+                                            const float* colm = nullptr) {
+  const bool col_mode = kStoreP && colm != nullptr;
+  const float cs_col = c_scale;            // column mode: S*c - m_a, then exp2 as is
+  if (col_mode) {
+    c_scale = 1.f;
+    neg_m0 = neg_m1 = 0.f;
+  }
   int c = 0, ch = 0;
 #pragma unroll 1
   for (; c + 64 <= kpad; c += 64, ++ch) {
@@ -759,6 +788,7 @@ __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int
       uint32_t pk[16];
       slab_ld64(s_col + c, v);
       if (c + 64 > k) slab_mask<8>(v, c, j4, k);
+      if (col_mode) bc_col_shift<8>(v, c, j4, k, cs_col, colm);
       slab_exp<8>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
       slab_st_p32(s_col + bc_p_col(ch, wide), pk);
       bc_store_p<8, kStoreP>(g0, g1, c, j4, pk);
@@ -774,6 +804,7 @@ __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int
         uint32_t pk[8];
         slab_ld32(s_col + c, v);
         if (c + 32 > k) slab_mask<4>(v, c, j4, k);
+        if (col_mode) bc_col_shift<4>(v, c, j4, k, cs_col, colm);
         slab_exp<4>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
         slab_st_p16(pc, pk);
         bc_store_p<4, kStoreP>(g0, g1, c, j4, pk);
@@ -784,6 +815,7 @@ __device__ __forceinline__ void bc_slab_exp(uint32_t s_col, int k, int kpad, int
         uint32_t pk[4];
         slab_ld16(s_col + c16, v);
         if (c16 + 16 > k) slab_mask<2>(v, c16, j4, k);
+        if (col_mode) bc_col_shift<2>(v, c16, j4, k, cs_col, colm);
         slab_exp<2>(v, c_scale, neg_m0, neg_m1, pk, l0, l1);
         slab_st_p8(pc + (c16 - c) / 2, pk);
         bc_store_p<2, kStoreP>(g0, g1, c16, j4, pk);
@@ -1011,7 +1043,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         if constexpr (kBias) {
           bc_slab_bias_max(s_col, p.k, kpad, j4, p.c, rb, t0, t1, bw0, bw1);
-        } else {
+        } else if (!(kStats && p.stats.col_ml)) {   // column mode: no row max
           bc_slab_max(s_col, p.k, kpad, j4, t0, t1);
         }
         t0 = row4_max(t0) * ce;
@@ -1024,8 +1056,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t* g1 = q0 + r1 < p.N ? reinterpret_cast<uint32_t*>(
                                            p.stats.p + (bh * p.N + q0 + r1) * (long long)kpad)
                                      : nullptr;
+        const float* colm = p.stats.col_ml ? p.stats.col_ml + bh * p.k * 2 : nullptr;
         bc_slab_exp<true>(s_col, p.k, kpad, j4, wide, ce, -t0, -t1, l0, l1, ok, bars->p_chunk[g],
-                          g0, g1);
+                          g0, g1, colm);
       } else {
         bc_slab_exp(s_col, p.k, kpad, j4, wide, ce, -t0, -t1, l0, l1, ok, bars->p_chunk[g]);
       }
@@ -1046,6 +1079,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       warp_arrive(&bars->o_free[g]);           // the buffer may take the next S now
       if constexpr (kStats) {
+        if (p.stats.col_ml) continue;          // column mode: the exponentials only
         // D = dO . O over the row's columns (this thread's pairs, then the 4
         // threads of the row), and the row's max and sum, by its first thread
         const bool in0 = q0 + r0 < p.N, in1 = q0 + r1 < p.N;
@@ -1308,7 +1342,7 @@ inline cudaError_t tc_launch_broadcast(const void* q, const void* agents, long l
   p.total_tiles = BH * p.tiles_per_slice;
   p.ctas = (int)(p.total_tiles < sm_count ? p.total_tiles : sm_count);
   p.bias = bias ? *bias : BiasParams{nullptr, 0};
-  p.stats = with_stats ? *stats : BcStats{nullptr, nullptr, nullptr, nullptr};
+  p.stats = with_stats ? *stats : BcStats{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
   return launch_kernel(biased       ? agent_broadcast_tc_kernel<true>
                        : with_stats ? agent_broadcast_tc_kernel<false, true>
                                     : agent_broadcast_tc_kernel<false>,
