@@ -228,9 +228,13 @@ AA_API int agent_attn_forward_bias(const void* q, const void* k, const void* v,
  *   dagents_or_null : [B, H, k, d] fp32 output (gradient of each slice's
  *                     agents; sum over B for agents shared over the batch),
  *                     or NULL.
- * Runs on SIMT kernels with fp32 arithmetic (the forward statistics are
- * recomputed); the per-agent sums use fp32 atomic additions, so results may
- * differ from run to run at rounding level.  B*H <= 65535. */
+ * The gradient kernels are SIMT with fp32 arithmetic.  The forward statistics
+ * are recomputed; for bf16 with d <= 64 on the tensor cores, which also
+ * supply the exponentials of both softmaxes as bf16 (the values the forward
+ * pass's P V products use), so the scratch holds one [B, H, N, k rounded up
+ * to 16] bf16 array beside the fp32 accumulators.  The per-agent sums use
+ * fp32 atomic additions, so results may differ from run to run at rounding
+ * level.  B*H <= 65535. */
 AA_API int agent_attn_backward(const void* q, const void* k, const void* v,
                                const void* agents_or_null, const void* dout, void* dq, void* dk,
                                void* dv, float* dagents_or_null, int B, int H, int N, int d,

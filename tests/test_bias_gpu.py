@@ -59,16 +59,18 @@ def test_bias_matches_oracle(dtype, B, H, gh, gw, ph, pw, d, drop1, drop2):
     assert_close(f64(out), ref, dtype, "biased O")
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_bias_admitting_one_token_selects_its_value_on_gpu(dtype):
-    """B1 = -1e4 everywhere but one token: every agent's V_A is that token's
-    V row, and so is every output row (bf16: the -1e4 components sum to
-    -2e4, inside the dense copy's fp16 range)."""
+@pytest.mark.parametrize("dtype,mask", [(torch.float32, -1e4), (torch.bfloat16, -1e4),
+                                        (torch.bfloat16, -1e6)])
+def test_bias_admitting_one_token_selects_its_value_on_gpu(dtype, mask):
+    """B1 = mask everywhere but one token: every agent's V_A is that token's
+    V row, and so is every output row.  bf16 holds B1 * log2(e) in fp16: -1e4
+    components (sum -2e4) lie inside its range, -1e6 saturate at -65504 and
+    still give the admitted token all the weight."""
     gh, gw, ph, pw, d, ys, xs = 9, 7, 3, 3, 16, 4, 2
     q, kk, v = random_qkv((1, 2, gh * gw, d), seed=3, dtype=dtype)
-    row = torch.full((2, 9, gh), -1e4)
+    row = torch.full((2, 9, gh), mask)
     row[:, :, ys] = 0.0
-    col = torch.full((2, 9, gw), -1e4)
+    col = torch.full((2, 9, gw), mask)
     col[:, :, xs] = 0.0
     out = run(q, kk, v, gh, gw, ph, pw, 0.25, [row, col, None], parts(2, 9, gh, gw, 5), dtype)
     want = v[:, :, ys * gw + xs][:, :, None, :].expand_as(out.cpu())
