@@ -207,6 +207,34 @@ __device__ __forceinline__ void bwd_rows_acc_reg(float (&acc)[4][4], const float
   }
 }
 
+// out[r][c] += mul * sum_{j < valid} W[r][j] M[j][c] for d <= 64 on 4 x 4
+// register tiles (rows rq + 16 i, channels c..c+3: 8 shared reads per 64
+// FMAs, against 6 per 32 in bwd_rows_acc), added into the shared rows once
+// per chunk.
+__device__ __forceinline__ void bwd_rows_acc_tile(float* out, const float* W, const float* M,
+                                                  int d, int dp, int valid, float mul) {
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+  bwd_rows_acc_reg(acc, W, M, d, dp, valid);
+  const int nq = d >> 2;
+  const int t = threadIdx.x;
+  if (t >= 16 * nq) return;
+  const int rq = t / nq, c = 4 * (t - rq * nq);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float4* o = reinterpret_cast<float4*>(out + (rq + 16 * i) * dp + c);
+    float4 u = *o;
+    u.x += mul * acc[i][0];
+    u.y += mul * acc[i][1];
+    u.z += mul * acc[i][2];
+    u.w += mul * acc[i][3];
+    *o = u;
+  }
+}
+
 // Four consecutive floats added into global memory by one vector reduction
 // (16-byte aligned address): a quarter of the L2 atomic operations of four
 // scalar atomicAdds.
@@ -509,8 +537,13 @@ __global__ void __launch_bounds__(kBwdThreads, 3) bwd_key_kernel(BwdArgs p) {
       }
     }
     __syncthreads();
-    bwd_rows_acc(s_dk, s_g, s_a, d, dp, valid, p.scale);        // dK_r += s sum_j dS1 A_j
-    bwd_rows_acc(s_dv, s_t, s_dva, d, dp, valid, 1.f);          // dV_r += sum_j P1 dV_A_j
+    if (d <= 64) {                                              // 16 (d / 4) <= 256 threads
+      bwd_rows_acc_tile(s_dk, s_g, s_a, d, dp, valid, p.scale);   // dK_r += s sum_j dS1 A_j
+      bwd_rows_acc_tile(s_dv, s_t, s_dva, d, dp, valid, 1.f);     // dV_r += sum_j P1 dV_A_j
+    } else {
+      bwd_rows_acc(s_dk, s_g, s_a, d, dp, valid, p.scale);
+      bwd_rows_acc(s_dv, s_t, s_dva, d, dp, valid, 1.f);
+    }
     bwd_agents_acc(da, j0, s_g, s_x, d, dp, valid, p.scale);    // dA_j += s sum_r dS1 K_r
   }
   __syncthreads();
