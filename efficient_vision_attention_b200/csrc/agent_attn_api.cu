@@ -214,6 +214,7 @@ void set_bias(SimtAttendArgs& a, const Problem& p, const AgentBiasRef* b, bool t
 struct Scratch {
   size_t a_off, va_off, pu_off, pml_off, total;
   size_t b1d_off, b2d_off;   // dense fp16 copies of B1 and B2 (tensor-core bias)
+  size_t b2t_off;            // B2's tokens-contiguous copy, before its transpose
   SplitPlan plan;
   int simt_row_blocks;
   int simt_cols_per_split;
@@ -256,6 +257,9 @@ void plan_scratch(const Problem& p, int sm_count, Scratch* s) {
   s->b2d_off = off;
   if (use_tensor_cores(p) && p.b2 && p.b2->any())
     off += round256((size_t)p.H * p.N * bias_ld_b2(p) * sizeof(__half));
+  s->b2t_off = off;
+  if (use_tensor_cores(p) && p.b2 && p.b2->any())
+    off += round256((size_t)p.H * p.k * bias_ld_b1(p) * sizeof(__half));
   s->total = off;
 }
 
@@ -264,8 +268,8 @@ void plan_scratch(const Problem& p, int sm_count, Scratch* s) {
 // n = (y, x) of head h, the block term from the floor-partition cell
 // (floor(y pool_h / grid_h), floor(x pool_w / grid_w)).
 //   bias_dense_tokens_kernel: B1 [H][k][ld] (ld >= N, zero for n >= N);
-//   bias_dense_agents_kernel: B2 [H][N][ld] (ld = k rounded up to 16, zero
-//                             for a >= k).
+//   B2 [H][N][ld] (ld = k rounded up to 16, zero for a >= k): the same
+//   builder into scratch, then bias_transpose_kernel.
 // Both read the components along their token axis (coalesced) and write
 // whole rows of the dense copy.  fits32: every index product (grid side x
 // pool side, the thread count) is below 2^31, so 32-bit divisions suffice.
@@ -340,59 +344,36 @@ __global__ void __launch_bounds__(256) bias_dense_tokens_kernel(AgentBiasRef b,
   }
 }
 
-// Block per (head, 32 consecutive tokens), 256 threads: the tile [32 tokens]
-// [ld agents] is summed into shared memory with a warp's lanes on 32
-// consecutive tokens (row stride 257 floats: lane t of agent a hits bank
-// (t + a) % 32), then each warp writes whole token rows, lanes on agent pairs.
-constexpr int kBiasTileTokens = 32;
-constexpr int kBiasTileStride = 257;
-__global__ void __launch_bounds__(256) bias_dense_agents_kernel(AgentBiasRef b,
-                                                                __half* __restrict__ out, int H,
-                                                                int k, int N, int gh, int gw,
-                                                                int ph, int pw, int ld,
-                                                                bool fits32) {
-  __shared__ float tile[kBiasTileTokens * kBiasTileStride];
-  const int tiles = (N + kBiasTileTokens - 1) / kBiasTileTokens;
-  const int h = blockIdx.x / tiles;
-  const int n0 = (blockIdx.x - h * tiles) * kBiasTileTokens;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int n = n0 + tx;
-  const bool in = n < N;
-  int y = 0, x = 0;
-  long long cell = 0;
-  if (in) {
-    y = n / gw;
-    x = n - y * gw;
-    cell = floor_div((long long)y * ph, gh, fits32) * pw + floor_div((long long)x * pw, gw, fits32);
-  }
-  const long long n_cells = (long long)ph * pw;
-  // agents a = ty + 8 i (ld <= 256): the components' offsets advance by 8 rows
-  long long ro = ((long long)h * k + ty) * gh + y;
-  long long co = ((long long)h * k + ty) * gw + x;
-  long long bo = ((long long)h * k + ty) * n_cells + cell;
-  const long long sr = 8LL * gh, sc = 8LL * gw, sb = 8 * n_cells;
-#pragma unroll 8
-  for (int i = 0; i < 32; ++i) {
-    const int a = ty + 8 * i;
-    if (a < ld) {
-      float v = 0.f;
-      if (in && a < k) {
-        if (b.row) v += __ldg(b.row + ro);
-        if (b.col) v += __ldg(b.col + co);
-        if (b.block) v += __ldg(b.block + bo);
-      }
-      tile[tx * kBiasTileStride + a] = v;
-    }
-    ro += sr;
-    co += sc;
-    bo += sb;
+// B2 in the agents-contiguous layout from its tokens-contiguous copy (built
+// by bias_dense_tokens_kernel into scratch): src [H][k][lds] -> dst
+// [H][N][ldd], zero for agents k .. ldd.  Block per (64 tokens, 64 agents,
+// head), 256 threads: half2 loads along the tokens into a [64][66]-half tile
+// (33 words a row: a warp's loads hit 32 banks), half2 stores along the
+// agents.
+constexpr int kBiasT = 64;
+__global__ void __launch_bounds__(256) bias_transpose_kernel(const __half* __restrict__ src,
+                                                             __half* __restrict__ dst, int k,
+                                                             int N, int lds, int ldd) {
+  __shared__ __half2 tile[kBiasT * (kBiasT / 2 + 1)];   // [agent][token pair], 33 a row
+  constexpr int kRow = kBiasT / 2 + 1;
+  const int n0 = blockIdx.x * kBiasT, a0 = blockIdx.y * kBiasT;
+  const long long h = blockIdx.z;
+  const __half2* s2 = reinterpret_cast<const __half2*>(src);
+  for (int i = threadIdx.x; i < kBiasT * (kBiasT / 2); i += blockDim.x) {
+    const int a = i / (kBiasT / 2), pr = i - a * (kBiasT / 2);
+    const int n = n0 + 2 * pr;                          // even; n + 1 < lds when n < N
+    __half2 v = __floats2half2_rn(0.f, 0.f);
+    if (a0 + a < k && n < N) v = s2[((h * k + a0 + a) * lds + n) / 2];
+    tile[a * kRow + pr] = v;
   }
   __syncthreads();
-  for (int j = ty; j < kBiasTileTokens && n0 + j < N; j += 8) {
-    __half2* row = reinterpret_cast<__half2*>(out + ((long long)h * N + n0 + j) * ld);
-    for (int a = 2 * tx; a < ld; a += 64)
-      row[a / 2] = __floats2half2_rn(bias_logit(tile[j * kBiasTileStride + a]),
-                                     bias_logit(tile[j * kBiasTileStride + a + 1]));
+  __half2* d2 = reinterpret_cast<__half2*>(dst);
+  for (int i = threadIdx.x; i < kBiasT * (kBiasT / 2); i += blockDim.x) {
+    const int jn = i / (kBiasT / 2), q = i - jn * (kBiasT / 2);
+    const int n = n0 + jn, a = a0 + 2 * q;
+    if (n >= N || a >= ldd) continue;
+    const __half2 x = tile[(2 * q) * kRow + jn / 2], y = tile[(2 * q + 1) * kRow + jn / 2];
+    d2[((h * N + n) * ldd + a) / 2] = (jn & 1) ? __highs2half2(x, y) : __lows2half2(x, y);
   }
 }
 
@@ -507,8 +488,10 @@ int launch_simt_attend(const SimtAttendArgs& args, long long BH, cudaStream_t st
 
 std::atomic<int> g_bias_tokens_smem[kMaxDevices];
 
+// B1 (tokens_minor) straight into `out`; B2 through `tmp` (a tokens-contiguous
+// copy of H k (N rounded up to 8) halves).
 int launch_bias_dense(const Problem& p, const AgentBiasRef& b, __half* out, bool tokens_minor,
-                      cudaStream_t st) {
+                      cudaStream_t st, __half* tmp) {
   const long long lim = 0x7fffffffLL;
   bool fits32 = (long long)p.grid_h * p.pool_h <= lim && (long long)p.grid_w * p.pool_w <= lim;
   if (tokens_minor) {
@@ -519,10 +502,15 @@ int launch_bias_dense(const Problem& p, const AgentBiasRef& b, __half* out, bool
     bias_dense_tokens_kernel<<<(unsigned)(rows < 65535 ? rows : 65535), 256, smem, st>>>(
         b, out, p.H, p.k, p.N, p.grid_h, p.grid_w, p.pool_h, p.pool_w, bias_ld_b1(p), fits32);
   } else {
-    const long long blocks = (long long)p.H * ((p.N + kBiasTileTokens - 1) / kBiasTileTokens);
-    if (blocks > lim) return AA_ERR_SHAPE;
-    bias_dense_agents_kernel<<<(unsigned)blocks, 256, 0, st>>>(
-        b, out, p.H, p.k, p.N, p.grid_h, p.grid_w, p.pool_h, p.pool_w, bias_ld_b2(p), fits32);
+    // tokens-contiguous into `tmp`, then transposed into `out`
+    if (tmp == nullptr) return AA_ERR_WORKSPACE;
+    int rc = launch_bias_dense(p, b, tmp, true, st, nullptr);
+    if (rc != AA_OK) return rc;
+    const int ldd = bias_ld_b2(p);
+    const dim3 grid((unsigned)((p.N + kBiasT - 1) / kBiasT), (unsigned)((ldd + kBiasT - 1) / kBiasT),
+                    (unsigned)p.H);
+    if (p.H > 65535) return AA_ERR_SHAPE;
+    bias_transpose_kernel<<<grid, 256, 0, st>>>(tmp, out, p.k, p.N, bias_ld_b1(p), ldd);
   }
   AA_CUDA(cudaGetLastError());
   return AA_OK;
@@ -655,11 +643,13 @@ int run_forward(const Problem& p, const Scratch& s, const void* q, const void* k
     // the dense bias copies, before the pool: every later kernel of the pass
     // starts after they have completed (the pool launches without overlap)
     if (p.b1 && p.b1->any()) {
-      int rc = launch_bias_dense(p, *p.b1, reinterpret_cast<__half*>(ws + s.b1d_off), true, st);
+      int rc = launch_bias_dense(p, *p.b1, reinterpret_cast<__half*>(ws + s.b1d_off), true, st,
+                                 nullptr);
       if (rc != AA_OK) return rc;
     }
     if (p.b2 && p.b2->any()) {
-      int rc = launch_bias_dense(p, *p.b2, reinterpret_cast<__half*>(ws + s.b2d_off), false, st);
+      int rc = launch_bias_dense(p, *p.b2, reinterpret_cast<__half*>(ws + s.b2d_off), false, st,
+                                 reinterpret_cast<__half*>(ws + s.b2t_off));
       if (rc != AA_OK) return rc;
     }
   }
@@ -1316,7 +1306,7 @@ int agent_attn_stage_aggregate_static(const void* agents, long long agents_batch
   const size_t need = s.total - s.pu_off;
   if (need > (size_t)AA_STATIC_SCRATCH_BYTES) return AA_ERR_WORKSPACE;
   Scratch r = s;
-  r.a_off = r.va_off = r.b1d_off = r.b2d_off = 0;
+  r.a_off = r.va_off = r.b1d_off = r.b2d_off = r.b2t_off = 0;
   r.pml_off = s.pml_off - s.pu_off;
   r.pu_off = 0;
   r.total = need;
