@@ -347,33 +347,39 @@ __global__ void __launch_bounds__(256) bias_dense_tokens_kernel(AgentBiasRef b,
 // B2 in the agents-contiguous layout from its tokens-contiguous copy (built
 // by bias_dense_tokens_kernel into scratch): src [H][k][lds] -> dst
 // [H][N][ldd], zero for agents k .. ldd.  Block per (64 tokens, 64 agents,
-// head), 256 threads: half2 loads along the tokens into a [64][66]-half tile
-// (33 words a row: a warp's loads hit 32 banks), half2 stores along the
-// agents.
+// head), 256 threads.  Each thread loads 8 tokens of one agent as one 16-byte
+// word and scatters them into a token-major tile (rows of 66 halves, 33
+// words), then gathers 8 agents of one token as four 32-bit words (a warp's
+// reads hit 32 banks) and stores them as one 16-byte word.
 constexpr int kBiasT = 64;
+constexpr int kBiasTRow = kBiasT + 2;               // halves per tile row
 __global__ void __launch_bounds__(256) bias_transpose_kernel(const __half* __restrict__ src,
                                                              __half* __restrict__ dst, int k,
                                                              int N, int lds, int ldd) {
-  __shared__ __half2 tile[kBiasT * (kBiasT / 2 + 1)];   // [agent][token pair], 33 a row
-  constexpr int kRow = kBiasT / 2 + 1;
+  __shared__ __align__(16) __half tile[kBiasT * kBiasTRow];   // [token][agent]
   const int n0 = blockIdx.x * kBiasT, a0 = blockIdx.y * kBiasT;
   const long long h = blockIdx.z;
-  const __half2* s2 = reinterpret_cast<const __half2*>(src);
-  for (int i = threadIdx.x; i < kBiasT * (kBiasT / 2); i += blockDim.x) {
-    const int a = i / (kBiasT / 2), pr = i - a * (kBiasT / 2);
-    const int n = n0 + 2 * pr;                          // even; n + 1 < lds when n < N
-    __half2 v = __floats2half2_rn(0.f, 0.f);
-    if (a0 + a < k && n < N) v = s2[((h * k + a0 + a) * lds + n) / 2];
-    tile[a * kRow + pr] = v;
+  for (int i = threadIdx.x; i < kBiasT * (kBiasT / 8); i += blockDim.x) {
+    const int a = i / (kBiasT / 8), p = i - a * (kBiasT / 8);
+    const int n = n0 + 8 * p;                           // n < N: the 8 tokens lie in the row
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (a0 + a < k && n < N)
+      w = *reinterpret_cast<const uint4*>(src + (h * k + a0 + a) * lds + n);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      tile[(8 * p + 2 * e) * kBiasTRow + a] = __ushort_as_half((unsigned short)(u[e] & 0xffffu));
+      tile[(8 * p + 2 * e + 1) * kBiasTRow + a] = __ushort_as_half((unsigned short)(u[e] >> 16));
+    }
   }
   __syncthreads();
-  __half2* d2 = reinterpret_cast<__half2*>(dst);
-  for (int i = threadIdx.x; i < kBiasT * (kBiasT / 2); i += blockDim.x) {
-    const int jn = i / (kBiasT / 2), q = i - jn * (kBiasT / 2);
-    const int n = n0 + jn, a = a0 + 2 * q;
+  const uint32_t* t32 = reinterpret_cast<const uint32_t*>(tile);
+  for (int i = threadIdx.x; i < kBiasT * (kBiasT / 8); i += blockDim.x) {
+    const int jn = i / (kBiasT / 8), q = i - jn * (kBiasT / 8);
+    const int n = n0 + jn, a = a0 + 8 * q;
     if (n >= N || a >= ldd) continue;
-    const __half2 x = tile[(2 * q) * kRow + jn / 2], y = tile[(2 * q + 1) * kRow + jn / 2];
-    d2[((h * N + n) * ldd + a) / 2] = (jn & 1) ? __highs2half2(x, y) : __lows2half2(x, y);
+    const uint32_t* r = t32 + jn * (kBiasTRow / 2) + 4 * q;
+    *reinterpret_cast<uint4*>(dst + (h * N + n) * ldd + a) = make_uint4(r[0], r[1], r[2], r[3]);
   }
 }
 
