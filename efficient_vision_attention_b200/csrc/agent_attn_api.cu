@@ -177,10 +177,12 @@ int validate_grid(int N, int grid_h, int grid_w, int pool_h, int pool_w) {
 }
 
 bool has_bias(const Problem& p) { return (p.b1 && p.b1->any()) || (p.b2 && p.b2->any()); }
-// Shared memory of the B1 dense-copy builder: one agent row's row, column and
-// block terms and the grid's cell tables.
+// Shared memory of the dense-copy builder (it builds B1, and B2 before its
+// transpose): one agent row's row, column and block terms and the grid's cell
+// tables, the per-axis arrays padded to 4 entries.
 __host__ __device__ inline size_t bias_tokens_smem_bytes(int gh, int gw, int ph, int pw) {
-  return sizeof(float) * (2 * ((size_t)gh + gw) + (size_t)ph * pw);
+  const size_t gh4 = ((size_t)gh + 3) & ~(size_t)3, gw4 = ((size_t)gw + 3) & ~(size_t)3;
+  return sizeof(float) * (2 * (gh4 + gw4) + (size_t)ph * pw);
 }
 constexpr size_t kBiasSmemMax = 160 * 1024;
 // The tensor-core kernels take the agent bias through dense copies while the
@@ -293,27 +295,28 @@ __device__ __forceinline__ long long floor_div(long long a, int b, bool fits32) 
 // the row's components (row terms [grid_h], column terms [grid_w], block
 // terms [pool_h * pool_w]) are staged in shared memory beside the cell
 // tables (cell row offset cy * pool_w per grid row, cell column per grid
-// column), then each thread writes token pairs 512 apart, tracking (y, x)
-// by adding the stride's quotient and remainder (no division per token).
+// column); each thread then writes runs of 8 tokens as one 16-byte store.
+// With grid_w a multiple of 8 a run lies in one grid row: its column terms
+// and cell columns come as two 16-byte shared words each; otherwise each
+// token finds its (y, x) by a division.
 __global__ void __launch_bounds__(256) bias_dense_tokens_kernel(AgentBiasRef b,
                                                                 __half* __restrict__ out, int H,
                                                                 int k, int N, int gh, int gw,
                                                                 int ph, int pw, int ld,
                                                                 bool fits32) {
-  extern __shared__ float bsm[];
+  extern __shared__ __align__(16) float bsm[];
   const int n_cells = ph * pw;
-  float* s_row = bsm;
-  float* s_col = s_row + gh;
-  float* s_blk = s_col + gw;
-  int* s_cyo = reinterpret_cast<int*>(s_blk + n_cells);
-  int* s_cx = s_cyo + gh;
+  const int gh4 = (gh + 3) & ~3, gw4 = (gw + 3) & ~3;
+  float* s_row = bsm;                                   // [gh4]
+  float* s_col = s_row + gh4;                           // [gw4], 16-byte aligned
+  int* s_cx = reinterpret_cast<int*>(s_col + gw4);      // [gw4], 16-byte aligned
+  int* s_cyo = s_cx + gw4;                              // [gh4]
+  float* s_blk = reinterpret_cast<float*>(s_cyo + gh4); // [n_cells]
   const int tid = threadIdx.x;
   for (int i = tid; i < gh; i += blockDim.x)
     s_cyo[i] = (int)floor_div((long long)i * ph, gh, fits32) * pw;
   for (int i = tid; i < gw; i += blockDim.x) s_cx[i] = (int)floor_div((long long)i * pw, gw, fits32);
-  const int step = 2 * blockDim.x;           // tokens between a thread's pairs
-  const int qy = step / gw, qx = step - qy * gw;
-  const int y0 = (2 * tid) / gw, x0 = 2 * tid - y0 * gw;
+  const bool runs = (gw & 7) == 0;
   const long long rows = (long long)H * k;
   for (long long r = blockIdx.x; r < rows; r += gridDim.x) {
     __syncthreads();                         // the previous row's terms are read
@@ -322,24 +325,47 @@ __global__ void __launch_bounds__(256) bias_dense_tokens_kernel(AgentBiasRef b,
     for (int i = tid; i < n_cells; i += blockDim.x)
       s_blk[i] = b.block ? __ldg(b.block + r * n_cells + i) : 0.f;
     __syncthreads();
-    __half2* o = reinterpret_cast<__half2*>(out + r * ld);
-    int y = y0, x = x0;
-    for (int n = 2 * tid; n < ld; n += step) {
-      float v0 = 0.f, v1 = 0.f;
-      if (n < N) v0 = s_row[y] + s_col[x] + s_blk[s_cyo[y] + s_cx[x]];
-      int x1 = x + 1, y1 = y;
-      if (x1 == gw) {
-        x1 = 0;
-        ++y1;
+    for (int c0 = 8 * tid; c0 < ld; c0 += 8 * blockDim.x) {
+      float v[8];
+      if (runs) {                            // N = grid_h grid_w is a multiple of 8 too
+        if (c0 < N) {
+          const int y = c0 / gw, x = c0 - y * gw;
+          const float rw = s_row[y];
+          const int cy = s_cyo[y];
+          const float4 ca = *reinterpret_cast<const float4*>(s_col + x);
+          const float4 cb = *reinterpret_cast<const float4*>(s_col + x + 4);
+          const int4 xa = *reinterpret_cast<const int4*>(s_cx + x);
+          const int4 xb = *reinterpret_cast<const int4*>(s_cx + x + 4);
+          v[0] = rw + ca.x + s_blk[cy + xa.x];
+          v[1] = rw + ca.y + s_blk[cy + xa.y];
+          v[2] = rw + ca.z + s_blk[cy + xa.z];
+          v[3] = rw + ca.w + s_blk[cy + xa.w];
+          v[4] = rw + cb.x + s_blk[cy + xb.x];
+          v[5] = rw + cb.y + s_blk[cy + xb.y];
+          v[6] = rw + cb.z + s_blk[cy + xb.z];
+          v[7] = rw + cb.w + s_blk[cy + xb.w];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int n = c0 + e;
+          v[e] = 0.f;
+          if (n < N) {
+            const int y = n / gw, x = n - y * gw;
+            v[e] = s_row[y] + s_col[x] + s_blk[s_cyo[y] + s_cx[x]];
+          }
+        }
       }
-      if (n + 1 < N) v1 = s_row[y1] + s_col[x1] + s_blk[s_cyo[y1] + s_cx[x1]];
-      o[n / 2] = __floats2half2_rn(bias_logit(v0), bias_logit(v1));
-      x += qx;
-      y += qy;
-      if (x >= gw) {
-        x -= gw;
-        ++y;
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __half2 h2 = __floats2half2_rn(bias_logit(v[2 * e]), bias_logit(v[2 * e + 1]));
+        memcpy(&w[e], &h2, sizeof(uint32_t));
       }
+      *reinterpret_cast<uint4*>(out + r * ld + c0) = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
 }
