@@ -199,9 +199,11 @@ AA_API int agent_attn_stage_aggregate_static(const void* agents, long long agent
  * in agent_attn_forward.  bf16 problems first build a dense copy of each bias
  * (B * log2(e) as fp16: 11-bit significands, values saturated at +-65504,
  * i.e. |B| up to about 45000) and add it inside the tensor-core score tiles;
- * fp32 problems add the fp32 components on the SIMT kernels.  Scratch for the
- * dense copies (2 bytes per agent and token and head, for each of B1 and B2)
- * comes from the library's stream-ordered pool. */
+ * fp32 problems, and grids whose components do not fit the builder's shared
+ * memory (grid_h + grid_w above about 20000), add the fp32 components on the
+ * SIMT kernels.  Scratch for the dense copies (2 bytes per agent, token and
+ * head for B1; twice that for B2, built tokens-contiguous and then
+ * transposed) comes from the library's stream-ordered pool. */
 AA_API int agent_attn_forward_bias(const void* q, const void* k, const void* v,
                                    const void* agents_or_null, const float* b1_row,
                                    const float* b1_col, const float* b1_block,
