@@ -584,11 +584,31 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const float* __restrict
                                                          const float* __restrict__ da, T* dq,
                                                          int N, int d, int grid_h, int grid_w,
                                                          int pool_h, int pool_w, int pooled) {
+  // the adaptive bins' bounds along each axis, once per block (pool sides
+  // <= 256: k <= 256)
+  __shared__ int s_by[2][256], s_bx[2][256];
+  if (pooled) {
+    for (int i = threadIdx.x; i < pool_h; i += blockDim.x) {
+      s_by[0][i] = bin_start(i, grid_h, pool_h);
+      s_by[1][i] = bin_end(i, grid_h, pool_h);
+    }
+    for (int i = threadIdx.x; i < pool_w; i += blockDim.x) {
+      s_bx[0][i] = bin_start(i, grid_w, pool_w);
+      s_bx[1][i] = bin_end(i, grid_w, pool_w);
+    }
+    __syncthreads();
+  }
   const long long bh = blockIdx.y;
   const int groups = d >> 3;
   const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= (long long)N * groups) return;
-  const int n = (int)(e / groups), g = (int)(e - (long long)n * groups);
+  // 32-bit divisions when the index products fit (every grid below 46341
+  // tokens a side)
+  const bool f32 = (long long)N * groups <= 0x7fffffffLL &&
+                   (long long)grid_h * pool_h <= 0x7fffffffLL &&
+                   (long long)grid_w * pool_w <= 0x7fffffffLL;
+  const int n = f32 ? (int)e / groups : (int)(e / groups);
+  const int g = (int)(e - (long long)n * groups);
   const long long off = (bh * N + n) * (long long)d + g * 8;
   const float4 s0 = *reinterpret_cast<const float4*>(dq_acc + off);
   const float4 s1 = *reinterpret_cast<const float4*>(dq_acc + off + 4);
@@ -597,9 +617,10 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const float* __restrict
     const int y = n / grid_w, x = n - y * grid_w;
     // first and last bin holding the token along each axis, with their sizes
     int by0 = -1, by1 = -1, sy0 = 1, sy1 = 1, bx0 = -1, bx1 = -1, sx0 = 1, sx1 = 1;
-    const int cy = (int)(((long long)y * pool_h) / grid_h), cx = (int)(((long long)x * pool_w) / grid_w);
+    const int cy = f32 ? (y * pool_h) / grid_h : (int)(((long long)y * pool_h) / grid_h);
+    const int cx = f32 ? (x * pool_w) / grid_w : (int)(((long long)x * pool_w) / grid_w);
     for (int py = max(0, cy - 1); py <= min(pool_h - 1, cy + 1); ++py) {
-      const int y0 = bin_start(py, grid_h, pool_h), y1 = bin_end(py, grid_h, pool_h);
+      const int y0 = s_by[0][py], y1 = s_by[1][py];
       if (y >= y0 && y < y1) {
         if (by0 < 0) {
           by0 = py;
@@ -611,7 +632,7 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const float* __restrict
       }
     }
     for (int px = max(0, cx - 1); px <= min(pool_w - 1, cx + 1); ++px) {
-      const int x0 = bin_start(px, grid_w, pool_w), x1 = bin_end(px, grid_w, pool_w);
+      const int x0 = s_bx[0][px], x1 = s_bx[1][px];
       if (x >= x0 && x < x1) {
         if (bx0 < 0) {
           bx0 = px;
